@@ -1,0 +1,485 @@
+#!/usr/bin/env python
+"""Benchmark of the QLoRA quantized linear layer on B200.
+
+One step = the whole hot path over one batch of the 65B-shaped decoder block
+(q/k/v/o W[8192,8192], gate/up W[22016,8192], down W[8192,22016]; Student-t(5)
+weights with 0.1% x10 outliers; 2048 tokens per GPU; LoRA r=64 alpha=16):
+NF4 + Double Quantization of all 7 weights, forward of every linear, backward
+(dX, dA, dB) of every linear, and with N > 1 GPUs one NCCL all-reduce of the
+LoRA gradients (data parallel, weak scaling).
+
+Printed metric: algorithmic fwd+bwd TFLOP/s of the step (sum over ranks /
+max-over-ranks device time).  Extra keys: roofline of the dominant kernel
+(live CUDA-event times), e2e (host buffers, copies inside the timed region),
+cpu_baseline (the CPU oracle on a bounded sample), clocks, kernel launch count,
+and the small-M decode sweep in HBM GB/s.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import glob
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "QLoRA linear fwd+bwd TFLOP/s and small-M GB/s, as fraction of B200 roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+PACKED_BYTES_PER_WEIGHT = 0.5 + 1 / 64 + 4 / (64 * 256)     # codes + E4M3 constants + c2
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="block65b")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-decode", action="store_true")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def step_flops(wl, M):
+    """Algorithmic fwd+bwd flops of one step on one rank: per linear
+    fwd 2MNK + 2Mr(N+K), bwd 2MNK + 4Mr(N+K)."""
+    total = 0
+    for (N, K) in wl.linears:
+        total += 2 * M * N * K + 2 * M * wl.r * (N + K)
+        total += 2 * M * N * K + 4 * M * wl.r * (N + K)
+    return total
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampled every 200 ms while the timed region runs."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}", "--format=csv,noheader",
+                 "-lms", "200"], stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.file.flush()
+        with open(self.file.name) as f:
+            rows = [ln.strip().split(", ") for ln in f if ln.strip()]
+        os.unlink(self.file.name)
+        sm, mx, reasons, util = [], None, set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < 10:
+                continue
+            try:
+                clk = float(r[1].split()[0])
+                mx = float(r[2].split()[0])
+                u = float(r[4].split()[0])
+            except ValueError:
+                continue
+            util.append(u)
+            if u >= 50:
+                sm.append(clk)
+                for name, v in zip(names, r[6:10]):
+                    if v.strip().lower() == "active":
+                        reasons.add(name)
+        sm_med = sorted(sm)[len(sm) // 2] if sm else None
+        return {"sm_mhz": sm_med, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples_under_load": len(sm)}
+
+
+# ----------------------------------------------------------------------------- traffic from ncu
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "bit_nf4_quantized_23_b200", "csrc", "*"))):
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel_kind: str):
+    """DRAM bytes per launch recorded from an ncu capture (profiles/traffic.txt), or None
+    when the kernel sources changed since the capture."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    sha = kernel_source_sha()
+    with open(path) as f:
+        for ln in f:
+            ln = ln.split("#")[0].strip()
+            if not ln:
+                continue
+            kv = dict(part.split("=", 1) for part in ln.split())
+            if kv.get("kind") == kernel_kind and kv.get("source_sha") == sha:
+                return float(kv["bytes_per_launch"])
+    return None
+
+
+# ----------------------------------------------------------------------------- CPU oracle sample
+
+def oracle_sample(wl, rows: int = 256, reps: int = 1, w_rows: int | None = None):
+    """Time the CPU oracle on one linear of the workload (quantize all of W, or its first
+    `w_rows` rows, dequantize, forward and backward on `rows` token rows).
+    Returns (flops, seconds, description)."""
+    import numpy as np
+    import synthetic_inputs as si
+    from oracle import nf4_oracle as o
+    N, K = wl.linears[0]
+    W = si.bf16_bits(si.weight(wl, 0))
+    if w_rows is not None and w_rows < N:
+        N = w_rows
+        W = W[:N]
+        B_rows = N
+    else:
+        B_rows = N
+    X = si.bf16_bits(si.activations(wl, K, wl.M if isinstance(wl.M, int) else 16))[:rows]
+    A, B = (si.bf16_bits(t) for t in si.lora(wl, 0))
+    B = B[:B_rows]
+    dY = si.bf16_bits(si.grad_output(wl, 0, wl.M if isinstance(wl.M, int) else 16))[:rows, :N]
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        qw = o.quantize_nf4_dq(W)
+        Wh = o.dequantize(qw["codes"], qw["c1_codes"], qw["c2"], qw["mu"], N, K)
+        o.linear_forward(X, Wh, A, B, wl.alpha, wl.r)
+        o.linear_backward(X, dY, Wh, A, B, wl.alpha, wl.r)
+    dt = (time.perf_counter() - t0) / reps
+    m = X.shape[0]
+    flops = 2 * m * N * K + 2 * m * wl.r * (N + K) + 2 * m * N * K + 4 * m * wl.r * (N + K)
+    desc = (f"oracle (NumPy, fp64 GEMMs) on linear 0 of {wl.name} restricted to W[{N},{K}]: full NF4+DQ "
+            f"quantize and dequantize of that W, then fwd+bwd on {m} of the {wl.M} token rows")
+    return flops, dt, desc
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 0) for d in threadpool_info() if d.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import synthetic_inputs as si
+    wl = si.WORKLOADS[args.workload]
+    times = []
+    flops = 0
+    desc = ""
+    # about 2 minutes in all: a full W[8192,8192] sample takes ~16 s on 8 host cores
+    n_calls = args.warmup + args.steps
+    w_rows = int(max(256, min(wl.linears[0][0], wl.linears[0][0] * 120.0 / (16.0 * n_calls))) // 256 * 256)
+    for i in range(n_calls):
+        f, dt, desc = oracle_sample(wl, w_rows=w_rows)
+        if i >= args.warmup:
+            times.append(dt)
+            flops = f
+    sec = sum(times) / len(times)
+    value = flops / sec / 1e12
+    cores = blas_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": wl.description, "sample": desc},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- our arm
+
+class Linear:
+    pass
+
+
+def setup_workload(wl, rank, device):
+    import torch
+    import bit_nf4_quantized_23_b200 as q4
+    import synthetic_inputs as si
+    M = wl.M
+    xs = {}
+    lins = []
+    for i, (N, K) in enumerate(wl.linears):
+        L = Linear()
+        L.N, L.K = N, K
+        L.W = si.weight(wl, i).to(device)                        # frozen weight (replicated)
+        if K not in xs:
+            xs[K] = si.activations(wl, K, M, seed=rank).to(device)
+        L.X = xs[K]
+        L.A, L.B = (t.to(device) for t in si.lora(wl, i))
+        L.dY = si.grad_output(wl, i, M, seed=rank).to(device)
+        L.w = q4.NF4Weight.empty(N, K, device)
+        L.qws = torch.empty(q4.qlora_nf4_sizes(N, K)["workspace"], dtype=torch.uint8, device=device)
+        L.lws = torch.empty(max(16, q4.qlora_linear_workspace_size(M, N, K, wl.r)), dtype=torch.uint8,
+                            device=device)
+        L.Y = torch.empty(M, N, dtype=torch.bfloat16, device=device)
+        L.U = torch.empty(M, wl.r, dtype=torch.float32, device=device)
+        L.dX = torch.empty(M, K, dtype=torch.bfloat16, device=device)
+        lins.append(L)
+    n_grad = sum(wl.r * L.K + L.N * wl.r for L in lins)
+    grads = torch.empty(n_grad, dtype=torch.float32, device=device)
+    off = 0
+    for L in lins:
+        L.dA = grads[off:off + wl.r * L.K].view(wl.r, L.K)
+        off += wl.r * L.K
+        L.dB = grads[off:off + L.N * wl.r].view(L.N, wl.r)
+        off += L.N * wl.r
+    return lins, grads
+
+
+def make_step(wl, lins, grads, world):
+    import torch
+    import bit_nf4_quantized_23_b200 as q4
+
+    def step():
+        for L in lins:
+            q4.qlora_quantize_nf4_dq(L.W, out=L.w, workspace=L.qws)
+        for L in lins:
+            q4.qlora_linear_fwd(L.w, L.X, L.A, L.B, wl.r, wl.alpha, out=L.Y, U_out=L.U, workspace=L.lws)
+        for L in reversed(lins):
+            q4.qlora_linear_bwd(L.w, L.X, L.dY, L.A, L.B, wl.r, wl.alpha, U_saved=L.U, dX=L.dX,
+                                dA=L.dA, dB=L.dB, workspace=L.lws)
+        if world > 1:
+            torch.distributed.all_reduce(grads)
+    return step
+
+
+def timed_steps(step, steps, flush, stream):
+    """Device time of `steps` steps (L2 flushed before each, outside the timing)."""
+    import torch
+    total = 0.0
+    for _ in range(steps):
+        flush()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        step()
+        b.record(stream)
+        b.synchronize()
+        total += a.elapsed_time(b)
+    return total
+
+
+def decode_sweep(device, peaks):
+    """Small-M forward on the decode shapes: HBM GB/s over packed NF4 + DQ constant bytes."""
+    import torch
+    import bit_nf4_quantized_23_b200 as q4
+    import synthetic_inputs as si
+    wl = si.WORKLOADS["decode"]
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    out = {}
+    for i, (N, K) in enumerate(wl.linears):
+        W = si.weight(wl, i).to(device)
+        A, B = (t.to(device) for t in si.lora(wl, i))
+        wbytes = PACKED_BYTES_PER_WEIGHT * N * K
+        copies = max(2, int(3 * l2 // wbytes) + 1)
+        ws = [q4.qlora_quantize_nf4_dq(W) for _ in range(copies)]
+        del W
+        for M in wl.M:
+            X = si.activations(wl, K, M).to(device)
+            Y = torch.empty(M, N, dtype=torch.bfloat16, device=device)
+            lws = torch.empty(max(16, q4.qlora_linear_workspace_size(M, N, K, wl.r)), dtype=torch.uint8,
+                              device=device)
+            for j in range(3):
+                q4.qlora_linear_fwd(ws[j % copies], X, A, B, wl.r, wl.alpha, out=Y, save_U=False, workspace=lws)
+            reps = 4 * copies
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            a.record()
+            for j in range(reps):
+                q4.qlora_linear_fwd(ws[j % copies], X, A, B, wl.r, wl.alpha, out=Y, save_U=False, workspace=lws)
+            b.record()
+            b.synchronize()
+            ms = a.elapsed_time(b) / reps
+            gbs = wbytes / (ms * 1e-3) / 1e9
+            out[f"W[{N},{K}] M={M}"] = {"us_per_call": round(ms * 1e3, 2), "GB/s": round(gbs, 1),
+                                        "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 3)}
+        del ws
+        torch.cuda.empty_cache()
+    return out
+
+
+def run_ours(args):
+    import torch
+    import bit_nf4_quantized_23_b200 as q4
+    import synthetic_inputs as si
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    q4._lib.lib()
+    peaks, peak_kind = load_peaks()
+    wl = si.WORKLOADS[args.workload]
+    lins, grads = setup_workload(wl, rank, device)
+    step = make_step(wl, lins, grads, world)
+    stream = torch.cuda.current_stream()
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    flush = lambda: flush_buf.zero_()
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    assert q4.qlora_read_device_errors(clear=True) == 0
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    barrier()
+    clocks.start()
+    q4.qlora_timing_read("fwd_main", reset=True)
+    q4.qlora_timing_enable(True)
+    launches0 = q4.qlora_launch_count()
+    ms_total = timed_steps(step, args.steps, flush, stream)
+    launches = q4.qlora_launch_count() - launches0
+    barrier()
+    q4.qlora_timing_enable(False)
+    clk = clocks.stop()
+    if world > 1:
+        t = torch.tensor([ms_total], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    flops_rank = step_flops(wl, wl.M)
+    value = flops_rank * world / (ms_step * 1e-3) / 1e12
+
+    # dominant kernel, measured live over the timed region
+    kinds = {k: q4.qlora_timing_read(k) for k in ("quantize", "fwd_main", "dx_main", "lora")}
+    fwd_flops = sum(2 * wl.M * L.N * L.K + 2 * wl.M * L.N * wl.r for L in lins)
+    dx_flops = sum(2 * wl.M * L.N * L.K + 2 * wl.M * L.K * wl.r for L in lins)
+    cand = {"fwd_main": fwd_flops, "dx_main": dx_flops}
+    dom = max(cand, key=lambda k: kinds[k][1])
+    n_l, ms_l = kinds[dom]
+    per_launch_flops = cand[dom] / len(lins)
+    achieved = per_launch_flops / (ms_l / n_l * 1e-3) / 1e12 if n_l else None
+    peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": (achieved / peak) if achieved else None,
+                "peak_source": f"{peak_kind} bf16 sustained (MEASURED_PEAKS.json)" if peak_kind == "measured"
+                else "fallback",
+                "traffic": recorded_traffic(dom),
+                "per_launch_flops": per_launch_flops, "launches": n_l,
+                "avg_launch_ms": ms_l / n_l if n_l else None}
+    breakdown = {k: {"launches": v[0], "ms_per_step": v[1] / args.steps} for k, v in kinds.items()}
+
+    # end to end through the public API with host buffers (pinned), copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        host = []
+        for L in lins:
+            for name in ("W", "X", "A", "B", "dY"):
+                t = getattr(L, name)
+                if not any(t is h[0] for h in host):
+                    host.append((t, t.cpu().pin_memory()))
+        grads_host = torch.empty(grads.numel(), dtype=torch.float32).pin_memory()
+        h2d = sum(h.numel() * h.element_size() for _, h in host)
+        d2h = grads.numel() * 4
+
+        def e2e_step():
+            for dev_t, h in host:
+                dev_t.copy_(h, non_blocking=True)
+            step()
+            grads_host.copy_(grads, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        barrier()
+        ms_e2e = timed_steps(e2e_step, max(1, min(args.steps, 5)), flush, stream) / max(1, min(args.steps, 5))
+        if world > 1:
+            t = torch.tensor([ms_e2e], device=device, dtype=torch.float64)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        e2e = {"value": flops_rank * world / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
+
+    decode = None
+    if rank == 0 and not args.no_decode:
+        del lins
+        torch.cuda.empty_cache()
+        decode = decode_sweep(device, peaks)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        f, dt, desc = oracle_sample(wl)
+        cpu = {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": desc, "seconds": dt}
+
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.description, "tokens_per_gpu": wl.M, "global_batch_tokens": wl.M * world,
+                       "r": wl.r, "alpha": wl.alpha, "parallelism": f"dp{world}",
+                       "l2": "flushed before every timed step (256 MiB write, outside the timed region)",
+                       "step": "quantize all 7 weights + fwd + bwd of all 7 linears"
+                               + (" + NCCL all-reduce of dA/dB" if world > 1 else "")},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+            "clocks": clk, "kernels": breakdown, "decode_small_m": decode}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

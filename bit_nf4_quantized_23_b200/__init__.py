@@ -1,0 +1,209 @@
+"""B200 (sm_100a) QLoRA quantized linear layer: NF4 + Double Quantization, dequantization,
+and the LoRA-augmented forward/backward through the frozen dequantized weight.
+
+The Python functions below carry the names of the C entry points of libqlora.so
+(include/qlora.h).  They only marshal arguments: they allocate outputs with
+torch (device memory), pass raw pointers and the current CUDA stream, and check
+the returned status.  Every step of the computation runs in the library's CUDA
+kernels; there is no CPU or PyTorch fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+from ctypes import byref, c_float, c_size_t, c_uint32
+from dataclasses import dataclass
+
+import torch
+
+from ._lib import (QLORA_DTYPE_BF16, QLORA_DTYPE_F32, TIMER_KINDS, NF4WeightC, QloraError, check, lib)
+
+__all__ = [
+    "NF4Weight", "QloraError", "qlora_nf4_sizes", "qlora_nf4_codebook", "qlora_quantize_nf4_dq",
+    "qlora_dequantize", "qlora_linear_workspace_size", "qlora_linear_fwd", "qlora_linear_bwd",
+    "qlora_read_device_errors", "qlora_launch_count", "qlora_timing_enable", "qlora_timing_read",
+]
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t: torch.Tensor, dtype, name: str, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _dtype_code(dtype) -> int:
+    if dtype == torch.bfloat16:
+        return QLORA_DTYPE_BF16
+    if dtype == torch.float32:
+        return QLORA_DTYPE_F32
+    raise TypeError("output dtype must be torch.bfloat16 or torch.float32")
+
+
+@dataclass
+class NF4Weight:
+    """The four stored buffers of an NF4 + DQ weight (device tensors) and its shape."""
+    codes: torch.Tensor      # uint8 [N*K/2]
+    c1_codes: torch.Tensor   # uint8 [N*K/64]  (FP8 E4M3 bit patterns)
+    c2: torch.Tensor         # fp32 [ceil(N*K/64/256)]
+    mu: torch.Tensor         # fp32 [1]
+    N: int
+    K: int
+
+    def c_struct(self) -> NF4WeightC:
+        return NF4WeightC(self.codes.data_ptr(), self.c1_codes.data_ptr(), self.c2.data_ptr(),
+                          self.mu.data_ptr(), self.N, self.K, 64, 256)
+
+    @staticmethod
+    def empty(N: int, K: int, device="cuda") -> "NF4Weight":
+        s = qlora_nf4_sizes(N, K)
+        return NF4Weight(torch.empty(s["codes"], dtype=torch.uint8, device=device),
+                         torch.empty(s["c1_codes"], dtype=torch.uint8, device=device),
+                         torch.empty(s["c2"] // 4, dtype=torch.float32, device=device),
+                         torch.empty(1, dtype=torch.float32, device=device), N, K)
+
+
+def qlora_nf4_sizes(N: int, K: int, blocksize: int = 64, blocksize2: int = 256) -> dict:
+    a, b, c, d = c_size_t(), c_size_t(), c_size_t(), c_size_t()
+    check(lib().qlora_nf4_sizes(N, K, blocksize, blocksize2, byref(a), byref(b), byref(c), byref(d)),
+          "qlora_nf4_sizes")
+    return {"codes": a.value, "c1_codes": b.value, "c2": c.value, "workspace": d.value}
+
+
+def qlora_nf4_codebook():
+    """(values[16], thresholds[15]) of the library, as Python float lists."""
+    v = (c_float * 16)()
+    t = (c_float * 15)()
+    check(lib().qlora_nf4_codebook(v, t), "qlora_nf4_codebook")
+    return list(v), list(t)
+
+
+def qlora_quantize_nf4_dq(W: torch.Tensor, blocksize: int = 64, blocksize2: int = 256,
+                          out: NF4Weight | None = None, workspace: torch.Tensor | None = None,
+                          stream=None) -> NF4Weight:
+    _need(W, torch.bfloat16, "W")
+    if W.dim() != 2:
+        raise ValueError("W must be 2-D [N, K]")
+    N, K = W.shape
+    sizes = qlora_nf4_sizes(N, K, blocksize, blocksize2)
+    if out is None:
+        out = NF4Weight.empty(N, K, W.device)
+    if workspace is None:
+        workspace = torch.empty(sizes["workspace"], dtype=torch.uint8, device=W.device)
+    ws = out.c_struct()
+    check(lib().qlora_quantize_nf4_dq(_ptr(W), N, K, blocksize, blocksize2, byref(ws), _ptr(workspace),
+                                      workspace.numel(), _stream(stream)), "qlora_quantize_nf4_dq")
+    return out
+
+
+def qlora_dequantize(w: NF4Weight, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    if out is None:
+        out = torch.empty(w.N, w.K, dtype=torch.bfloat16, device=w.codes.device)
+    _need(out, torch.bfloat16, "out", (w.N, w.K))
+    ws = w.c_struct()
+    check(lib().qlora_dequantize(byref(ws), _ptr(out), _stream(stream)), "qlora_dequantize")
+    return out
+
+
+def qlora_linear_workspace_size(M: int, N: int, K: int, r: int) -> int:
+    n = c_size_t()
+    check(lib().qlora_linear_workspace_size(M, N, K, r, byref(n)), "qlora_linear_workspace_size")
+    return n.value
+
+
+def _workspace(M, N, K, r, device, workspace):
+    need = qlora_linear_workspace_size(M, N, K, r)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=device)
+    return workspace
+
+
+def qlora_linear_fwd(w: NF4Weight, X: torch.Tensor, A: torch.Tensor, B: torch.Tensor, r: int,
+                     alpha: float, y_dtype=torch.bfloat16, save_U: bool = True,
+                     out: torch.Tensor | None = None, U_out: torch.Tensor | None = None,
+                     workspace: torch.Tensor | None = None, stream=None):
+    """Y = X W_hat^T + (alpha/r) (X A^T) B^T.  Returns (Y, U) with U fp32 [M,r] (or None)."""
+    M = X.shape[0]
+    _need(X, torch.bfloat16, "X", (M, w.K))
+    _need(A, torch.bfloat16, "A", (r, w.K))
+    _need(B, torch.bfloat16, "B", (w.N, r))
+    if out is None:
+        out = torch.empty(M, w.N, dtype=y_dtype, device=X.device)
+    _need(out, y_dtype, "Y", (M, w.N))
+    if save_U and U_out is None:
+        U_out = torch.empty(M, r, dtype=torch.float32, device=X.device)
+    if U_out is not None:
+        _need(U_out, torch.float32, "U", (M, r))
+    workspace = _workspace(M, w.N, w.K, r, X.device, workspace)
+    ws = w.c_struct()
+    check(lib().qlora_linear_fwd(byref(ws), _ptr(X), M, _ptr(A), _ptr(B), r, c_float(alpha), _ptr(out),
+                                 _dtype_code(y_dtype), _ptr(U_out), _ptr(workspace), workspace.numel(),
+                                 _stream(stream)), "qlora_linear_fwd")
+    return out, U_out
+
+
+def qlora_linear_bwd(w: NF4Weight, X: torch.Tensor, dY: torch.Tensor, A: torch.Tensor, B: torch.Tensor,
+                     r: int, alpha: float, U_saved: torch.Tensor | None = None, need_dX: bool = True,
+                     dx_dtype=torch.bfloat16, dX: torch.Tensor | None = None,
+                     dA: torch.Tensor | None = None, dB: torch.Tensor | None = None,
+                     workspace: torch.Tensor | None = None, stream=None):
+    """(dX, dA, dB) of <dY, Y> through the frozen W_hat.  dX is None when need_dX is False."""
+    M = X.shape[0]
+    _need(X, torch.bfloat16, "X", (M, w.K))
+    _need(dY, torch.bfloat16, "dY", (M, w.N))
+    _need(A, torch.bfloat16, "A", (r, w.K))
+    _need(B, torch.bfloat16, "B", (w.N, r))
+    if U_saved is not None:
+        _need(U_saved, torch.float32, "U_saved", (M, r))
+    if need_dX and dX is None:
+        dX = torch.empty(M, w.K, dtype=dx_dtype, device=X.device)
+    if dX is not None:
+        _need(dX, dx_dtype, "dX", (M, w.K))
+    if dA is None:
+        dA = torch.empty(r, w.K, dtype=torch.float32, device=X.device)
+    if dB is None:
+        dB = torch.empty(w.N, r, dtype=torch.float32, device=X.device)
+    _need(dA, torch.float32, "dA", (r, w.K))
+    _need(dB, torch.float32, "dB", (w.N, r))
+    workspace = _workspace(M, w.N, w.K, r, X.device, workspace)
+    ws = w.c_struct()
+    check(lib().qlora_linear_bwd(byref(ws), _ptr(X), _ptr(dY), M, _ptr(A), _ptr(B), r, c_float(alpha),
+                                 _ptr(U_saved), _ptr(dX), _dtype_code(dx_dtype), _ptr(dA), _ptr(dB),
+                                 _ptr(workspace), workspace.numel(), _stream(stream)), "qlora_linear_bwd")
+    return dX, dA, dB
+
+
+def qlora_read_device_errors(clear: bool = True, stream=None) -> int:
+    """Synchronize and return the device error flags (1: timeout, 2: non-finite weight)."""
+    f = c_uint32()
+    lib().qlora_read_device_errors(_stream(stream), 1 if clear else 0, byref(f))
+    return f.value
+
+
+def qlora_launch_count() -> int:
+    return int(lib().qlora_launch_count())
+
+
+def qlora_timing_enable(on: bool = True) -> None:
+    check(lib().qlora_timing_enable(1 if on else 0), "qlora_timing_enable")
+
+
+def qlora_timing_read(kind: str, reset: bool = False):
+    """(timed units, total device ms) recorded for one kind since the last reset."""
+    n = ctypes.c_uint64()
+    ms = ctypes.c_double()
+    check(lib().qlora_timing_read(TIMER_KINDS[kind], byref(n), byref(ms), 1 if reset else 0),
+          "qlora_timing_read")
+    return int(n.value), float(ms.value)

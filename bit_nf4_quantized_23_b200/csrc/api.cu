@@ -1,0 +1,297 @@
+// The C ABI of libqlora.so (declared in include/qlora.h): argument validation
+// on the host, then the kernel launches of each operation.
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "qlora_internal.cuh"
+#include "gemm_simt.cuh"
+#include "timing.cuh"
+
+namespace qlora {
+
+size_t quantize_workspace_bytes(int64_t nb1);
+qlora_status launch_quantize(const void* W, int64_t N, int64_t K, const qlora_nf4_weight* out,
+                             void* workspace, cudaStream_t stream);
+qlora_status launch_dequantize(const qlora_nf4_weight* w, void* W_out, cudaStream_t stream);
+uint32_t* device_error_word();
+
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+qlora_status check_blocks(int32_t bs, int32_t bs2) {
+    return (bs == 64 && bs2 == 256) ? QLORA_OK : QLORA_ERR_UNSUPPORTED;
+}
+
+qlora_status check_shape(int64_t N, int64_t K) {
+    if (N < 1 || K < 1 || K % 64 != 0) return QLORA_ERR_SHAPE;
+    if (N > (int64_t(1) << 40) / K) return QLORA_ERR_SHAPE;   // keeps every flat index in int64 range
+    return QLORA_OK;
+}
+
+qlora_status check_weight(const qlora_nf4_weight* w) {
+    if (!w) return QLORA_ERR_INVALID_ARG;
+    QLORA_TRY(check_blocks(w->blocksize, w->blocksize2));
+    QLORA_TRY(check_shape(w->N, w->K));
+    if (!w->codes || !w->c1_codes || !w->c2 || !w->mu) return QLORA_ERR_INVALID_ARG;
+    if (!aligned16(w->codes) || !aligned16(w->c1_codes) || !aligned16(w->c2) || !aligned16(w->mu))
+        return QLORA_ERR_ALIGN;
+    return QLORA_OK;
+}
+
+qlora_status check_dev(const void* p) {
+    if (!p) return QLORA_ERR_INVALID_ARG;
+    return aligned16(p) ? QLORA_OK : QLORA_ERR_ALIGN;
+}
+
+qlora_status check_lora(int64_t M, int32_t r, float alpha) {
+    if (M < 1 || M > (int64_t(1) << 31)) return QLORA_ERR_SHAPE;
+    if (r < 1 || r > 256) return QLORA_ERR_INVALID_ARG;
+    if (!std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
+    return QLORA_OK;
+}
+
+// Workspace of the linear layer: U (fp32 [M,r]) and dU (fp32 [M,r]).
+struct LinearWs {
+    size_t u_off, du_off, total;
+};
+
+LinearWs linear_ws(int64_t M, int32_t r) {
+    LinearWs l;
+    l.u_off = 0;
+    l.du_off = align_up((size_t)M * r * sizeof(float), 256);
+    l.total = l.du_off + align_up((size_t)M * r * sizeof(float), 256);
+    return l;
+}
+
+}  // namespace
+
+void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+}  // namespace qlora
+
+using namespace qlora;
+
+extern "C" {
+
+const char* qlora_status_string(qlora_status s) {
+    switch (s) {
+        case QLORA_OK: return "QLORA_OK";
+        case QLORA_ERR_INVALID_ARG: return "QLORA_ERR_INVALID_ARG: null pointer or argument out of range";
+        case QLORA_ERR_SHAPE: return "QLORA_ERR_SHAPE: need N, K, M >= 1 and K % 64 == 0";
+        case QLORA_ERR_ALIGN: return "QLORA_ERR_ALIGN: device pointers must be 16-byte aligned";
+        case QLORA_ERR_UNSUPPORTED: return "QLORA_ERR_UNSUPPORTED: only blocksize 64 and blocksize2 256";
+        case QLORA_ERR_NONFINITE: return "QLORA_ERR_NONFINITE: the weight held Inf or NaN";
+        case QLORA_ERR_TIMEOUT: return "QLORA_ERR_TIMEOUT: a bounded device wait ran out";
+        case QLORA_ERR_CUDA: return "QLORA_ERR_CUDA: a CUDA call or kernel launch failed";
+        case QLORA_ERR_WORKSPACE: return "QLORA_ERR_WORKSPACE: workspace missing or too small";
+    }
+    return "QLORA_ERR_UNKNOWN";
+}
+
+qlora_status qlora_nf4_sizes(int64_t N, int64_t K, int32_t blocksize, int32_t blocksize2,
+                             size_t* codes_bytes, size_t* c1_codes_bytes, size_t* c2_bytes,
+                             size_t* quant_workspace_bytes) {
+    QLORA_TRY(check_blocks(blocksize, blocksize2));
+    QLORA_TRY(check_shape(N, K));
+    const int64_t nb1 = N * K / 64;
+    const int64_t nb2 = (nb1 + 255) / 256;
+    if (codes_bytes) *codes_bytes = (size_t)(N * K / 2);
+    if (c1_codes_bytes) *c1_codes_bytes = (size_t)nb1;
+    if (c2_bytes) *c2_bytes = (size_t)nb2 * sizeof(float);
+    if (quant_workspace_bytes) *quant_workspace_bytes = quantize_workspace_bytes(nb1);
+    return QLORA_OK;
+}
+
+qlora_status qlora_nf4_codebook(float values[16], float thresholds[15]) {
+    const NF4Tables& tb = host_tables();
+    if (values) std::memcpy(values, tb.q, sizeof(tb.q));
+    if (thresholds) std::memcpy(thresholds, tb.t, sizeof(tb.t));
+    return QLORA_OK;
+}
+
+qlora_status qlora_quantize_nf4_dq(const void* W, int64_t N, int64_t K, int32_t blocksize,
+                                   int32_t blocksize2, const qlora_nf4_weight* out,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+    QLORA_TRY(check_blocks(blocksize, blocksize2));
+    QLORA_TRY(check_shape(N, K));
+    QLORA_TRY(check_dev(W));
+    QLORA_TRY(check_weight(out));
+    if (out->N != N || out->K != K) return QLORA_ERR_SHAPE;
+    if (!workspace || workspace_bytes < quantize_workspace_bytes(N * K / 64)) return QLORA_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return QLORA_ERR_ALIGN;
+    TimerScope t(QLORA_TIMER_QUANTIZE, static_cast<cudaStream_t>(stream));
+    return launch_quantize(W, N, K, out, workspace, static_cast<cudaStream_t>(stream));
+}
+
+qlora_status qlora_dequantize(const qlora_nf4_weight* w, void* W_out, void* stream) {
+    QLORA_TRY(check_weight(w));
+    QLORA_TRY(check_dev(W_out));
+    TimerScope t(QLORA_TIMER_DEQUANTIZE, static_cast<cudaStream_t>(stream));
+    return launch_dequantize(w, W_out, static_cast<cudaStream_t>(stream));
+}
+
+qlora_status qlora_linear_workspace_size(int64_t M, int64_t N, int64_t K, int32_t r, size_t* bytes) {
+    QLORA_TRY(check_shape(N, K));
+    QLORA_TRY(check_lora(M, r, 1.0f));
+    if (!bytes) return QLORA_ERR_INVALID_ARG;
+    *bytes = linear_ws(M, r).total;
+    return QLORA_OK;
+}
+
+qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const void* X, int64_t M,
+                              const void* A, const void* B, int32_t r, float alpha,
+                              void* Y, int32_t y_dtype, float* U_save,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+    QLORA_TRY(check_weight(w));
+    QLORA_TRY(check_lora(M, r, alpha));
+    QLORA_TRY(check_dev(X));
+    QLORA_TRY(check_dev(A));
+    QLORA_TRY(check_dev(B));
+    QLORA_TRY(check_dev(Y));
+    if (y_dtype != QLORA_DTYPE_BF16 && y_dtype != QLORA_DTYPE_F32) return QLORA_ERR_INVALID_ARG;
+    if (U_save && !aligned16(U_save)) return QLORA_ERR_ALIGN;
+    const LinearWs lw = linear_ws(M, r);
+    if (!workspace || workspace_bytes < lw.total) return QLORA_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return QLORA_ERR_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t N = w->N, K = w->K;
+    float* U = U_save ? U_save : reinterpret_cast<float*>(static_cast<char*>(workspace) + lw.u_off);
+    const float scale = alpha / (float)r;
+
+    SimtGemm g{};
+    g.nseg = 1;
+    g.seg[0].a = simt_dense(SIMT_BF16, X, K, 1);
+    g.seg[0].b = simt_dense(SIMT_BF16, A, K, 1);
+    g.seg[0].K = K; g.seg[0].scale = 1.f;
+    g.M = M; g.N = r; g.C = U; g.c_dtype = QLORA_DTYPE_F32; g.ldc = r;
+    {
+        TimerScope t(QLORA_TIMER_LORA, s);
+        QLORA_TRY(launch_simt_gemm(g, s));
+    }
+
+    SimtGemm y{};
+    y.nseg = 2;
+    y.seg[0].a = simt_dense(SIMT_BF16, X, K, 1);
+    y.seg[0].b = simt_nf4(w, false);
+    y.seg[0].K = K; y.seg[0].scale = 1.f;
+    y.seg[1].a = simt_dense(SIMT_F32, U, r, 1);
+    y.seg[1].b = simt_dense(SIMT_BF16, B, r, 1);
+    y.seg[1].K = r; y.seg[1].scale = scale;
+    y.M = M; y.N = N; y.C = Y; y.c_dtype = y_dtype; y.ldc = N;
+    TimerScope t(QLORA_TIMER_FWD_MAIN, s);
+    return launch_simt_gemm(y, s);
+}
+
+qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const void* X, const void* dY, int64_t M,
+                              const void* A, const void* B, int32_t r, float alpha,
+                              const float* U_saved, void* dX, int32_t dx_dtype,
+                              float* dA, float* dB,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+    QLORA_TRY(check_weight(w));
+    QLORA_TRY(check_lora(M, r, alpha));
+    QLORA_TRY(check_dev(X));
+    QLORA_TRY(check_dev(dY));
+    QLORA_TRY(check_dev(A));
+    QLORA_TRY(check_dev(B));
+    QLORA_TRY(check_dev(dA));
+    QLORA_TRY(check_dev(dB));
+    if (dX) {
+        QLORA_TRY(check_dev(dX));
+        if (dx_dtype != QLORA_DTYPE_BF16 && dx_dtype != QLORA_DTYPE_F32) return QLORA_ERR_INVALID_ARG;
+    }
+    if (U_saved && !aligned16(U_saved)) return QLORA_ERR_ALIGN;
+    const LinearWs lw = linear_ws(M, r);
+    if (!workspace || workspace_bytes < lw.total) return QLORA_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return QLORA_ERR_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t N = w->N, K = w->K;
+    char* ws = static_cast<char*>(workspace);
+    const float scale = alpha / (float)r;
+
+    const float* U = U_saved;
+    if (!U) {
+        float* Uw = reinterpret_cast<float*>(ws + lw.u_off);
+        SimtGemm g{};
+        g.nseg = 1;
+        g.seg[0].a = simt_dense(SIMT_BF16, X, K, 1);
+        g.seg[0].b = simt_dense(SIMT_BF16, A, K, 1);
+        g.seg[0].K = K; g.seg[0].scale = 1.f;
+        g.M = M; g.N = r; g.C = Uw; g.c_dtype = QLORA_DTYPE_F32; g.ldc = r;
+        TimerScope t(QLORA_TIMER_LORA, s);
+        QLORA_TRY(launch_simt_gemm(g, s));
+        U = Uw;
+    }
+    float* dU = reinterpret_cast<float*>(ws + lw.du_off);
+    {   // dU = s dY B
+        SimtGemm g{};
+        g.nseg = 1;
+        g.seg[0].a = simt_dense(SIMT_BF16, dY, N, 1);
+        g.seg[0].b = simt_dense(SIMT_BF16, B, 1, r);
+        g.seg[0].K = N; g.seg[0].scale = scale;
+        g.M = M; g.N = r; g.C = dU; g.c_dtype = QLORA_DTYPE_F32; g.ldc = r;
+        TimerScope t(QLORA_TIMER_LORA, s);
+        QLORA_TRY(launch_simt_gemm(g, s));
+    }
+    if (dX) {   // dX = dY W_hat + dU A
+        SimtGemm g{};
+        g.nseg = 2;
+        g.seg[0].a = simt_dense(SIMT_BF16, dY, N, 1);
+        g.seg[0].b = simt_nf4(w, true);
+        g.seg[0].K = N; g.seg[0].scale = 1.f;
+        g.seg[1].a = simt_dense(SIMT_F32, dU, r, 1);
+        g.seg[1].b = simt_dense(SIMT_BF16, A, 1, K);
+        g.seg[1].K = r; g.seg[1].scale = 1.f;
+        g.M = M; g.N = K; g.C = dX; g.c_dtype = dx_dtype; g.ldc = K;
+        TimerScope t(QLORA_TIMER_DX_MAIN, s);
+        QLORA_TRY(launch_simt_gemm(g, s));
+    }
+    {   // dA = dU^T X   ([r,K])
+        SimtGemm g{};
+        g.nseg = 1;
+        g.seg[0].a = simt_dense(SIMT_F32, dU, 1, r);
+        g.seg[0].b = simt_dense(SIMT_BF16, X, 1, K);
+        g.seg[0].K = M; g.seg[0].scale = 1.f;
+        g.M = r; g.N = K; g.C = dA; g.c_dtype = QLORA_DTYPE_F32; g.ldc = K;
+        TimerScope t(QLORA_TIMER_LORA, s);
+        QLORA_TRY(launch_simt_gemm(g, s));
+    }
+    {   // dB = s dY^T U   ([N,r])
+        SimtGemm g{};
+        g.nseg = 1;
+        g.seg[0].a = simt_dense(SIMT_BF16, dY, 1, N);
+        g.seg[0].b = simt_dense(SIMT_F32, U, 1, r);
+        g.seg[0].K = M; g.seg[0].scale = scale;
+        g.M = N; g.N = r; g.C = dB; g.c_dtype = QLORA_DTYPE_F32; g.ldc = r;
+        TimerScope t(QLORA_TIMER_LORA, s);
+        QLORA_TRY(launch_simt_gemm(g, s));
+    }
+    return QLORA_OK;
+}
+
+qlora_status qlora_read_device_errors(void* stream, int32_t clear, uint32_t* flags) {
+    uint32_t* word = device_error_word();
+    if (!word) return QLORA_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t h = 0;
+    if (cudaMemcpyAsync(&h, word, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (clear && h) {
+        if (cudaMemsetAsync(word, 0, sizeof(uint32_t), s) != cudaSuccess) return QLORA_ERR_CUDA;
+        if (cudaStreamSynchronize(s) != cudaSuccess) return QLORA_ERR_CUDA;
+    }
+    if (flags) *flags = h;
+    if (h & ERR_FLAG_TIMEOUT) return QLORA_ERR_TIMEOUT;
+    if (h & ERR_FLAG_NONFINITE) return QLORA_ERR_NONFINITE;
+    return QLORA_OK;
+}
+
+uint64_t qlora_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

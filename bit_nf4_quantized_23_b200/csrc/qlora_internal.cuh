@@ -1,0 +1,99 @@
+// Internal declarations shared by the translation units of libqlora.so.
+// Device helpers here use only IEEE basic operations with explicit rounding
+// (__fmul_rn, __fadd_rn, __fdiv_rn, __float2bfloat16_rn) so that no FMA
+// contraction or approximate division changes a bit-exact result.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+#include "../../include/qlora.h"
+
+namespace qlora {
+
+// NF4 code values (ascending) and the 15 decision thresholds, passed to
+// kernels by value (they land in the kernel-parameter constant bank).
+struct NF4Tables {
+    float q[16];
+    float t[15];
+};
+
+// Host side: the library's tables, built once (codebook.cu).
+const NF4Tables& host_tables();
+
+// Host side: count of kernels launched by this library (api.cu).
+void note_launches(int n);
+
+// Device error flag word (one per device that loaded the library).  Kernels in
+// quantize.cu set it directly; other kernels get its address as an argument.
+enum : uint32_t { ERR_FLAG_TIMEOUT = 1u, ERR_FLAG_NONFINITE = 2u };
+
+// Host side: device address of the error word of the current device (cached
+// per device; nullptr on failure).
+uint32_t* device_error_word();
+
+// Bounded mbarrier/flag waits give up after this many polls (well above any
+// legitimate wait, far below a GPU hang).
+constexpr uint32_t kSpinLimit = 1u << 26;
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) {
+    return __uint_as_float(b << 16);
+}
+
+__device__ __forceinline__ uint32_t f32_to_bf16_bits_rn(float x) {
+    __nv_bfloat16 h = __float2bfloat16_rn(x);
+    return (uint32_t)(*reinterpret_cast<unsigned short*>(&h));
+}
+
+// Two fp32 -> packed bf16x2 (low half = a), round to nearest even.
+__device__ __forceinline__ uint32_t pack_bf16x2_rn(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Exact value of an FP8 E4M3 (finite-only) code: sign, 4-bit exponent with
+// bias 7, 3-bit mantissa; exponent field 0 holds the subnormals m * 2^-9.
+__device__ __forceinline__ float e4m3_to_f32(uint32_t c) {
+    const uint32_t s = (c & 0x80u) << 24;
+    const uint32_t e = (c >> 3) & 0xFu;
+    const uint32_t m = c & 0x7u;
+    const float v = (e == 0u) ? (float)m * 0.001953125f
+                              : __uint_as_float(((e + 120u) << 23) | (m << 20));
+    return __uint_as_float(__float_as_uint(v) | s);
+}
+
+// fp32 -> FP8 E4M3 code, round to nearest even, saturating to +-448.
+__device__ __forceinline__ uint32_t f32_to_e4m3_rn_sat(float x) {
+    return (uint32_t)__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3);
+}
+
+// Rebuilt block constant c1' = fp32(fp32(v8 * c2) + mu), two roundings, no FMA.
+__device__ __forceinline__ float rebuild_c1(uint32_t c1_code, float c2, float mu) {
+    return __fadd_rn(__fmul_rn(e4m3_to_f32(c1_code), c2), mu);
+}
+
+// The dequantized weight value in bf16 bits: bf16_rn(fp32(q * c1')).
+__device__ __forceinline__ uint32_t dequant_bits(float q, float c1p) {
+    return f32_to_bf16_bits_rn(__fmul_rn(q, c1p));
+}
+
+}  // namespace qlora
+
+// Launch helpers (host).  Every launch in the library goes through these so
+// that the launch counter is exact and launch errors map to QLORA_ERR_CUDA.
+#define QLORA_CHECK_LAUNCH()                                   \
+    do {                                                       \
+        qlora::note_launches(1);                               \
+        if (cudaPeekAtLastError() != cudaSuccess) {            \
+            (void)cudaGetLastError();                          \
+            return QLORA_ERR_CUDA;                             \
+        }                                                      \
+    } while (0)
+
+#define QLORA_TRY(expr)                                        \
+    do {                                                       \
+        qlora_status _s = (expr);                              \
+        if (_s != QLORA_OK) return _s;                         \
+    } while (0)

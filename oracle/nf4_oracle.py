@@ -373,6 +373,38 @@ def dequantize_rows(qw: dict, rows: np.ndarray, q: np.ndarray | None = None) -> 
     return f32_to_bf16_bits(prod)
 
 
+def quantize_rows(W_bits: np.ndarray, rows, q: np.ndarray | None = None) -> dict:
+    """Quantize with the double-quantized constants of the whole tensor, but the
+    per-element codes of the selected rows only (same steps as quantize_nf4_dq;
+    for checking large tensors by sampling)."""
+    W_bits = np.asarray(W_bits, dtype=np.uint16)
+    N, K = W_bits.shape
+    check_args(N, K)
+    q = nf4_codebook() if q is None else q
+    rows = np.asarray(rows, dtype=np.int64)
+    c1 = block_absmax(bf16_bits_to_f32(W_bits).ravel(), BLOCKSIZE).astype(np.float32)
+    c1_codes, c2, mu = double_quantize(c1)
+    bpr = K // BLOCKSIZE
+    w_rows = bf16_bits_to_f32(W_bits[rows]).ravel()
+    c1_rows = c1.reshape(N, bpr)[rows].ravel()
+    codes = nearest_code(normalize_blocks(w_rows, c1_rows), q)
+    return {"codes_rows": pack_nibbles(codes).reshape(len(rows), K // 2), "c1_codes": c1_codes,
+            "c2": c2, "mu": np.float32(mu), "c1": c1, "N": N, "K": K}
+
+
+def dequantize_cols(qw: dict, cols, q: np.ndarray | None = None) -> np.ndarray:
+    """W_hat for selected columns only (uint16 bits [N, len(cols)]); same arithmetic as dequantize."""
+    q = nf4_codebook() if q is None else q
+    N, K = qw["N"], qw["K"]
+    cols = np.asarray(cols, dtype=np.int64)
+    flat = np.arange(N, dtype=np.int64)[:, None] * K + cols[None, :]
+    byte = np.asarray(qw["codes"], dtype=np.uint8)[flat >> 1]
+    idx = np.where((flat & 1) == 1, byte & 0xF, byte >> 4)
+    c1p = dq_constants(qw["c1_codes"], qw["c2"], qw["mu"])
+    prod = (q[idx] * c1p[flat >> 6]).astype(np.float32)
+    return f32_to_bf16_bits(prod)
+
+
 # ---------------------------------------------------------------------------
 # The linear layer in fp64 ([QP] Section 7 diagram; [QR] Section 4.4; R7, R8)
 # ---------------------------------------------------------------------------

@@ -1,0 +1,275 @@
+"""GPU parity: the CUDA library (through its C ABI) against the CPU oracle.
+
+Bit-exact: packed NF4 codes, E4M3 constant codes, c2, mu and the dequantized
+bf16 weight.  Within tolerance (tests/parity.py): Y, dX, dA, dB.  Small shapes
+are compared element by element in full; the full-size workloads are compared
+on seeded samples of rows/columns the oracle computes one by one, plus full
+dA and dB.
+"""
+import numpy as np
+import pytest
+import torch
+
+import bit_nf4_quantized_23_b200 as q4
+import synthetic_inputs as si
+from oracle import nf4_oracle as o
+from parity import assert_close, to_numpy_bits
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib_built():
+    from bit_nf4_quantized_23_b200.build import build
+    build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    q4.qlora_read_device_errors(clear=True)
+    yield
+    assert q4.qlora_read_device_errors(clear=True) == 0
+
+
+def quantize_on_gpu(W_cpu):
+    w = q4.qlora_quantize_nf4_dq(W_cpu.to(DEV))
+    torch.cuda.synchronize()
+    return w
+
+
+def check_quantize_exact(W_cpu, w_gpu, qw=None):
+    bits = si.bf16_bits(W_cpu)
+    qw = o.quantize_nf4_dq(bits) if qw is None else qw
+    assert np.array_equal(w_gpu.codes.cpu().numpy(), qw["codes"])
+    assert np.array_equal(w_gpu.c1_codes.cpu().numpy(), qw["c1_codes"])
+    assert np.array_equal(w_gpu.c2.cpu().numpy().view(np.uint32), qw["c2"].view(np.uint32))
+    assert w_gpu.mu.cpu().numpy().view(np.uint32)[0] == np.float32(qw["mu"]).view(np.uint32)
+    return qw
+
+
+def check_dequantize_exact(w_gpu, qw):
+    Wh = q4.qlora_dequantize(w_gpu)
+    ref = o.dequantize(qw["codes"], qw["c1_codes"], qw["c2"], qw["mu"], qw["N"], qw["K"])
+    assert np.array_equal(to_numpy_bits(Wh), ref)
+    return ref
+
+
+# ------------------------------------------------------------------ quantize / dequantize
+
+SHAPES = [(256, 256), (1, 64), (3, 320), (5, 4160), (17, 1024), (64, 192), (2, 16384)]
+
+
+@pytest.mark.parametrize("N,K", SHAPES)
+def test_quantize_and_dequantize_bit_exact(N, K):
+    W = si.custom_linear(N, K, 1, 1, seed=N * 131 + K)[0]
+    w = quantize_on_gpu(W)
+    qw = check_quantize_exact(W, w)
+    check_dequantize_exact(w, qw)
+
+
+def test_quantize_heavy_tailed_weights_bit_exact():
+    W = si.custom_linear(96, 8192, 1, 1, seed=3, dist="t5")[0]
+    w = quantize_on_gpu(W)
+    check_dequantize_exact(w, check_quantize_exact(W, w))
+
+
+def _boundary_weight(seed=0):
+    """Blocks whose values straddle every decision threshold of every scale.
+
+    Each block holds its absmax c (so c1 = c) and bf16 values next to t_j * c
+    for the 15 midpoints t_j of neighbouring codes, with both signs."""
+    g = np.random.default_rng(seed)
+    q = o.nf4_codebook().astype(np.float64)
+    mids = (q[:-1] + q[1:]) / 2
+    rows = []
+    for _ in range(1024):
+        c = np.float32(2.0 ** g.uniform(-20, 20))
+        c_bits = o.f32_to_bf16_bits(np.array([c], np.float32))
+        c = o.bf16_bits_to_f32(c_bits)[0]
+        centre = o.f32_to_bf16_bits((mids * c).astype(np.float32)).astype(np.int64)
+        cand = np.concatenate([centre + d for d in (-2, -1, 0, 1, 2)])
+        cand = cand[(cand & 0x7F80) != 0x7F80].astype(np.uint16)     # finite only
+        pick = g.choice(cand, 63, replace=True)
+        block = np.concatenate([c_bits, pick]).astype(np.uint16)
+        g.shuffle(block)
+        rows.append(block)
+    return np.concatenate(rows).reshape(-1, 1024)
+
+
+def test_quantize_decision_boundaries_bit_exact():
+    bits = _boundary_weight()
+    W = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+    w = quantize_on_gpu(W)
+    check_dequantize_exact(w, check_quantize_exact(W, w))
+
+
+def test_quantize_every_finite_bf16_value():
+    g = np.random.default_rng(1)
+    allb = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    allb = allb[(allb & 0x7F80) != 0x7F80]                      # drop Inf/NaN
+    allb = np.concatenate([allb, np.zeros((-allb.size) % 1024, np.uint16)])
+    # sort by magnitude within shuffled neighbourhoods so that blocks hold values of similar scale
+    mag = o.bf16_bits_to_f32(allb)
+    order = np.argsort(np.abs(mag) * np.exp(g.normal(0, 0.5, allb.size)))
+    W = torch.from_numpy(allb[order].view(np.int16).reshape(-1, 1024)).view(torch.bfloat16)
+    w = quantize_on_gpu(W)
+    check_dequantize_exact(w, check_quantize_exact(W, w))
+
+
+def test_zero_blocks_and_signed_zeros():
+    bits = si.bf16_bits(si.custom_linear(4, 512, 1, 1, seed=9)[0]).copy()
+    bits[0, :64] = 0
+    bits[1, 64:128] = 0x8000          # -0.0
+    bits[2, :] = 0
+    W = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+    w = quantize_on_gpu(W)
+    check_dequantize_exact(w, check_quantize_exact(W, w))
+
+
+def test_nonfinite_weight_sets_flag():
+    bits = si.bf16_bits(si.custom_linear(2, 128, 1, 1, seed=4)[0]).copy()
+    bits[1, 5] = 0x7F80               # +Inf
+    W = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(DEV)
+    q4.qlora_read_device_errors(clear=True)
+    q4.qlora_quantize_nf4_dq(W)
+    flags = q4.qlora_read_device_errors(clear=True)
+    assert flags & 2
+
+
+# ------------------------------------------------------------------ linear forward / backward
+
+def run_linear(W, X, A, B, dY, r, alpha, y_dtype=torch.bfloat16, dx_dtype=torch.bfloat16, save_U=True):
+    w = quantize_on_gpu(W)
+    Xd, Ad, Bd, dYd = (t.to(DEV) for t in (X, A, B, dY))
+    Y, U = q4.qlora_linear_fwd(w, Xd, Ad, Bd, r, alpha, y_dtype=y_dtype, save_U=save_U)
+    dX, dA, dB = q4.qlora_linear_bwd(w, Xd, dYd, Ad, Bd, r, alpha, U_saved=U, dx_dtype=dx_dtype)
+    torch.cuda.synchronize()
+    return w, Y, U, dX, dA, dB
+
+
+def check_linear_full(W, X, A, B, dY, r, alpha, **kw):
+    w, Y, U, dX, dA, dB = run_linear(W, X, A, B, dY, r, alpha, **kw)
+    qw = o.quantize_nf4_dq(si.bf16_bits(W))
+    Wh = o.dequantize(qw["codes"], qw["c1_codes"], qw["c2"], qw["mu"], qw["N"], qw["K"])
+    bX, bA, bB, bdY = (si.bf16_bits(t) for t in (X, A, B, dY))
+    Yr, Ur = o.linear_forward(bX, Wh, bA, bB, alpha, r)
+    g = o.linear_backward(bX, bdY, Wh, bA, bB, alpha, r)
+    assert_close(Y, Yr, "Y")
+    if U is not None:
+        assert_close(U, Ur, "U")
+    assert_close(dX, g["dX"], "dX")
+    assert_close(dA, g["dA"], "dA")
+    assert_close(dB, g["dB"], "dB")
+    return w
+
+
+def test_tiny_workload_full():
+    wl = si.WORKLOADS["tiny"]
+    W = si.weight(wl, 0)
+    N, K = wl.linears[0]
+    X = si.activations(wl, K, wl.M)
+    A, B = si.lora(wl, 0)
+    dY = si.grad_output(wl, 0, wl.M)
+    for y_dtype in (torch.bfloat16, torch.float32):
+        check_linear_full(W, X, A, B, dY, wl.r, wl.alpha, y_dtype=y_dtype, dx_dtype=y_dtype)
+
+
+@pytest.mark.parametrize("M,N,K,r", [(1, 64, 64, 1), (3, 192, 128, 5), (17, 320, 192, 16),
+                                     (130, 96, 640, 64), (33, 128, 256, 256)])
+def test_ragged_linear(M, N, K, r):
+    W, X, A, B, dY = si.custom_linear(N, K, M, r, seed=M + N + K + r)
+    check_linear_full(W, X, A, B, dY, r, alpha=2.0 * r)
+
+
+def test_recompute_U_and_no_dX():
+    W, X, A, B, dY = si.custom_linear(128, 256, 24, 8, seed=77)
+    w = quantize_on_gpu(W)
+    Xd, Ad, Bd, dYd = (t.to(DEV) for t in (X, A, B, dY))
+    _, U = q4.qlora_linear_fwd(w, Xd, Ad, Bd, 8, 16.0)
+    dX1, dA1, dB1 = q4.qlora_linear_bwd(w, Xd, dYd, Ad, Bd, 8, 16.0, U_saved=U)
+    dX2, dA2, dB2 = q4.qlora_linear_bwd(w, Xd, dYd, Ad, Bd, 8, 16.0, U_saved=None, need_dX=False)
+    assert dX2 is None
+    assert torch.allclose(dA1, dA2, rtol=1e-5, atol=1e-6)
+    assert torch.allclose(dB1, dB2, rtol=1e-5, atol=1e-6)
+
+
+def test_backward_leaves_weight_buffers_untouched():
+    W, X, A, B, dY = si.custom_linear(256, 512, 64, 16, seed=5)
+    w = quantize_on_gpu(W)
+    before = [t.clone() for t in (w.codes, w.c1_codes, w.c2, w.mu)]
+    Xd, Ad, Bd, dYd = (t.to(DEV) for t in (X, A, B, dY))
+    _, U = q4.qlora_linear_fwd(w, Xd, Ad, Bd, 16, 32.0)
+    q4.qlora_linear_bwd(w, Xd, dYd, Ad, Bd, 16, 32.0, U_saved=U)
+    torch.cuda.synchronize()
+    for a, b in zip(before, (w.codes, w.c1_codes, w.c2, w.mu)):
+        assert torch.equal(a, b)
+
+
+def test_alpha_zero_and_zero_B():
+    W, X, A, B, dY = si.custom_linear(64, 128, 8, 4, seed=6)
+    check_linear_full(W, X, A, B, dY, 4, alpha=0.0)
+    Bz = torch.zeros_like(B)
+    w, Y, U, dX, dA, dB = run_linear(W, X, A, Bz, dY, 4, 8.0)
+    assert torch.count_nonzero(dA) == 0
+
+
+# ------------------------------------------------------------------ full-size workloads, sampled
+
+def _sampled_linear_check(wl_name, i, M, bwd=True, nrows=64, seed=0):
+    wl = si.WORKLOADS[wl_name]
+    N, K = wl.linears[i]
+    W = si.weight(wl, i)
+    X = si.activations(wl, K, M)
+    A, B = si.lora(wl, i)
+    bits = si.bf16_bits(W)
+    g = np.random.default_rng(seed + i)
+    rows_w = np.sort(g.choice(N, min(nrows, N), replace=False))
+    w = quantize_on_gpu(W)
+    part = o.quantize_rows(bits, rows_w)
+    assert np.array_equal(w.codes.cpu().numpy().reshape(N, K // 2)[rows_w], part["codes_rows"])
+    assert np.array_equal(w.c1_codes.cpu().numpy(), part["c1_codes"])
+    assert np.array_equal(w.c2.cpu().numpy().view(np.uint32), part["c2"].view(np.uint32))
+    assert w.mu.cpu().numpy().view(np.uint32)[0] == np.float32(part["mu"]).view(np.uint32)
+    qw = {"codes": w.codes.cpu().numpy(), "c1_codes": part["c1_codes"], "c2": part["c2"],
+          "mu": part["mu"], "N": N, "K": K}       # codes already verified on the sampled rows
+    Xd, Ad, Bd = X.to(DEV), A.to(DEV), B.to(DEV)
+    Y, U = q4.qlora_linear_fwd(w, Xd, Ad, Bd, wl.r, wl.alpha)
+    bX, bA, bB = si.bf16_bits(X), si.bf16_bits(A), si.bf16_bits(B)
+    rows_m = np.sort(g.choice(M, min(nrows, M), replace=False))
+    cols_n = np.sort(g.choice(N, min(nrows, N), replace=False))
+    Wh_rows = o.dequantize_rows(qw, cols_n)                      # W_hat[n, :] for sampled n
+    Yref = o.linear_forward(o._f64(bX)[rows_m], Wh_rows, bA, bB[cols_n], wl.alpha, wl.r)[0]
+    assert_close(Y[torch.as_tensor(rows_m)][:, torch.as_tensor(cols_n)].contiguous(), Yref, "Y sampled")
+    if not bwd:
+        return
+    dY = si.grad_output(wl, i, M)
+    dYd = dY.to(DEV)
+    dX, dA, dB = q4.qlora_linear_bwd(w, Xd, dYd, Ad, Bd, wl.r, wl.alpha, U_saved=U)
+    torch.cuda.synchronize()
+    bdY = si.bf16_bits(dY)
+    s = wl.alpha / wl.r
+    cols_k = np.sort(g.choice(K, min(nrows, K), replace=False))
+    Wh_cols = o._f64(o.dequantize_cols(qw, cols_k))                # [N, len(cols_k)]
+    dYs = o._f64(bdY)[rows_m]
+    dU_s = s * (dYs @ o._f64(bB))
+    dXref = dYs @ Wh_cols + dU_s @ o._f64(bA)[:, cols_k]
+    assert_close(dX[torch.as_tensor(rows_m)][:, torch.as_tensor(cols_k)].contiguous(), dXref, "dX sampled")
+    Xf, dYf = o._f64(bX), o._f64(bdY)
+    dU = s * (dYf @ o._f64(bB))
+    assert_close(dA, dU.T @ Xf, "dA full")
+    assert_close(dB, s * (dYf.T @ (Xf @ o._f64(bA).T)), "dB full")
+
+
+def test_attn7b_quantize_and_forward():
+    _sampled_linear_check("attn7b", 0, 512, bwd=False)
+
+
+def test_mlp7b_down_projection_fwd_bwd():
+    _sampled_linear_check("mlp7b", 2, 4096)
+
+
+def test_block65b_mlp_up_fwd_bwd():
+    _sampled_linear_check("block65b", 4, 2048)
+
+
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_decode_forward(M):
+    _sampled_linear_check("decode", 1, M, bwd=False)

@@ -446,3 +446,17 @@ def test_row_subsets_match_full():
                        o.linear_forward(X, Wh, A, B, 4.0, 2)[0][rows], rtol=1e-14, atol=0)
     assert np.allclose(o.backward_dx_rows(dY, Wh, A, B, 4.0, 2, rows),
                        o.linear_backward(X, dY, Wh, A, B, 4.0, 2)["dX"][rows], rtol=1e-14, atol=0)
+
+
+def test_row_and_column_samplers_match_full_quantize():
+    W = si.custom_linear(24, 512, 1, 8, 31)[0]
+    bits = si.bf16_bits(W)
+    full = o.quantize_nf4_dq(bits)
+    rows = np.array([0, 7, 23])
+    part = o.quantize_rows(bits, rows)
+    assert np.array_equal(part["codes_rows"], full["codes"].reshape(24, 256)[rows])
+    for k in ("c1_codes", "c2", "mu"):
+        assert np.array_equal(part[k], full[k])
+    Wh = o.dequantize(full["codes"], full["c1_codes"], full["c2"], full["mu"], 24, 512)
+    cols = np.array([0, 1, 63, 64, 511])
+    assert np.array_equal(o.dequantize_cols(full, cols), Wh[:, cols])
