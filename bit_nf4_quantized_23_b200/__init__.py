@@ -19,6 +19,7 @@ from ._lib import (QLORA_DTYPE_BF16, QLORA_DTYPE_F32, TIMER_KINDS, NF4WeightC, Q
 
 __all__ = [
     "NF4Weight", "QloraError", "qlora_nf4_sizes", "qlora_nf4_codebook", "qlora_quantize_nf4_dq",
+    "qlora_quantize_nf4_dq_noalloc",
     "qlora_dequantize", "qlora_linear_workspace_size", "qlora_linear_fwd", "qlora_linear_bwd",
     "qlora_read_device_errors", "qlora_launch_count", "qlora_timing_enable", "qlora_timing_read",
 ]
@@ -105,6 +106,18 @@ def qlora_quantize_nf4_dq(W: torch.Tensor, blocksize: int = 64, blocksize2: int 
     ws = out.c_struct()
     check(lib().qlora_quantize_nf4_dq(_ptr(W), N, K, blocksize, blocksize2, byref(ws), _ptr(workspace),
                                       workspace.numel(), _stream(stream)), "qlora_quantize_nf4_dq")
+    return out
+
+
+def qlora_quantize_nf4_dq_noalloc(W: torch.Tensor, out: NF4Weight, stream=None) -> NF4Weight:
+    """Quantize into caller-allocated `out` using the library's static device scratch (no
+    workspace, no allocation in the call).  At most 67,108,864 weights; calls that overlap on
+    the GPU race on the shared scratch."""
+    _need(W, torch.bfloat16, "W")
+    N, K = W.shape
+    ws = out.c_struct()
+    check(lib().qlora_quantize_nf4_dq_noalloc(_ptr(W), N, K, 64, 256, byref(ws), _stream(stream)),
+          "qlora_quantize_nf4_dq_noalloc")
     return out
 
 

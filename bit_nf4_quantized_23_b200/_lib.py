@@ -16,7 +16,7 @@ QLORA_OK = 0
 STATUS_NAMES = {
     0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_SHAPE", 3: "QLORA_ERR_ALIGN",
     4: "QLORA_ERR_UNSUPPORTED", 5: "QLORA_ERR_NONFINITE", 6: "QLORA_ERR_TIMEOUT",
-    7: "QLORA_ERR_CUDA", 8: "QLORA_ERR_WORKSPACE",
+    7: "QLORA_ERR_CUDA", 8: "QLORA_ERR_WORKSPACE", 9: "QLORA_ERR_TOO_LARGE",
 }
 QLORA_DTYPE_BF16 = 0
 QLORA_DTYPE_F32 = 1
@@ -40,6 +40,7 @@ SIGNATURES = {
     "qlora_nf4_codebook": (c_int32, [POINTER(c_float), POINTER(c_float)]),
     "qlora_quantize_nf4_dq": (c_int32, [c_void_p, c_int64, c_int64, c_int32, c_int32, _W, c_void_p,
                                         c_size_t, c_void_p]),
+    "qlora_quantize_nf4_dq_noalloc": (c_int32, [c_void_p, c_int64, c_int64, c_int32, c_int32, _W, c_void_p]),
     "qlora_dequantize": (c_int32, [_W, c_void_p, c_void_p]),
     "qlora_linear_workspace_size": (c_int32, [c_int64, c_int64, c_int64, c_int32, POINTER(c_size_t)]),
     "qlora_linear_fwd": (c_int32, [_W, c_void_p, c_int64, c_void_p, c_void_p, c_int32, c_float, c_void_p,

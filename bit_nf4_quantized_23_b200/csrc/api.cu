@@ -91,6 +91,9 @@ const char* qlora_status_string(qlora_status s) {
         case QLORA_ERR_TIMEOUT: return "QLORA_ERR_TIMEOUT: a bounded device wait ran out";
         case QLORA_ERR_CUDA: return "QLORA_ERR_CUDA: a CUDA call or kernel launch failed";
         case QLORA_ERR_WORKSPACE: return "QLORA_ERR_WORKSPACE: workspace missing or too small";
+        case QLORA_ERR_TOO_LARGE:
+            return "QLORA_ERR_TOO_LARGE: more than 67108864 weights for the static scratch of "
+                   "qlora_quantize_nf4_dq_noalloc";
     }
     return "QLORA_ERR_UNKNOWN";
 }

@@ -54,7 +54,8 @@ typedef enum {
     QLORA_ERR_NONFINITE = 5,     /* the weight held Inf or NaN (reported by qlora_read_device_errors) */
     QLORA_ERR_TIMEOUT = 6,       /* a bounded device wait ran out (reported by qlora_read_device_errors) */
     QLORA_ERR_CUDA = 7,          /* a CUDA runtime call or kernel launch failed */
-    QLORA_ERR_WORKSPACE = 8      /* workspace pointer null or smaller than the size query returned */
+    QLORA_ERR_WORKSPACE = 8,     /* workspace pointer null or smaller than the size query returned */
+    QLORA_ERR_TOO_LARGE = 9      /* tensor larger than qlora_quantize_nf4_dq_noalloc's static scratch */
 } qlora_status;
 
 typedef enum { QLORA_DTYPE_BF16 = 0, QLORA_DTYPE_F32 = 1 } qlora_dtype;
@@ -137,6 +138,28 @@ qlora_status qlora_quantize_nf4_dq(const void* W, int64_t N, int64_t K,
                                    int32_t blocksize, int32_t blocksize2,
                                    const qlora_nf4_weight* out,
                                    void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * qlora_quantize_nf4_dq without a workspace argument, for callers that cannot
+ * allocate device memory when they quantize (for example a plugin whose host
+ * framework owns every device allocation and passes only input and output
+ * pointers, or a latency-critical path that must not call cudaMalloc/cudaFree,
+ * which may synchronize the device).  The pages have no counterpart: this is a
+ * deployment variant of the same operation with the same bit-exact results.
+ *   Scratch: a static array of 4.25 MiB in the library's device image, held by
+ *   every GPU that loads the library until the process exits.  Tensors of more
+ *   than 67,108,864 weights (e.g. larger than W[8192,8192]) return
+ *   QLORA_ERR_TOO_LARGE before anything is launched.
+ *   The call allocates nothing.  All calls on a device share the one array and
+ *   it keeps the last call's contents (nothing in it needs to start at zero);
+ *   calls that overlap on the GPU race and give wrong results.  The first call
+ *   on a device looks up the array's device address (once, with that device
+ *   current): make that first call before any stream capture.
+ *   Other arguments and errors as qlora_quantize_nf4_dq.
+ */
+qlora_status qlora_quantize_nf4_dq_noalloc(const void* W, int64_t N, int64_t K,
+                                           int32_t blocksize, int32_t blocksize2,
+                                           const qlora_nf4_weight* out, void* stream);
 
 /*
  * Dequantize to bf16 ([SD] section 4 (1): W_hat = Dequant(W_NF4) * c1):
