@@ -7,6 +7,7 @@
 
 #include "qlora_internal.cuh"
 #include "gemm_simt.cuh"
+#include "gemm_tc.cuh"
 #include "timing.cuh"
 
 namespace qlora {
@@ -16,6 +17,9 @@ qlora_status launch_quantize(const void* W, int64_t N, int64_t K, const qlora_nf
                              void* workspace, cudaStream_t stream);
 qlora_status launch_dequantize(const qlora_nf4_weight* w, void* W_out, cudaStream_t stream);
 uint32_t* device_error_word();
+qlora_status launch_split_hi_lo(const float* V, int64_t M, int r, int R, float scale, void* V2, cudaStream_t s);
+qlora_status launch_dup_cols(const void* B, int64_t N, int r, int R, void* B2, cudaStream_t s);
+qlora_status launch_dup_rows(const void* A, int r, int R, int64_t K, void* A2, cudaStream_t s);
 
 namespace {
 
@@ -57,16 +61,31 @@ qlora_status check_lora(int64_t M, int32_t r, float alpha) {
     return QLORA_OK;
 }
 
-// Workspace of the linear layer: U (fp32 [M,r]) and dU (fp32 [M,r]).
+// LoRA rank padded to a multiple of 32 (two halves of R give 64-wide reduction steps).
+inline int32_t rank_pad(int32_t r) { return (r + 31) / 32 * 32; }
+
+// Workspace of the linear layer (every piece 256-byte aligned):
+//   U   fp32 [M,r]        (when the caller keeps none)
+//   dU  fp32 [M,r]
+//   U2  bf16 [M,2R]       hi/lo split of s*U
+//   B2  bf16 [N,2R]       [B | B]
+//   dU2 bf16 [M,2R]       hi/lo split of dU
+//   A2  bf16 [2R,K]       [A ; A]
 struct LinearWs {
-    size_t u_off, du_off, total;
+    size_t u_off, du_off, u2_off, b2_off, du2_off, a2_off, total;
 };
 
-LinearWs linear_ws(int64_t M, int32_t r) {
+LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int32_t r) {
+    const size_t R = (size_t)rank_pad(r);
     LinearWs l;
-    l.u_off = 0;
-    l.du_off = align_up((size_t)M * r * sizeof(float), 256);
-    l.total = l.du_off + align_up((size_t)M * r * sizeof(float), 256);
+    size_t o = 0;
+    l.u_off = o;   o += align_up((size_t)M * r * sizeof(float), 256);
+    l.du_off = o;  o += align_up((size_t)M * r * sizeof(float), 256);
+    l.u2_off = o;  o += align_up((size_t)M * 2 * R * 2, 256);
+    l.b2_off = o;  o += align_up((size_t)N * 2 * R * 2, 256);
+    l.du2_off = o; o += align_up((size_t)M * 2 * R * 2, 256);
+    l.a2_off = o;  o += align_up(2 * R * (size_t)K * 2, 256);
+    l.total = o;
     return l;
 }
 
@@ -144,7 +163,7 @@ qlora_status qlora_linear_workspace_size(int64_t M, int64_t N, int64_t K, int32_
     QLORA_TRY(check_shape(N, K));
     QLORA_TRY(check_lora(M, r, 1.0f));
     if (!bytes) return QLORA_ERR_INVALID_ARG;
-    *bytes = linear_ws(M, r).total;
+    *bytes = linear_ws(M, N, K, r).total;
     return QLORA_OK;
 }
 
@@ -160,13 +179,15 @@ qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const void* X, int64_t 
     QLORA_TRY(check_dev(Y));
     if (y_dtype != QLORA_DTYPE_BF16 && y_dtype != QLORA_DTYPE_F32) return QLORA_ERR_INVALID_ARG;
     if (U_save && !aligned16(U_save)) return QLORA_ERR_ALIGN;
-    const LinearWs lw = linear_ws(M, r);
+    const LinearWs lw = linear_ws(M, w->N, w->K, r);
     if (!workspace || workspace_bytes < lw.total) return QLORA_ERR_WORKSPACE;
     if (!aligned16(workspace)) return QLORA_ERR_ALIGN;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int64_t N = w->N, K = w->K;
-    float* U = U_save ? U_save : reinterpret_cast<float*>(static_cast<char*>(workspace) + lw.u_off);
+    char* ws = static_cast<char*>(workspace);
+    float* U = U_save ? U_save : reinterpret_cast<float*>(ws + lw.u_off);
     const float scale = alpha / (float)r;
+    const int32_t R = rank_pad(r);
 
     SimtGemm g{};
     g.nseg = 1;
@@ -178,18 +199,18 @@ qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const void* X, int64_t 
         TimerScope t(QLORA_TIMER_LORA, s);
         QLORA_TRY(launch_simt_gemm(g, s));
     }
-
-    SimtGemm y{};
-    y.nseg = 2;
-    y.seg[0].a = simt_dense(SIMT_BF16, X, K, 1);
-    y.seg[0].b = simt_nf4(w, false);
-    y.seg[0].K = K; y.seg[0].scale = 1.f;
-    y.seg[1].a = simt_dense(SIMT_F32, U, r, 1);
-    y.seg[1].b = simt_dense(SIMT_BF16, B, r, 1);
-    y.seg[1].K = r; y.seg[1].scale = scale;
-    y.M = M; y.N = N; y.C = Y; y.c_dtype = y_dtype; y.ldc = N;
+    void* U2 = ws + lw.u2_off;
+    void* B2 = ws + lw.b2_off;
+    {
+        TimerScope t(QLORA_TIMER_LORA, s);
+        QLORA_TRY(launch_split_hi_lo(U, M, r, R, scale, U2, s));
+        QLORA_TRY(launch_dup_cols(B, N, r, R, B2, s));
+    }
+    TcGemmArgs a{};
+    a.w = w; a.A0 = X; a.A1 = U2; a.B1 = B2; a.Rpad = R;
+    a.p.M = M; a.p.Nout = N; a.p.out = Y; a.p.ldo = N; a.p.out_f32 = (y_dtype == QLORA_DTYPE_F32);
     TimerScope t(QLORA_TIMER_FWD_MAIN, s);
-    return launch_simt_gemm(y, s);
+    return launch_tc_gemm_nf4(a, false, s);
 }
 
 qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const void* X, const void* dY, int64_t M,
@@ -210,13 +231,14 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const void* X, const vo
         if (dx_dtype != QLORA_DTYPE_BF16 && dx_dtype != QLORA_DTYPE_F32) return QLORA_ERR_INVALID_ARG;
     }
     if (U_saved && !aligned16(U_saved)) return QLORA_ERR_ALIGN;
-    const LinearWs lw = linear_ws(M, r);
+    const LinearWs lw = linear_ws(M, w->N, w->K, r);
     if (!workspace || workspace_bytes < lw.total) return QLORA_ERR_WORKSPACE;
     if (!aligned16(workspace)) return QLORA_ERR_ALIGN;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int64_t N = w->N, K = w->K;
     char* ws = static_cast<char*>(workspace);
     const float scale = alpha / (float)r;
+    const int32_t R = rank_pad(r);
 
     const float* U = U_saved;
     if (!U) {
@@ -242,7 +264,20 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const void* X, const vo
         TimerScope t(QLORA_TIMER_LORA, s);
         QLORA_TRY(launch_simt_gemm(g, s));
     }
-    if (dX) {   // dX = dY W_hat + dU A
+    if (dX && N % 8 == 0) {   // dX = dY W_hat + dU A on the tensor cores (dY rows must be 16-byte strided)
+        void* dU2 = ws + lw.du2_off;
+        void* A2 = ws + lw.a2_off;
+        {
+            TimerScope t(QLORA_TIMER_LORA, s);
+            QLORA_TRY(launch_split_hi_lo(dU, M, r, R, 1.f, dU2, s));
+            QLORA_TRY(launch_dup_rows(A, r, R, K, A2, s));
+        }
+        TcGemmArgs a{};
+        a.w = w; a.A0 = dY; a.A1 = dU2; a.B1 = A2; a.Rpad = R;
+        a.p.M = M; a.p.Nout = K; a.p.out = dX; a.p.ldo = K; a.p.out_f32 = (dx_dtype == QLORA_DTYPE_F32);
+        TimerScope t(QLORA_TIMER_DX_MAIN, s);
+        QLORA_TRY(launch_tc_gemm_nf4(a, true, s));
+    } else if (dX) {   // same product on the CUDA cores
         SimtGemm g{};
         g.nseg = 2;
         g.seg[0].a = simt_dense(SIMT_BF16, dY, N, 1);

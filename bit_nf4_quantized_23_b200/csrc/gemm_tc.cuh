@@ -1,0 +1,42 @@
+// Host interface of the tcgen05 fused dequant-GEMM (gemm_tc.cu).
+#pragma once
+
+#include <cuda.h>
+
+#include "qlora_internal.cuh"
+
+namespace qlora {
+
+struct TcGemmParams {
+    int64_t M;              // output rows (tokens)
+    int64_t Nout;           // output columns (N for the forward, K for dX)
+    int32_t ksteps0;        // 64-wide reduction steps over the frozen weight
+    int32_t ksteps1;        // 64-wide reduction steps over the LoRA operands
+    const uint8_t* c1_codes;
+    const float* c2;
+    const float* mu;
+    int64_t WN, WK;         // shape of W
+    void* out;
+    int64_t ldo;
+    int32_t out_f32;
+    uint32_t* err;
+    NF4Tables tb;
+};
+
+struct TcGemmArgs {
+    const qlora_nf4_weight* w;
+    const void* A0;         // X [M,K] (forward) or dY [M,N] (dX), bf16
+    const void* A1;         // U2 or dU2 [M, 2*Rpad], bf16
+    const void* B1;         // B2 [N, 2*Rpad] (forward) or A2 [2*Rpad, K] (dX), bf16
+    int32_t Rpad;           // LoRA rank padded to a multiple of 32
+    TcGemmParams p;
+    CUtensorMap tmA0, tmCodes, tmA1, tmB1;
+};
+
+// Encodes the tensor maps and launches the forward (dx = false) or dX kernel.
+qlora_status launch_tc_gemm_nf4(TcGemmArgs& a, bool dx, cudaStream_t stream);
+
+bool make_tmap_2d(CUtensorMap* map, bool bf16, const void* base, uint64_t inner, uint64_t outer,
+                  uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128);
+
+}  // namespace qlora
