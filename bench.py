@@ -48,6 +48,11 @@ def parse_args():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-decode", action="store_true")
+    p.add_argument("--case", choices=["fwd", "bwd", "quantize", "dequantize"], default=None,
+                   help="profiling mode: run one op of one linear --reps times and exit")
+    p.add_argument("--shape", default="2048,22016,8192", help="M,N,K for --case")
+    p.add_argument("--rank", type=int, default=64, help="LoRA rank for --case")
+    p.add_argument("--reps", type=int, default=3)
     return p.parse_args()
 
 
@@ -474,8 +479,40 @@ def run_ours(args):
     return 0
 
 
+def run_case(args):
+    """Run one op of one linear a few times (for ncu captures); prints device time per call."""
+    import torch
+    import bit_nf4_quantized_23_b200 as q4
+    import synthetic_inputs as si
+    M, N, K = (int(v) for v in args.shape.split(","))
+    r = args.rank
+    W, X, A, B, dY = (t.cuda() for t in si.custom_linear(N, K, M, r, seed=7))
+    w = q4.qlora_quantize_nf4_dq(W)
+    Y, U = q4.qlora_linear_fwd(w, X, A, B, r, 2.0 * r)
+    ops = {
+        "quantize": lambda: q4.qlora_quantize_nf4_dq(W, out=w),
+        "dequantize": lambda: q4.qlora_dequantize(w),
+        "fwd": lambda: q4.qlora_linear_fwd(w, X, A, B, r, 2.0 * r, out=Y, U_out=U),
+        "bwd": lambda: q4.qlora_linear_bwd(w, X, dY, A, B, r, 2.0 * r, U_saved=U),
+    }
+    op = ops[args.case]
+    op()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.reps):
+        op()
+    b.record()
+    b.synchronize()
+    assert q4.qlora_read_device_errors(clear=True) == 0
+    print(json.dumps({"case": args.case, "shape": [M, N, K], "r": r, "ms_per_call": a.elapsed_time(b) / args.reps}))
+    return 0
+
+
 def main():
     args = parse_args()
+    if args.case:
+        return run_case(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

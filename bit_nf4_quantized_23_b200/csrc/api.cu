@@ -1,5 +1,6 @@
 // The C ABI of libqlora.so (declared in include/qlora.h): argument validation
 // on the host, then the kernel launches of each operation.
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstring>
@@ -20,6 +21,11 @@ uint32_t* device_error_word();
 qlora_status launch_split_hi_lo(const float* V, int64_t M, int r, int R, float scale, void* V2, cudaStream_t s);
 qlora_status launch_dup_cols(const void* B, int64_t N, int r, int R, void* B2, cudaStream_t s);
 qlora_status launch_dup_rows(const void* A, int r, int R, int64_t K, void* A2, cudaStream_t s);
+qlora_status launch_transpose_pad(const void* B, int64_t N, int r, int R, void* Bt, cudaStream_t s);
+qlora_status launch_reduce_rows(const float* partial, int splits, int64_t rows, int r, int R, float scale_out,
+                                float* out, float scale_v2, void* V2, cudaStream_t s);
+qlora_status launch_reduce_transposed(const float* partial, int splits, int64_t rows, int r, int R, float* out,
+                                      cudaStream_t s);
 
 namespace {
 
@@ -61,18 +67,20 @@ qlora_status check_lora(int64_t M, int32_t r, float alpha) {
     return QLORA_OK;
 }
 
-// LoRA rank padded to a multiple of 32 (two halves of R give 64-wide reduction steps).
-inline int32_t rank_pad(int32_t r) { return (r + 31) / 32 * 32; }
+// LoRA rank padded to a multiple of 64 (each hi/lo half fills whole 64-wide reduction steps).
+inline int32_t rank_pad(int32_t r) { return (r + 63) / 64 * 64; }
 
 // Workspace of the linear layer (every piece 256-byte aligned):
 //   U   fp32 [M,r]        (when the caller keeps none)
 //   dU  fp32 [M,r]
 //   U2  bf16 [M,2R]       hi/lo split of s*U
-//   B2  bf16 [N,2R]       [B | B]
 //   dU2 bf16 [M,2R]       hi/lo split of dU
+//   B2  bf16 [N,2R]       [B | B]
 //   A2  bf16 [2R,K]       [A ; A]
+//   Bt  bf16 [R,N]        B^T, zero-padded
+//   partial fp32          split-reduction partial sums of the LoRA GEMMs
 struct LinearWs {
-    size_t u_off, du_off, u2_off, b2_off, du2_off, a2_off, total;
+    size_t u_off, du_off, u2_off, du2_off, b2_off, a2_off, bt_off, part_off, total;
 };
 
 LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int32_t r) {
@@ -82,11 +90,28 @@ LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int32_t r) {
     l.u_off = o;   o += align_up((size_t)M * r * sizeof(float), 256);
     l.du_off = o;  o += align_up((size_t)M * r * sizeof(float), 256);
     l.u2_off = o;  o += align_up((size_t)M * 2 * R * 2, 256);
-    l.b2_off = o;  o += align_up((size_t)N * 2 * R * 2, 256);
     l.du2_off = o; o += align_up((size_t)M * 2 * R * 2, 256);
+    l.b2_off = o;  o += align_up((size_t)N * 2 * R * 2, 256);
     l.a2_off = o;  o += align_up(2 * R * (size_t)K * 2, 256);
+    l.bt_off = o;  o += align_up(R * (size_t)N * 2, 256);
+    size_t part = lora_partial_bytes(M, K, (int)R);
+    part = std::max(part, lora_partial_bytes(M, N, (int)R));
+    part = std::max(part, lora_partial_bytes(K, M, (int)R));
+    part = std::max(part, lora_partial_bytes(N, M, (int)R));
+    l.part_off = o; o += align_up(part, 256);
     l.total = o;
     return l;
+}
+
+// U = X A^T on the tensor cores, reduced into U (fp32, may be null) and U2 = hi/lo(s U).
+qlora_status lora_U(const void* X, const void* A2, int64_t M, int64_t K, int32_t r, int32_t R, float s_lora,
+                    float* U, void* U2, float* partial, cudaStream_t s) {
+    TimerScope t(QLORA_TIMER_LORA, s);
+    LoraGemmArgs g{};
+    g.mn_major = false; g.A = X; g.lda = K; g.B = A2; g.ldb = K; g.rows = M; g.red = K; g.R = R; g.partial = partial;
+    QLORA_TRY(launch_lora_gemm(g, s));
+    const int splits = lora_splits(M, (int)((K + 63) / 64));
+    return launch_reduce_rows(partial, splits, M, r, R, 1.f, U, s_lora, U2, s);
 }
 
 }  // namespace
@@ -188,24 +213,16 @@ qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const void* X, int64_t 
     float* U = U_save ? U_save : reinterpret_cast<float*>(ws + lw.u_off);
     const float scale = alpha / (float)r;
     const int32_t R = rank_pad(r);
-
-    SimtGemm g{};
-    g.nseg = 1;
-    g.seg[0].a = simt_dense(SIMT_BF16, X, K, 1);
-    g.seg[0].b = simt_dense(SIMT_BF16, A, K, 1);
-    g.seg[0].K = K; g.seg[0].scale = 1.f;
-    g.M = M; g.N = r; g.C = U; g.c_dtype = QLORA_DTYPE_F32; g.ldc = r;
-    {
-        TimerScope t(QLORA_TIMER_LORA, s);
-        QLORA_TRY(launch_simt_gemm(g, s));
-    }
     void* U2 = ws + lw.u2_off;
     void* B2 = ws + lw.b2_off;
+    void* A2 = ws + lw.a2_off;
+    float* partial = reinterpret_cast<float*>(ws + lw.part_off);
     {
         TimerScope t(QLORA_TIMER_LORA, s);
-        QLORA_TRY(launch_split_hi_lo(U, M, r, R, scale, U2, s));
+        QLORA_TRY(launch_dup_rows(A, r, R, K, A2, s));
         QLORA_TRY(launch_dup_cols(B, N, r, R, B2, s));
     }
+    QLORA_TRY(lora_U(X, A2, M, K, r, R, scale, U, U2, partial, s));
     TcGemmArgs a{};
     a.w = w; a.A0 = X; a.A1 = U2; a.B1 = B2; a.Rpad = R;
     a.p.M = M; a.p.Nout = N; a.p.out = Y; a.p.ldo = N; a.p.out_f32 = (y_dtype == QLORA_DTYPE_F32);
@@ -240,6 +257,58 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const void* X, const vo
     const float scale = alpha / (float)r;
     const int32_t R = rank_pad(r);
 
+    if (N % 8 == 0) {
+        // Tensor-core path (dY rows are 16-byte strided, so dY can be a TMA source).
+        void* U2 = ws + lw.u2_off;
+        void* dU2 = ws + lw.du2_off;
+        void* A2 = ws + lw.a2_off;
+        void* Bt = ws + lw.bt_off;
+        float* dUf = reinterpret_cast<float*>(ws + lw.du_off);
+        float* partial = reinterpret_cast<float*>(ws + lw.part_off);
+        {
+            TimerScope t(QLORA_TIMER_LORA, s);
+            QLORA_TRY(launch_dup_rows(A, r, R, K, A2, s));
+            QLORA_TRY(launch_transpose_pad(B, N, r, R, Bt, s));
+            if (U_saved) QLORA_TRY(launch_split_hi_lo(U_saved, M, r, R, scale, U2, s));
+        }
+        if (!U_saved) QLORA_TRY(lora_U(X, A2, M, K, r, R, scale, nullptr, U2, partial, s));
+        {   // dU = s dY B  ->  dU (fp32) and its hi/lo split
+            TimerScope t(QLORA_TIMER_LORA, s);
+            LoraGemmArgs g{};
+            g.mn_major = false; g.A = dY; g.lda = N; g.B = Bt; g.ldb = N; g.rows = M; g.red = N; g.R = R;
+            g.partial = partial;
+            QLORA_TRY(launch_lora_gemm(g, s));
+            QLORA_TRY(launch_reduce_rows(partial, lora_splits(M, (int)((N + 63) / 64)), M, r, R, scale, dUf, scale,
+                                         dU2, s));
+        }
+        if (dX) {   // dX = dY W_hat + dU A
+            TcGemmArgs a{};
+            a.w = w; a.A0 = dY; a.A1 = dU2; a.B1 = A2; a.Rpad = R;
+            a.p.M = M; a.p.Nout = K; a.p.out = dX; a.p.ldo = K; a.p.out_f32 = (dx_dtype == QLORA_DTYPE_F32);
+            TimerScope t(QLORA_TIMER_DX_MAIN, s);
+            QLORA_TRY(launch_tc_gemm_nf4(a, true, s));
+        }
+        {   // dA = dU^T X, computed as dA^T [K, R] = X^T dU
+            TimerScope t(QLORA_TIMER_LORA, s);
+            LoraGemmArgs g{};
+            g.mn_major = true; g.A = X; g.lda = K; g.B = dU2; g.ldb = 2 * R; g.rows = K; g.red = M; g.R = R;
+            g.partial = partial;
+            QLORA_TRY(launch_lora_gemm(g, s));
+            QLORA_TRY(launch_reduce_transposed(partial, lora_splits(K, (int)((M + 63) / 64)), K, r, R, dA, s));
+        }
+        {   // dB = s dY^T U = dY^T (s U)
+            TimerScope t(QLORA_TIMER_LORA, s);
+            LoraGemmArgs g{};
+            g.mn_major = true; g.A = dY; g.lda = N; g.B = U2; g.ldb = 2 * R; g.rows = N; g.red = M; g.R = R;
+            g.partial = partial;
+            QLORA_TRY(launch_lora_gemm(g, s));
+            QLORA_TRY(launch_reduce_rows(partial, lora_splits(N, (int)((M + 63) / 64)), N, r, R, 1.f, dB, 0.f,
+                                         nullptr, s));
+        }
+        return QLORA_OK;
+    }
+
+    // CUDA-core path for N % 8 != 0.
     const float* U = U_saved;
     if (!U) {
         float* Uw = reinterpret_cast<float*>(ws + lw.u_off);
@@ -264,20 +333,7 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const void* X, const vo
         TimerScope t(QLORA_TIMER_LORA, s);
         QLORA_TRY(launch_simt_gemm(g, s));
     }
-    if (dX && N % 8 == 0) {   // dX = dY W_hat + dU A on the tensor cores (dY rows must be 16-byte strided)
-        void* dU2 = ws + lw.du2_off;
-        void* A2 = ws + lw.a2_off;
-        {
-            TimerScope t(QLORA_TIMER_LORA, s);
-            QLORA_TRY(launch_split_hi_lo(dU, M, r, R, 1.f, dU2, s));
-            QLORA_TRY(launch_dup_rows(A, r, R, K, A2, s));
-        }
-        TcGemmArgs a{};
-        a.w = w; a.A0 = dY; a.A1 = dU2; a.B1 = A2; a.Rpad = R;
-        a.p.M = M; a.p.Nout = K; a.p.out = dX; a.p.ldo = K; a.p.out_f32 = (dx_dtype == QLORA_DTYPE_F32);
-        TimerScope t(QLORA_TIMER_DX_MAIN, s);
-        QLORA_TRY(launch_tc_gemm_nf4(a, true, s));
-    } else if (dX) {   // same product on the CUDA cores
+    if (dX) {   // dX = dY W_hat + dU A on the CUDA cores
         SimtGemm g{};
         g.nseg = 2;
         g.seg[0].a = simt_dense(SIMT_BF16, dY, N, 1);

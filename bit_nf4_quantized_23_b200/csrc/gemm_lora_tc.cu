@@ -1,0 +1,224 @@
+// LoRA-side GEMMs of the QLoRA linear layer on the tcgen05 tensor cores.
+//
+// The low-rank products ("QLoRA 的原理是什么？4-bit 量化权重真的参与训练吗？",
+// section 7: only the LoRA parameters are trained; walkthrough of "QLoRA:
+// Efficient Finetuning of Quantized LLMs", section 4.4: gradients flow through
+// the frozen weight into the adapters) have one dimension of size r:
+//     U  = X  A^T      [M, r]    reduction over K
+//     dU = s dY B      [M, r]    reduction over N
+//     dA = dU^T X      [r, K]    reduction over M   (computed as dA^T [K, r])
+//     dB = s dY^T U    [N, r]    reduction over M
+// Each is a [rows x R] output (R = r padded to a multiple of 64) with a long
+// reduction, so the reduction is split over CTAs (deterministic: every split
+// writes its own fp32 partial tile, a reduce kernel adds them in fixed order).
+//
+// Two operand modes:
+//   K-major  A [rows, red] and B [R, red], both with the reduction contiguous
+//            (X with A, dY with B^T); one MMA per 16-wide step.
+//   MN-major A from S [red, rows] (X or dY, rows contiguous) and B from the
+//            bf16 hi/lo split V2 [red, 2R] of dU or s*U; two MMAs per step
+//            (hi then lo) into the same fp32 accumulator, so the fp32 factor
+//            keeps ~16 significant bits.
+// Roles (192 threads): warp 0 lane 0 TMA, warp 1 TMEM owner + MMA issuer,
+// warps 2-5 epilogue (TMEM -> fp32 partial tile).  No TMA multicast.
+#include <cuda.h>
+
+#include "qlora_internal.cuh"
+#include "tc_ptx.cuh"
+#include "gemm_tc.cuh"
+
+namespace qlora {
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kStages = 2;
+constexpr uint32_t kAStage = 128 * 128;           // 128 rows x 64 bf16
+constexpr uint32_t kBStage = 64 * 1024;           // up to R=256 hi+lo MN-major images
+constexpr uint32_t kOffB = kStages * kAStage;
+constexpr uint32_t kOffBars = kOffB + kStages * kBStage;
+constexpr uint32_t kOffSlot = kOffBars + (2 * kStages + 1) * 8;
+constexpr uint32_t kOffAbort = kOffSlot + 4;
+constexpr uint32_t kSmemAlloc = kOffAbort + 4 + 1024;
+
+template <bool MN>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_lora_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, LoraGemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t base = (ptx::smem_addr(smem_raw) + 1023u) & ~1023u;
+    uint8_t* gbase = smem_raw + (base - ptx::smem_addr(smem_raw));
+    const uint32_t sA = base, sB = base + kOffB;
+    const uint32_t bar_full = base + kOffBars;
+    const uint32_t bar_empty = bar_full + 8 * kStages;
+    const uint32_t bar_acc = bar_empty + 8 * kStages;
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gbase + kOffSlot);
+    volatile int* abort = reinterpret_cast<volatile int*>(gbase + kOffAbort);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int R = p.R;
+    const int64_t row0 = (int64_t)blockIdx.x * 128;
+    const int k_begin = blockIdx.y * p.ksteps_per_split;
+    const int k_end = min(p.ksteps_total, k_begin + p.ksteps_per_split);
+    const int nk = k_end - k_begin;
+    const uint32_t tmem_cols = p.tmem_cols;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            ptx::mbar_init(bar_full + 8 * s, 1);
+            ptx::mbar_init(bar_empty + 8 * s, 1);
+        }
+        ptx::mbar_init(bar_acc, 1);
+        *abort = 0;
+        ptx::fence_barrier_init();
+        ptx::fence_proxy_async_smem();
+        ptx::tma_prefetch_map(&tmA);
+        ptx::tma_prefetch_map(&tmB);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(base + kOffSlot, tmem_cols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const uint32_t b_bytes = MN ? (uint32_t)R * 256u : (uint32_t)R * 128u;
+            for (int i = 0; i < nk; ++i) {
+                const int s = i % kStages;
+                const uint32_t ph = (uint32_t)(i / kStages) & 1u;
+                if (!ptx::mbar_wait(bar_empty + 8 * s, ph ^ 1u, abort, p.err)) break;
+                const uint32_t fb = bar_full + 8 * s;
+                const int ks = k_begin + i;
+                const uint32_t a_dst = sA + s * kAStage, b_dst = sB + s * kBStage;
+                ptx::mbar_arrive_expect_tx(fb, kAStage + b_bytes);
+                if (!MN) {
+                    ptx::tma_load_2d(a_dst, &tmA, ks * 64, (int32_t)row0, fb);
+                    ptx::tma_load_2d(b_dst, &tmB, ks * 64, 0, fb);
+                } else {
+                    ptx::tma_load_2d(a_dst, &tmA, (int32_t)row0, ks * 64, fb);
+                    ptx::tma_load_2d(a_dst + 8192, &tmA, (int32_t)row0 + 64, ks * 64, fb);
+                    const int chunks = R / 64;
+                    for (int c = 0; c < chunks; ++c) {
+                        ptx::tma_load_2d(b_dst + c * 8192, &tmB, c * 64, ks * 64, fb);
+                        ptx::tma_load_2d(b_dst + (chunks + c) * 8192, &tmB, R + c * 64, ks * 64, fb);
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = ptx::idesc_bf16_f32_ab(128, R, MN ? 1 : 0, MN ? 1 : 0);
+            bool ok = true;
+            for (int i = 0; i < nk && ok; ++i) {
+                const int s = i % kStages;
+                const uint32_t ph = (uint32_t)(i / kStages) & 1u;
+                ok = ptx::mbar_wait(bar_full + 8 * s, ph, abort, p.err);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                const uint32_t a_base = sA + s * kAStage, b_base = sB + s * kBStage;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint32_t acc = (i | kk) != 0 ? 1u : 0u;
+                    if (!MN) {
+                        ptx::mma_bf16_ss(tmem, ptx::smem_desc_sw128(a_base + kk * 32, 16, 1024),
+                                         ptx::smem_desc_sw128(b_base + kk * 32, 16, 1024), idesc, acc);
+                    } else {
+                        const uint64_t ad = ptx::smem_desc_sw128(a_base + kk * 2048, 8192, 1024);
+                        ptx::mma_bf16_ss(tmem, ad, ptx::smem_desc_sw128(b_base + kk * 2048, 8192, 1024), idesc, acc);
+                        ptx::mma_bf16_ss(tmem, ad,
+                                         ptx::smem_desc_sw128(b_base + (R / 64) * 8192 + kk * 2048, 8192, 1024),
+                                         idesc, 1u);
+                    }
+                }
+                ptx::mma_commit(bar_empty + 8 * s);
+            }
+            ptx::mma_commit(bar_acc);
+        }
+    } else {
+        const bool acc_ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_acc, 0, abort, p.err));
+        ptx::tc_fence_after();
+        if (acc_ok) {
+            const uint32_t quad = (uint32_t)(warp & 3);
+            const int64_t row = row0 + quad * 32 + lane;
+            float* dst = p.partial + ((int64_t)blockIdx.y * p.rows + row) * R;
+#pragma unroll 1
+            for (int c = 0; c < R / 32; ++c) {
+                uint32_t v[32];
+                ptx::tmem_ld_32x32b_x32(tmem + ((quad * 32u) << 16) + c * 32, v);
+                ptx::tmem_ld_wait();
+                if (row < p.rows) {
+                    uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) d4[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                }
+            }
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, tmem_cols);
+    }
+}
+
+template <bool MN>
+qlora_status launch_lora(const CUtensorMap& tmA, const CUtensorMap& tmB, LoraGemmParams& p, int splits,
+                         cudaStream_t stream) {
+    static bool configured = false;
+    auto kern = tc_lora_gemm<MN>;
+    if (!configured) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemAlloc) != cudaSuccess)
+            return QLORA_ERR_CUDA;
+        configured = true;
+    }
+    const dim3 grid((unsigned)((p.rows + 127) / 128), (unsigned)splits);
+    kern<<<grid, kThreads, kSmemAlloc, stream>>>(tmA, tmB, p);
+    QLORA_CHECK_LAUNCH();
+    return QLORA_OK;
+}
+
+}  // namespace
+
+int lora_splits(int64_t rows, int ksteps_total) {
+    const int64_t tiles = (rows + 127) / 128;
+    int64_t splits = (2 * 148 + tiles - 1) / tiles;
+    if (splits > ksteps_total) splits = ksteps_total;
+    if (splits < 1) splits = 1;
+    const int64_t kps = (ksteps_total + splits - 1) / splits;
+    return (int)((ksteps_total + kps - 1) / kps);
+}
+
+qlora_status launch_lora_gemm(const LoraGemmArgs& a, cudaStream_t stream) {
+    LoraGemmParams p{};
+    p.rows = a.rows;
+    p.R = a.R;
+    p.ksteps_total = (int)((a.red + 63) / 64);
+    const int splits = lora_splits(a.rows, p.ksteps_total);
+    p.ksteps_per_split = (p.ksteps_total + splits - 1) / splits;
+    p.partial = a.partial;
+    p.tmem_cols = a.R <= 64 ? 64u : (a.R <= 128 ? 128u : 256u);
+    p.err = device_error_word();
+    if (!p.err) return QLORA_ERR_CUDA;
+    CUtensorMap tmA, tmB;
+    if (!a.mn_major) {
+        // A [rows, red] and B [R, red], reduction contiguous
+        if (!make_tmap_2d(&tmA, true, a.A, a.red, a.rows, a.lda * 2, 64, 128, true)) return QLORA_ERR_CUDA;
+        if (!make_tmap_2d(&tmB, true, a.B, a.red, a.R, a.ldb * 2, 64, (uint32_t)a.R, true)) return QLORA_ERR_CUDA;
+        return launch_lora<false>(tmA, tmB, p, splits, stream);
+    }
+    // S [red, rows] with rows contiguous, V2 [red, 2R] (hi | lo)
+    if (!make_tmap_2d(&tmA, true, a.A, a.rows, a.red, a.lda * 2, 64, 64, true)) return QLORA_ERR_CUDA;
+    if (!make_tmap_2d(&tmB, true, a.B, 2 * (uint64_t)a.R, a.red, a.ldb * 2, 64, 64, true)) return QLORA_ERR_CUDA;
+    return launch_lora<true>(tmA, tmB, p, splits, stream);
+}
+
+size_t lora_partial_bytes(int64_t rows, int64_t red, int R) {
+    const int ks = (int)((red + 63) / 64);
+    return (size_t)lora_splits(rows, ks) * (size_t)rows * (size_t)R * sizeof(float);
+}
+
+}  // namespace qlora

@@ -234,37 +234,56 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
         }
     } else {
         // ------------------------------------------------------------ dequant producers
+        // Unit u of thread t: forward: B row (t + 128u), i.e. W row n0 + row, K-block it;
+        // dX: W row it*64 + (t & 63), K-block (n0 + 64*kc)/64 with kc = (t >> 6) + 2u.
+        // The block constants of step it+1 are loaded while step it is expanded.
         const int t = threadIdx.x - 64;        // 0..127
         const float mu = *p.mu;
         const int64_t blocks_per_row = p.WK / 64;
+        uint32_t row_u[2], img_u[2], kc_u[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            if (!DX) {
+                row_u[u] = (uint32_t)(t + 128 * u);
+                img_u[u] = row_u[u] * 128u;
+                kc_u[u] = 0;
+            } else {
+                row_u[u] = (uint32_t)(t & 63);
+                kc_u[u] = (uint32_t)((t >> 6) + 2 * u);
+                img_u[u] = kc_u[u] * 8192u + row_u[u] * 128u;
+            }
+        }
+        // block index of unit u at step it, or -1 when the unit lies outside W
+        auto unit_block = [&](int u, int it) -> int64_t {
+            const int64_t n = DX ? (int64_t)it * 64 + row_u[u] : n0 + row_u[u];
+            const int64_t k = DX ? n0 + (int64_t)kc_u[u] * 64 : (int64_t)it * 64;
+            return (n < p.WN && k < p.WK) ? n * blocks_per_row + (k >> 6) : -1;
+        };
+        uint32_t code_nx[2] = {0, 0};
+        float c2_nx[2] = {0.f, 0.f};
+        int64_t blk_nx[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            blk_nx[u] = ks0 > 0 ? unit_block(u, 0) : -1;
+            if (blk_nx[u] >= 0) {
+                code_nx[u] = __ldg(p.c1_codes + blk_nx[u]);
+                c2_nx[u] = __ldg(p.c2 + (blk_nx[u] >> 8));
+            }
+        }
         bool ok = true;
         for (int it = 0; it < ks0 && ok; ++it) {
             const int s = it % kStages;
             const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-            // per-unit block constants (global loads issued before the wait)
-            int64_t n_u[2], k_u[2];
-            uint32_t row_u[2], img_u[2];
-            bool valid_u[2];
+            int64_t blk_cur[2];
             float c1p_u[2];
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
-                if (!DX) {
-                    row_u[u] = (uint32_t)(t + 128 * u);      // B row = n - n0
-                    img_u[u] = row_u[u] * 128u;
-                    n_u[u] = n0 + row_u[u];
-                    k_u[u] = (int64_t)it * 64;
-                } else {
-                    const uint32_t nl = (uint32_t)(t & 63), kc = (uint32_t)((t >> 6) + 2 * u);
-                    row_u[u] = nl;
-                    img_u[u] = kc * 8192u + nl * 128u;
-                    n_u[u] = (int64_t)it * 64 + nl;
-                    k_u[u] = n0 + kc * 64;
-                }
-                valid_u[u] = (n_u[u] < p.WN) && (k_u[u] < p.WK);
-                c1p_u[u] = 0.f;
-                if (valid_u[u]) {
-                    const int64_t blk = n_u[u] * blocks_per_row + (k_u[u] >> 6);
-                    c1p_u[u] = rebuild_c1(__ldg(p.c1_codes + blk), __ldg(p.c2 + (blk >> 8)), mu);
+                blk_cur[u] = blk_nx[u];
+                c1p_u[u] = blk_cur[u] >= 0 ? rebuild_c1(code_nx[u], c2_nx[u], mu) : 0.f;
+                blk_nx[u] = (it + 1 < ks0) ? unit_block(u, it + 1) : -1;
+                if (blk_nx[u] >= 0) {
+                    code_nx[u] = __ldg(p.c1_codes + blk_nx[u]);
+                    c2_nx[u] = __ldg(p.c2 + (blk_nx[u] >> 8));
                 }
             }
             ok = ptx::mbar_wait(bar_full_a + 8 * s, ph, abort, p.err);
@@ -275,7 +294,7 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
                 const uint32_t row_addr = b_base + img_u[u];
-                if (!valid_u[u]) {
+                if (blk_cur[u] < 0) {
                     zero_row(row_addr);
                     continue;
                 }
@@ -290,10 +309,9 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
                     c1 = first ? x : y;
                 } else {
                     // codes tile: 64 rows x 128 bytes, 128-byte swizzled; this unit's 32 bytes are chunks 2kc, 2kc+1
-                    const uint32_t kc = (uint32_t)((t >> 6) + 2 * u);
                     const uint32_t src = c_base + row_u[u] * 128u;
-                    c0 = ld_shared_v4(src + (((2u * kc) ^ (row_u[u] & 7u)) << 4));
-                    c1 = ld_shared_v4(src + (((2u * kc + 1u) ^ (row_u[u] & 7u)) << 4));
+                    c0 = ld_shared_v4(src + (((2u * kc_u[u]) ^ (row_u[u] & 7u)) << 4));
+                    c1 = ld_shared_v4(src + (((2u * kc_u[u] + 1u) ^ (row_u[u] & 7u)) << 4));
                 }
                 Lut lut;
                 build_lut(lut, c1p_u[u], p.tb);

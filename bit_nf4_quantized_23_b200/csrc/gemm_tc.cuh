@@ -36,6 +36,33 @@ struct TcGemmArgs {
 // Encodes the tensor maps and launches the forward (dx = false) or dX kernel.
 qlora_status launch_tc_gemm_nf4(TcGemmArgs& a, bool dx, cudaStream_t stream);
 
+// LoRA-side GEMM (gemm_lora_tc.cu): partial[split][rows][R] = sum over the
+// split's share of the reduction of A-operand rows times B-operand rows.
+struct LoraGemmParams {
+    int64_t rows;
+    int32_t R;
+    int32_t ksteps_total;
+    int32_t ksteps_per_split;
+    uint32_t tmem_cols;
+    float* partial;
+    uint32_t* err;
+};
+
+struct LoraGemmArgs {
+    bool mn_major;     // false: A [rows, red] (lda), B [R, red] (ldb); true: A from S [red, rows], B from V2 [red, 2R]
+    const void* A;
+    int64_t lda;
+    const void* B;
+    int64_t ldb;
+    int64_t rows, red;
+    int32_t R;
+    float* partial;
+};
+
+qlora_status launch_lora_gemm(const LoraGemmArgs& a, cudaStream_t stream);
+int lora_splits(int64_t rows, int ksteps_total);
+size_t lora_partial_bytes(int64_t rows, int64_t red, int R);
+
 bool make_tmap_2d(CUtensorMap* map, bool bf16, const void* base, uint64_t inner, uint64_t outer,
                   uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128);
 

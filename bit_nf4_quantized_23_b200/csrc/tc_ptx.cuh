@@ -155,11 +155,15 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
            ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
-// Instruction descriptor of kind::f16 with bf16 A and B, fp32 D, A K-major,
-// B K-major (b_mn = 0) or MN-major (b_mn = 1), shape M x N.
+// Instruction descriptor of kind::f16 with bf16 A and B, fp32 D, shape M x N;
+// A and B each K-major (0) or MN-major (1).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_ab(int M, int N, int a_mn, int b_mn) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int b_mn) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)b_mn << 16) | ((uint32_t)(N >> 3) << 17) |
-           ((uint32_t)(M >> 4) << 24);
+    return idesc_bf16_f32_ab(M, N, 0, b_mn);
 }
 
 }  // namespace ptx

@@ -173,7 +173,8 @@ def test_tiny_workload_full():
 
 
 @pytest.mark.parametrize("M,N,K,r", [(1, 64, 64, 1), (3, 192, 128, 5), (17, 320, 192, 16),
-                                     (130, 96, 640, 64), (33, 128, 256, 256)])
+                                     (130, 96, 640, 64), (33, 128, 256, 256), (5, 100, 128, 3),
+                                     (300, 520, 1088, 96), (257, 264, 320, 200)])
 def test_ragged_linear(M, N, K, r):
     W, X, A, B, dY = si.custom_linear(N, K, M, r, seed=M + N + K + r)
     check_linear_full(W, X, A, B, dY, r, alpha=2.0 * r)
