@@ -41,7 +41,7 @@ PACKED_BYTES_PER_WEIGHT = 0.5 + 1 / 64 + 4 / (64 * 256)     # codes + E4M3 const
 def parse_args():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="block65b")
@@ -78,56 +78,66 @@ def step_flops(wl, M):
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi sampled every 200 ms while the timed region runs."""
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event reasons sampled through NVML every 5 ms while the
+    timed region runs (the region can be far shorter than nvidia-smi's interval)."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.file = None
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.samples = []
+        self.max_mhz = None
+        self._stop = None
+        self._thread = None
+        self.error = None
+
+    def _handle(self, pynvml):
+        import torch
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            return pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(self.dev)
 
     def start(self):
+        import threading
         try:
-            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}", "--format=csv,noheader",
-                 "-lms", "200"], stdout=self.file, stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+            import pynvml
+            pynvml.nvmlInit()
+            h = self._handle(pynvml)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+        except Exception as e:          # no NVML: report why
+            self.error = f"nvml unavailable: {e}"
+            return
+        self._stop = threading.Event()
+
+        def run():
+            while not self._stop.is_set():
+                try:
+                    clk = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                    rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    self.samples.append((float(clk), int(rs)))
+                except Exception as e:
+                    self.error = str(e)
+                self._stop.wait(0.005)
+
+        self._thread = threading.Thread(target=run, daemon=True)
+        self._thread.start()
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.file.flush()
-        with open(self.file.name) as f:
-            rows = [ln.strip().split(", ") for ln in f if ln.strip()]
-        os.unlink(self.file.name)
-        sm, mx, reasons, util = [], None, set(), []
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
-            if len(r) < 10:
-                continue
-            try:
-                clk = float(r[1].split()[0])
-                mx = float(r[2].split()[0])
-                u = float(r[4].split()[0])
-            except ValueError:
-                continue
-            util.append(u)
-            if u >= 50:
-                sm.append(clk)
-                for name, v in zip(names, r[6:10]):
-                    if v.strip().lower() == "active":
-                        reasons.add(name)
-        sm_med = sorted(sm)[len(sm) // 2] if sm else None
-        return {"sm_mhz": sm_med, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples_under_load": len(sm)}
+        if self._thread is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.error or "not sampled"]}
+        self._stop.set()
+        self._thread.join(timeout=2)
+        clks = sorted(c for c, _ in self.samples)
+        reasons = set()
+        for _, rs in self.samples:
+            for bit, name in self.REASONS.items():
+                if rs & bit:
+                    reasons.add(name)
+        return {"sm_mhz": clks[len(clks) // 2] if clks else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(clks),
+                "sm_mhz_min": clks[0] if clks else None, "source": "NVML, every 5 ms during the timed steps"}
 
 
 # ----------------------------------------------------------------------------- traffic from ncu
@@ -310,7 +320,8 @@ def timed_steps(step, steps, flush, stream):
 
 
 def decode_sweep(device, peaks):
-    """Small-M forward on the decode shapes: HBM GB/s over packed NF4 + DQ constant bytes."""
+    """Small-M forward on the decode shapes: HBM GB/s over packed NF4 + DQ constant bytes, for the
+    whole forward call and for the weight-streaming kernel alone (live CUDA events)."""
     import torch
     import bit_nf4_quantized_23_b200 as q4
     import synthetic_inputs as si
@@ -329,24 +340,58 @@ def decode_sweep(device, peaks):
             Y = torch.empty(M, N, dtype=torch.bfloat16, device=device)
             lws = torch.empty(max(16, q4.qlora_linear_workspace_size(M, N, K, wl.r)), dtype=torch.uint8,
                               device=device)
+            call = lambda j: q4.qlora_linear_fwd(ws[j % copies], X, A, B, wl.r, wl.alpha, out=Y, save_U=False,
+                                                 workspace=lws)
             for j in range(3):
-                q4.qlora_linear_fwd(ws[j % copies], X, A, B, wl.r, wl.alpha, out=Y, save_U=False, workspace=lws)
-            reps = 4 * copies
+                call(j)
+            reps = 8 * copies
+            torch.cuda.synchronize()
+            q4.qlora_timing_read("decode", reset=True)
+            q4.qlora_timing_enable(True)
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
-            torch.cuda.synchronize()
             a.record()
             for j in range(reps):
-                q4.qlora_linear_fwd(ws[j % copies], X, A, B, wl.r, wl.alpha, out=Y, save_U=False, workspace=lws)
+                call(j)
             b.record()
             b.synchronize()
+            q4.qlora_timing_enable(False)
+            n_k, ms_k = q4.qlora_timing_read("decode", reset=True)
             ms = a.elapsed_time(b) / reps
-            gbs = wbytes / (ms * 1e-3) / 1e9
-            out[f"W[{N},{K}] M={M}"] = {"us_per_call": round(ms * 1e3, 2), "GB/s": round(gbs, 1),
-                                        "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 3)}
+            kms = ms_k / max(1, n_k)
+            out[f"W[{N},{K}] M={M}"] = {
+                "call_us": round(ms * 1e3, 2), "call_GB/s": round(wbytes / (ms * 1e-3) / 1e9, 1),
+                "kernel_us": round(kms * 1e3, 2), "kernel_GB/s": round(wbytes / (kms * 1e-3) / 1e9, 1),
+                "kernel_frac_of_hbm": round(wbytes / (kms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3)}
         del ws
         torch.cuda.empty_cache()
     return out
+
+
+def dequant_rate(device, peaks, wl):
+    """qlora_dequantize on the largest weight of the workload: GB/s over 0.516 B in + 2 B out per weight."""
+    import torch
+    import bit_nf4_quantized_23_b200 as q4
+    import synthetic_inputs as si
+    i = max(range(len(wl.linears)), key=lambda j: wl.linears[j][0] * wl.linears[j][1])
+    N, K = wl.linears[i]
+    w = q4.qlora_quantize_nf4_dq(si.weight(wl, i).to(device))
+    out = torch.empty(N, K, dtype=torch.bfloat16, device=device)
+    for _ in range(3):
+        q4.qlora_dequantize(w, out=out)
+    reps = 20
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(reps):
+        q4.qlora_dequantize(w, out=out)
+    b.record()
+    b.synchronize()
+    ms = a.elapsed_time(b) / reps
+    gbs = (PACKED_BYTES_PER_WEIGHT + 2.0) * N * K / (ms * 1e-3) / 1e9
+    return {"shape": [N, K], "us": round(ms * 1e3, 1), "GB/s": round(gbs, 1),
+            "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 3),
+            "bytes_per_weight": round(PACKED_BYTES_PER_WEIGHT + 2.0, 6)}
 
 
 def run_ours(args):
@@ -448,10 +493,17 @@ def run_ours(args):
         e2e = {"value": flops_rank * world / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
 
+    quant_bytes = sum((2.0 + PACKED_BYTES_PER_WEIGHT) * L.N * L.K for L in lins)
+    q_ms = kinds["quantize"][1] / args.steps
+    hbm = {"quantize": {"GB/s": round(quant_bytes / (q_ms * 1e-3) / 1e9, 1),
+                        "frac_of_hbm": round(quant_bytes / (q_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3),
+                        "ms_per_step": round(q_ms, 4), "bytes_per_weight": round(2.0 + PACKED_BYTES_PER_WEIGHT, 6),
+                        "source": "live CUDA events over the timed steps (7 calls per step)"}}
     decode = None
     if rank == 0 and not args.no_decode:
         del lins
         torch.cuda.empty_cache()
+        hbm["dequantize"] = dequant_rate(device, peaks, wl)
         decode = decode_sweep(device, peaks)
 
     cpu = None
@@ -474,7 +526,7 @@ def run_ours(args):
                        "step": "quantize all 7 weights + fwd + bwd of all 7 linears"
                                + (" + NCCL all-reduce of dA/dB" if world > 1 else "")},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
-            "clocks": clk, "kernels": breakdown, "decode_small_m": decode}
+            "clocks": clk, "kernels": breakdown, "hbm_bound_ops": hbm, "decode_small_m": decode}
     print(json.dumps(line), flush=True)
     return 0
 

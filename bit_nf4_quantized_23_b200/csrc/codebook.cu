@@ -13,6 +13,8 @@
 // (Handbook of Mathematical Functions) as a starting point, refined by Newton
 // steps on Phi(x) = erfc(-x / sqrt(2)) / 2 until the step vanishes.
 #include <cmath>
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "qlora_internal.cuh"
@@ -72,7 +74,51 @@ NF4Tables build_tables() {
     return tb;
 }
 
+// Bucket table of the quantize kernel (see QuantBuckets): for each sign and
+// bucket, the code of the bucket's lowest x and the one threshold inside it.
+QuantBuckets build_buckets(const NF4Tables& tb) {
+    QuantBuckets qb;
+    for (int sign = 0; sign < 2; ++sign) {
+        for (int k = 0; k < 42; ++k) {
+            float thr = INFINITY;
+            int base = 7;
+            if (k > 0) {
+                const uint32_t lo_bits = (uint32_t)(k - 1 + 0x3D0) << 20;    // |x| range [lo, hi)
+                const uint32_t hi_bits = (uint32_t)(k + 0x3D0) << 20;
+                float lo, hi;
+                std::memcpy(&lo, &lo_bits, 4);
+                std::memcpy(&hi, &hi_bits, 4);
+                base = 0;
+                int inside = 0;
+                for (int j = 0; j < 15; ++j) {
+                    const float t = tb.t[j];
+                    if (sign == 0) {          // x in [lo, hi)
+                        if (t < lo) ++base;
+                        else if (t < hi) { thr = t; ++inside; }
+                    } else {                  // x in (-hi, -lo]
+                        if (t <= -hi) ++base;
+                        else if (t <= -lo) { thr = t; ++inside; }
+                    }
+                }
+                if (inside > 1) std::abort();   // the bucket width is below every threshold gap
+            }
+            int32_t b = base;
+            float bf;
+            std::memcpy(&bf, &b, 4);
+            qb.e[sign * 42 + k] = make_float2(thr, bf);
+        }
+    }
+    return qb;
+}
+
 }  // namespace
+
+const QuantBuckets& host_buckets() {
+    static std::once_flag once;
+    static QuantBuckets qb;
+    std::call_once(once, [] { qb = build_buckets(host_tables()); });
+    return qb;
+}
 
 const NF4Tables& host_tables() {
     static std::once_flag once;

@@ -21,11 +21,11 @@
 //            apart), written either by the dequant warps from the NF4 codes
 //            or by TMA for the LoRA segment: the two give identical images;
 //   codes    the packed 4-bit codes of the B stage (8 KiB), loaded by TMA.
-// Warp roles (192 threads): warp 0 lane 0 issues TMA; warp 1 owns TMEM and
-// its lane 0 issues tcgen05.mma; warps 2-5 expand NF4 -> bf16 (one NF4 block
-// of 64 weights per unit, through a 16-entry per-block lookup table held in
-// byte-split registers and selected with byte permutes), then run the
-// epilogue (TMEM -> registers -> global, bf16 or fp32).
+// Warp roles (320 threads): warp 0 lane 0 issues TMA; warp 1 owns TMEM and
+// its lane 0 issues tcgen05.mma; warps 2-9 expand NF4 -> bf16 (one NF4 block
+// of 64 weights per thread and K-step, through a 16-entry per-block lookup
+// table held in byte-split registers and selected with byte permutes), then
+// run the epilogue (TMEM -> registers -> global, bf16 or fp32).
 // No TMA multicast is used anywhere.
 #include <cuda.h>
 
@@ -38,7 +38,10 @@ namespace {
 
 constexpr int kBN = 256;
 constexpr int kStages = 3;
-constexpr int kThreads = 192;
+constexpr int kThreads = 192;                 // decode kernel: TMA warp, MMA warp, 4 producer/epilogue warps
+constexpr int kProducerWarps = 8;             // fused GEMM: 8 producer/epilogue warps
+constexpr int kGemmThreads = 64 + 32 * kProducerWarps;
+constexpr int kGemmPrefetch = 2;              // block constants are loaded this many K-steps ahead
 constexpr uint32_t kBStageBytes = 256 * 128;
 constexpr uint32_t kCodesStageBytes = 8192;
 
@@ -84,22 +87,24 @@ __device__ __forceinline__ void build_lut(Lut& t, float c1p, const NF4Tables& tb
 }
 
 // 8 codes (4 packed bytes, element 2j in the high nibble of byte j) -> 8 bf16.
+// The nibbles of w run e1, e0, e3, e2, ... from the least significant end; the
+// table permutes keep that pair-swapped order and the final interleave undoes
+// it.  Bytes whose code is >= 8 take entries 8-15 (sign-replicated bit 3).
 __device__ __forceinline__ uint4 expand8(uint32_t w, const Lut& t) {
-    const uint32_t s = ((w >> 4) & 0x0F0F0F0Fu) | ((w << 4) & 0xF0F0F0F0u);   // nibble i = element i
+    const uint32_t u = w << 4;             // bit 3 of the low nibble of each byte -> that byte's bit 7
     uint32_t o[4];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-        const uint32_t sh = s >> (16 * h);
-        const uint32_t sel = sh & 0x7777u;
-        const uint32_t mask = prmt(sh << 4, sh, 0xD9C8);    // 0xFF bytes where code >= 8 (sign replicate)
+        const uint32_t sel = (w >> (16 * h)) & 0x7777u;
+        const uint32_t mask = prmt(u, w, h == 0 ? 0xD9C8u : 0xFBEAu);
         const uint32_t la = prmt(t.L[0], t.L[1], sel);
         const uint32_t lb = prmt(t.L[2], t.L[3], sel);
         const uint32_t ha = prmt(t.H[0], t.H[1], sel);
         const uint32_t hb = prmt(t.H[2], t.H[3], sel);
         const uint32_t lo = (la & ~mask) | (lb & mask);
         const uint32_t hi = (ha & ~mask) | (hb & mask);
-        o[2 * h] = prmt(lo, hi, 0x5140);
-        o[2 * h + 1] = prmt(lo, hi, 0x7362);
+        o[2 * h] = prmt(lo, hi, 0x4051);
+        o[2 * h + 1] = prmt(lo, hi, 0x6273);
     }
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
@@ -131,7 +136,7 @@ __device__ __forceinline__ void zero_row(uint32_t row_addr) {
 }
 
 template <int NUM_ACC, bool DX>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kGemmThreads, 1)
 tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmCodes,
             const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1, TcGemmParams p) {
     using L = Layout<NUM_ACC>;
@@ -154,7 +159,7 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             ptx::mbar_init(bar_full_a + 8 * s, 1);
-            ptx::mbar_init(bar_full_b + 8 * s, 4);
+            ptx::mbar_init(bar_full_b + 8 * s, kProducerWarps);
             ptx::mbar_init(bar_empty + 8 * s, 1);
         }
         ptx::mbar_init(bar_acc, 1);
@@ -234,88 +239,79 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
         }
     } else {
         // ------------------------------------------------------------ dequant producers
-        // Unit u of thread t: forward: B row (t + 128u), i.e. W row n0 + row, K-block it;
-        // dX: W row it*64 + (t & 63), K-block (n0 + 64*kc)/64 with kc = (t >> 6) + 2u.
-        // The block constants of step it+1 are loaded while step it is expanded.
-        const int t = threadIdx.x - 64;        // 0..127
+        // Thread t (0..255) owns one unit per K-step: forward: B row t = W row n0 + t, K-block it;
+        // dX: W row it*64 + (t & 63), K-block (n0 + 64*kc)/64 with kc = t >> 6.
+        // The block constants are loaded kGemmPrefetch K-steps ahead (register queue).
+        const int t = threadIdx.x - 64;
         const float mu = *p.mu;
         const int64_t blocks_per_row = p.WK / 64;
-        uint32_t row_u[2], img_u[2], kc_u[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            if (!DX) {
-                row_u[u] = (uint32_t)(t + 128 * u);
-                img_u[u] = row_u[u] * 128u;
-                kc_u[u] = 0;
-            } else {
-                row_u[u] = (uint32_t)(t & 63);
-                kc_u[u] = (uint32_t)((t >> 6) + 2 * u);
-                img_u[u] = kc_u[u] * 8192u + row_u[u] * 128u;
-            }
-        }
-        // block index of unit u at step it, or -1 when the unit lies outside W
-        auto unit_block = [&](int u, int it) -> int64_t {
-            const int64_t n = DX ? (int64_t)it * 64 + row_u[u] : n0 + row_u[u];
-            const int64_t k = DX ? n0 + (int64_t)kc_u[u] * 64 : (int64_t)it * 64;
+        const uint32_t row = DX ? (uint32_t)(t & 63) : (uint32_t)t;
+        const uint32_t kc = DX ? (uint32_t)(t >> 6) : 0u;
+        const uint32_t img = DX ? kc * 8192u + row * 128u : row * 128u;
+        auto unit_block = [&](int it) -> int64_t {
+            const int64_t n = DX ? (int64_t)it * 64 + row : n0 + row;
+            const int64_t k = DX ? n0 + (int64_t)kc * 64 : (int64_t)it * 64;
             return (n < p.WN && k < p.WK) ? n * blocks_per_row + (k >> 6) : -1;
         };
-        uint32_t code_nx[2] = {0, 0};
-        float c2_nx[2] = {0.f, 0.f};
-        int64_t blk_nx[2];
+        int64_t qblk[kGemmPrefetch];
+        uint32_t qcode[kGemmPrefetch];
+        float qc2[kGemmPrefetch];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            blk_nx[u] = ks0 > 0 ? unit_block(u, 0) : -1;
-            if (blk_nx[u] >= 0) {
-                code_nx[u] = __ldg(p.c1_codes + blk_nx[u]);
-                c2_nx[u] = __ldg(p.c2 + (blk_nx[u] >> 8));
+        for (int d = 0; d < kGemmPrefetch; ++d) {
+            qblk[d] = d < ks0 ? unit_block(d) : -1;
+            qcode[d] = 0;
+            qc2[d] = 0.f;
+            if (qblk[d] >= 0) {
+                qcode[d] = __ldg(p.c1_codes + qblk[d]);
+                qc2[d] = __ldg(p.c2 + (qblk[d] >> 8));
             }
         }
         bool ok = true;
         for (int it = 0; it < ks0 && ok; ++it) {
             const int s = it % kStages;
             const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-            int64_t blk_cur[2];
-            float c1p_u[2];
+            const int64_t blk = qblk[0];
+            const float c1p = blk >= 0 ? rebuild_c1(qcode[0], qc2[0], mu) : 0.f;
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                blk_cur[u] = blk_nx[u];
-                c1p_u[u] = blk_cur[u] >= 0 ? rebuild_c1(code_nx[u], c2_nx[u], mu) : 0.f;
-                blk_nx[u] = (it + 1 < ks0) ? unit_block(u, it + 1) : -1;
-                if (blk_nx[u] >= 0) {
-                    code_nx[u] = __ldg(p.c1_codes + blk_nx[u]);
-                    c2_nx[u] = __ldg(p.c2 + (blk_nx[u] >> 8));
+            for (int d = 0; d + 1 < kGemmPrefetch; ++d) {
+                qblk[d] = qblk[d + 1];
+                qcode[d] = qcode[d + 1];
+                qc2[d] = qc2[d + 1];
+            }
+            {
+                const int ahead = it + kGemmPrefetch;
+                const int64_t b = ahead < ks0 ? unit_block(ahead) : -1;
+                qblk[kGemmPrefetch - 1] = b;
+                if (b >= 0) {
+                    qcode[kGemmPrefetch - 1] = __ldg(p.c1_codes + b);
+                    qc2[kGemmPrefetch - 1] = __ldg(p.c2 + (b >> 8));
                 }
             }
-            ok = ptx::mbar_wait(bar_full_a + 8 * s, ph, abort, p.err);
-            ok = __all_sync(0xffffffffu, ok);          // leave the loop as a whole warp
+            ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_full_a + 8 * s, ph, abort, p.err));
             if (!ok) break;
-            const uint32_t b_base = sB + s * kBStageBytes;
-            const uint32_t c_base = sCodes + s * kCodesStageBytes;
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const uint32_t row_addr = b_base + img_u[u];
-                if (blk_cur[u] < 0) {
-                    zero_row(row_addr);
-                    continue;
-                }
+            const uint32_t row_addr = sB + s * kBStageBytes + img;
+            if (blk < 0) {
+                zero_row(row_addr);
+            } else {
+                const uint32_t c_base = sCodes + s * kCodesStageBytes;
                 uint4 c0, c1;
                 if (!DX) {
                     // codes tile: 256 rows x 32 bytes, unswizzled; stagger the two halves to avoid bank conflicts
-                    const uint32_t src = c_base + row_u[u] * 32u;
-                    const uint32_t first = (row_u[u] >> 2) & 1u;
+                    const uint32_t src = c_base + row * 32u;
+                    const uint32_t first = (row >> 2) & 1u;
                     const uint4 x = ld_shared_v4(src + first * 16u);
                     const uint4 y = ld_shared_v4(src + (first ^ 1u) * 16u);
                     c0 = first ? y : x;
                     c1 = first ? x : y;
                 } else {
                     // codes tile: 64 rows x 128 bytes, 128-byte swizzled; this unit's 32 bytes are chunks 2kc, 2kc+1
-                    const uint32_t src = c_base + row_u[u] * 128u;
-                    c0 = ld_shared_v4(src + (((2u * kc_u[u]) ^ (row_u[u] & 7u)) << 4));
-                    c1 = ld_shared_v4(src + (((2u * kc_u[u] + 1u) ^ (row_u[u] & 7u)) << 4));
+                    const uint32_t src = c_base + row * 128u;
+                    c0 = ld_shared_v4(src + (((2u * kc) ^ (row & 7u)) << 4));
+                    c1 = ld_shared_v4(src + (((2u * kc + 1u) ^ (row & 7u)) << 4));
                 }
                 Lut lut;
-                build_lut(lut, c1p_u[u], p.tb);
-                expand_block_row(row_addr, row_u[u] & 7u, c0, c1, lut);
+                build_lut(lut, c1p, p.tb);
+                expand_block_row(row_addr, row & 7u, c0, c1, lut);
             }
             ptx::fence_proxy_async_smem();
             __syncwarp();
@@ -323,15 +319,18 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
         }
 
         // ------------------------------------------------------------ epilogue
+        // Warp w reads TMEM lane quadrant (w & 3); the two warps of a quadrant split the columns.
         const bool acc_ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_acc, 0, abort, p.err));
         ptx::tc_fence_after();
         if (acc_ok) {
             const uint32_t quad = (uint32_t)(warp & 3);
+            const int half = (warp - 2) >> 2;                 // 0 or 1
 #pragma unroll 1
             for (int h = 0; h < NUM_ACC; ++h) {
                 const int64_t m = m0 + h * 128 + quad * 32 + lane;
 #pragma unroll 1
-                for (int c = 0; c < kBN / 32; ++c) {
+                for (int cc = 0; cc < kBN / 64; ++cc) {
+                    const int c = half * (kBN / 64) + cc;
                     const int64_t nb = n0 + c * 32;
                     if (nb >= p.Nout) break;
                     uint32_t v[32];
@@ -379,6 +378,238 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
     }
 }
 
+// ---------------------------------------------------------------------------- small-M forward
+//
+// Y[M,N] for M <= 16 tokens (decode), "swap-AB": D[n, m] = W_hat[n, :] X[m, :]^T
+// with the dequantized weight as the 128-row MMA operand A (K-major image
+// written by the producer warps) and the tokens as a 16-wide operand B (TMA).
+// The codes stream through a deep ring (weight bytes dominate the traffic);
+// the reduction over K is split across CTAs so every SM streams.  Split s
+// writes fp32 partial[s][m][n] (or Y directly when there is one split); the
+// LoRA steps run in split 0.
+constexpr int kDecCodeStages = 12;              // packed-code ring (the HBM stream)
+constexpr int kDecStages = 3;                   // dequantized-tile / token ring
+constexpr int kDecPrefetch = 4;                 // block constants are loaded this many K-steps ahead
+constexpr uint32_t kDecAStage = 128 * 128;      // W_hat or B2 tile [128 rows x 64]
+constexpr uint32_t kDecBStage = 16 * 128;       // X or U2 tile [16 tokens x 64]
+constexpr uint32_t kDecCodesStage = 128 * 32;   // packed codes [128 rows x 32 bytes]
+constexpr uint32_t kDecOffB = kDecStages * kDecAStage;
+constexpr uint32_t kDecOffCodes = kDecOffB + kDecStages * kDecBStage;
+constexpr uint32_t kDecOffBars = kDecOffCodes + kDecCodeStages * kDecCodesStage;
+// barriers: cfull[CS], cempty[CS], bfull[S], afull[S], aempty[S], acc
+constexpr uint32_t kDecOffSlot = kDecOffBars + (2 * kDecCodeStages + 3 * kDecStages + 1) * 8;
+constexpr uint32_t kDecOffAbort = kDecOffSlot + 4;
+constexpr uint32_t kDecAlloc = kDecOffAbort + 4 + 1024;
+
+__global__ void __launch_bounds__(kThreads, 1)
+tc_decode_nf4(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmCodes,
+              const __grid_constant__ CUtensorMap tmU2, const __grid_constant__ CUtensorMap tmB2, DecodeParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t base = (ptx::smem_addr(smem_raw) + 1023u) & ~1023u;
+    uint8_t* gbase = smem_raw + (base - ptx::smem_addr(smem_raw));
+    const uint32_t sA = base, sB = base + kDecOffB, sCodes = base + kDecOffCodes;
+    const uint32_t bar_cfull = base + kDecOffBars;
+    const uint32_t bar_cempty = bar_cfull + 8 * kDecCodeStages;
+    const uint32_t bar_bfull = bar_cempty + 8 * kDecCodeStages;
+    const uint32_t bar_afull = bar_bfull + 8 * kDecStages;
+    const uint32_t bar_aempty = bar_afull + 8 * kDecStages;
+    const uint32_t bar_acc = bar_aempty + 8 * kDecStages;
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gbase + kDecOffSlot);
+    volatile int* abort = reinterpret_cast<volatile int*>(gbase + kDecOffAbort);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t n0 = (int64_t)blockIdx.x * 128;
+    const int split = blockIdx.y;
+    const int kbeg = split * p.kps;
+    const int nk0 = max(0, min(p.ksteps0, kbeg + p.kps) - kbeg);
+    const int nk1 = split == 0 ? p.ksteps1 : 0;
+    const int ntot = nk0 + nk1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kDecCodeStages; ++s) {
+            ptx::mbar_init(bar_cfull + 8 * s, 1);
+            ptx::mbar_init(bar_cempty + 8 * s, 4);
+        }
+        for (int s = 0; s < kDecStages; ++s) {
+            ptx::mbar_init(bar_bfull + 8 * s, 1);
+            ptx::mbar_init(bar_afull + 8 * s, 4);
+            ptx::mbar_init(bar_aempty + 8 * s, 1);
+        }
+        ptx::mbar_init(bar_acc, 1);
+        *abort = 0;
+        ptx::fence_barrier_init();
+        ptx::fence_proxy_async_smem();
+        ptx::tma_prefetch_map(&tmX);
+        ptx::tma_prefetch_map(&tmCodes);
+        ptx::tma_prefetch_map(&tmU2);
+        ptx::tma_prefetch_map(&tmB2);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(base + kDecOffSlot, 32);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // codes run up to kDecCodeStages steps ahead of the tile ring
+            int next_code = 0;
+            bool ok = true;
+            for (int i = 0; i < ntot && ok; ++i) {
+                const int code_limit = min(nk0, i + kDecCodeStages);
+                while (next_code < code_limit && ok) {
+                    const int cs = next_code % kDecCodeStages;
+                    const uint32_t cph = (uint32_t)(next_code / kDecCodeStages) & 1u;
+                    ok = ptx::mbar_wait(bar_cempty + 8 * cs, cph ^ 1u, abort, p.err);
+                    if (!ok) break;
+                    ptx::mbar_arrive_expect_tx(bar_cfull + 8 * cs, kDecCodesStage);
+                    ptx::tma_load_2d(sCodes + cs * kDecCodesStage, &tmCodes, (kbeg + next_code) * 32, (int32_t)n0,
+                                     bar_cfull + 8 * cs);
+                    ++next_code;
+                }
+                if (!ok) break;
+                const int s = i % kDecStages;
+                const uint32_t ph = (uint32_t)(i / kDecStages) & 1u;
+                ok = ptx::mbar_wait(bar_aempty + 8 * s, ph ^ 1u, abort, p.err);
+                if (!ok) break;
+                const uint32_t fb = bar_bfull + 8 * s;
+                if (i < nk0) {
+                    ptx::mbar_arrive_expect_tx(fb, kDecBStage);
+                    ptx::tma_load_2d(sB + s * kDecBStage, &tmX, (kbeg + i) * 64, 0, fb);
+                } else {
+                    const int j = i - nk0;
+                    ptx::mbar_arrive_expect_tx(fb, kDecAStage + kDecBStage);
+                    ptx::tma_load_2d(sA + s * kDecAStage, &tmB2, j * 64, (int32_t)n0, fb);
+                    ptx::tma_load_2d(sB + s * kDecBStage, &tmU2, j * 64, 0, fb);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = ptx::idesc_bf16_f32_ab(128, 16, 0, 0);
+            bool ok = true;
+            for (int i = 0; i < ntot && ok; ++i) {
+                const int s = i % kDecStages;
+                const uint32_t ph = (uint32_t)(i / kDecStages) & 1u;
+                ok = ptx::mbar_wait(bar_bfull + 8 * s, ph, abort, p.err);
+                if (ok && i < nk0) ok = ptx::mbar_wait(bar_afull + 8 * s, ph, abort, p.err);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                const uint32_t a_base = sA + s * kDecAStage, b_base = sB + s * kDecBStage;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    ptx::mma_bf16_ss(tmem, ptx::smem_desc_sw128(a_base + kk * 32, 16, 1024),
+                                     ptx::smem_desc_sw128(b_base + kk * 32, 16, 1024), idesc,
+                                     (i | kk) != 0 ? 1u : 0u);
+                ptx::mma_commit(bar_aempty + 8 * s);
+            }
+            ptx::mma_commit(bar_acc);
+        }
+    } else {
+        // producers: thread t expands W row n0 + t for every K-step of this split
+        const int t = threadIdx.x - 64;
+        const int64_t n = n0 + t;
+        const bool row_ok = n < p.N;
+        const float mu = *p.mu;
+        const int64_t blk0 = n * (p.K / 64) + kbeg;
+        // block constants of steps i .. i+kDecPrefetch-1 (register queue, shifted each step)
+        uint32_t qcode[kDecPrefetch];
+        float qc2[kDecPrefetch];
+#pragma unroll
+        for (int d = 0; d < kDecPrefetch; ++d) {
+            qcode[d] = 0;
+            qc2[d] = 0.f;
+            if (row_ok && d < nk0) {
+                qcode[d] = __ldg(p.c1_codes + blk0 + d);
+                qc2[d] = __ldg(p.c2 + ((blk0 + d) >> 8));
+            }
+        }
+        bool ok = true;
+        for (int i = 0; i < nk0 && ok; ++i) {
+            const int cs = i % kDecCodeStages;
+            const uint32_t cph = (uint32_t)(i / kDecCodeStages) & 1u;
+            const int s = i % kDecStages;
+            const uint32_t ph = (uint32_t)(i / kDecStages) & 1u;
+            const float c1p = rebuild_c1(qcode[0], qc2[0], mu);
+#pragma unroll
+            for (int d = 0; d + 1 < kDecPrefetch; ++d) {
+                qcode[d] = qcode[d + 1];
+                qc2[d] = qc2[d + 1];
+            }
+            if (row_ok && i + kDecPrefetch < nk0) {
+                qcode[kDecPrefetch - 1] = __ldg(p.c1_codes + blk0 + i + kDecPrefetch);
+                qc2[kDecPrefetch - 1] = __ldg(p.c2 + ((blk0 + i + kDecPrefetch) >> 8));
+            }
+            bool w_ok = ptx::mbar_wait(bar_cfull + 8 * cs, cph, abort, p.err);
+            w_ok = w_ok && ptx::mbar_wait(bar_aempty + 8 * s, ph ^ 1u, abort, p.err);
+            ok = __all_sync(0xffffffffu, w_ok);
+            if (!ok) break;
+            const uint32_t row_addr = sA + s * kDecAStage + (uint32_t)t * 128u;
+            if (!row_ok) {
+                zero_row(row_addr);
+            } else {
+                const uint32_t src = sCodes + cs * kDecCodesStage + (uint32_t)t * 32u;
+                const uint32_t first = ((uint32_t)t >> 2) & 1u;
+                const uint4 x = ld_shared_v4(src + first * 16u);
+                const uint4 y = ld_shared_v4(src + (first ^ 1u) * 16u);
+                Lut lut;
+                build_lut(lut, c1p, p.tb);
+                expand_block_row(row_addr, (uint32_t)t & 7u, first ? y : x, first ? x : y, lut);
+            }
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                ptx::mbar_arrive(bar_cempty + 8 * cs);
+                ptx::mbar_arrive(bar_afull + 8 * s);
+            }
+        }
+        // epilogue: lane quadrant (warp & 3) holds W rows n0 + 32*quad + lane, columns = tokens
+        const bool acc_ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_acc, 0, abort, p.err));
+        ptx::tc_fence_after();
+        if (acc_ok && ntot > 0) {
+            const uint32_t quad = (uint32_t)(warp & 3);
+            uint32_t v[16];
+            ptx::tmem_ld_32x32b_x16(tmem + ((quad * 32u) << 16), v);
+            ptx::tmem_ld_wait();
+            const int64_t nn = n0 + quad * 32 + lane;
+            if (nn < p.N) {
+#pragma unroll
+                for (int m = 0; m < 16; ++m) {
+                    if (m >= p.M) break;
+                    const float val = __uint_as_float(v[m]);
+                    if (p.splits > 1) {
+                        p.partial[((int64_t)split * p.M + m) * p.N + nn] = val;
+                    } else if (p.out_f32) {
+                        static_cast<float*>(p.out)[(int64_t)m * p.N + nn] = val;
+                    } else {
+                        static_cast<uint16_t*>(p.out)[(int64_t)m * p.N + nn] = (uint16_t)f32_to_bf16_bits_rn(val);
+                    }
+                }
+            }
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, 32);
+    }
+}
+
+// out[m, n] = sum over splits of partial[s][m][n] (fixed order), converted to the output type.
+__global__ void decode_reduce(const float* __restrict__ partial, int splits, int64_t MN, void* out, int out_f32) {
+    const int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x;
+    if (i >= MN) return;
+    float acc = 0.f;
+    for (int s = 0; s < splits; ++s) acc = __fadd_rn(acc, partial[(int64_t)s * MN + i]);
+    if (out_f32) static_cast<float*>(out)[i] = acc;
+    else static_cast<uint16_t*>(out)[i] = (uint16_t)f32_to_bf16_bits_rn(acc);
+}
+
 // ---------------------------------------------------------------------------- host
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -424,8 +655,56 @@ static qlora_status launch_one(const TcGemmArgs& a, cudaStream_t stream) {
         configured = true;
     }
     const dim3 grid((unsigned)((a.p.Nout + kBN - 1) / kBN), (unsigned)((a.p.M + L::kBM - 1) / L::kBM));
-    kern<<<grid, kThreads, L::kAlloc, stream>>>(a.tmA0, a.tmCodes, a.tmA1, a.tmB1, a.p);
+    kern<<<grid, kGemmThreads, L::kAlloc, stream>>>(a.tmA0, a.tmCodes, a.tmA1, a.tmB1, a.p);
     QLORA_CHECK_LAUNCH();
+    return QLORA_OK;
+}
+
+// Splits of the reduction so that tiles x splits fills one wave of CTAs (two per SM).
+int decode_splits(int64_t N, int ksteps0, int sms) {
+    const int64_t tiles = (N + 127) / 128;
+    const int64_t slots = 2 * (int64_t)sms;
+    int64_t sp = slots / tiles;
+    if (sp > 16) sp = 16;
+    if (sp > ksteps0) sp = ksteps0;
+    return sp < 1 ? 1 : (int)sp;
+}
+
+qlora_status launch_tc_decode(const DecodeArgs& a, cudaStream_t stream) {
+    const qlora_nf4_weight* w = a.w;
+    const int64_t N = w->N, K = w->K;
+    const int64_t R2 = 2 * (int64_t)a.Rpad;
+    CUtensorMap tmX, tmCodes, tmU2, tmB2;
+    if (!make_tmap_2d(&tmX, true, a.X, K, a.M, K * 2, 64, 16, true)) return QLORA_ERR_CUDA;
+    if (!make_tmap_2d(&tmCodes, false, w->codes, K / 2, N, K / 2, 32, 128, false)) return QLORA_ERR_CUDA;
+    if (!make_tmap_2d(&tmU2, true, a.U2, R2, a.M, R2 * 2, 64, 16, true)) return QLORA_ERR_CUDA;
+    if (!make_tmap_2d(&tmB2, true, a.B2, R2, N, R2 * 2, 64, 128, true)) return QLORA_ERR_CUDA;
+    DecodeParams p{};
+    p.M = a.M; p.N = N; p.K = K;
+    p.ksteps0 = (int)(K / 64);
+    p.ksteps1 = (int)(R2 / 64);
+    p.kps = (p.ksteps0 + a.splits - 1) / a.splits;
+    p.splits = (p.ksteps0 + p.kps - 1) / p.kps;          // every split gets at least one K-step
+    p.c1_codes = w->c1_codes; p.c2 = w->c2; p.mu = w->mu;
+    p.out = a.out; p.out_f32 = a.out_f32; p.partial = a.partial;
+    p.tb = host_tables();
+    p.err = device_error_word();
+    if (!p.err) return QLORA_ERR_CUDA;
+    static bool configured = false;
+    if (!configured) {
+        if (cudaFuncSetAttribute(tc_decode_nf4, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDecAlloc) !=
+            cudaSuccess)
+            return QLORA_ERR_CUDA;
+        configured = true;
+    }
+    const dim3 grid((unsigned)((N + 127) / 128), (unsigned)p.splits);
+    tc_decode_nf4<<<grid, kThreads, kDecAlloc, stream>>>(tmX, tmCodes, tmU2, tmB2, p);
+    QLORA_CHECK_LAUNCH();
+    if (p.splits > 1) {
+        const int64_t MN = a.M * N;
+        decode_reduce<<<(unsigned)((MN + 255) / 256), 256, 0, stream>>>(a.partial, p.splits, MN, a.out, a.out_f32);
+        QLORA_CHECK_LAUNCH();
+    }
     return QLORA_OK;
 }
 

@@ -36,6 +36,37 @@ struct TcGemmArgs {
 // Encodes the tensor maps and launches the forward (dx = false) or dX kernel.
 qlora_status launch_tc_gemm_nf4(TcGemmArgs& a, bool dx, cudaStream_t stream);
 
+// Small-M forward (M <= 16): swap-AB fused dequant-GEMM with split-K.
+struct DecodeParams {
+    int64_t M, N, K;
+    int32_t ksteps0, ksteps1, kps, splits;
+    const uint8_t* c1_codes;
+    const float* c2;
+    const float* mu;
+    void* out;
+    int32_t out_f32;
+    float* partial;         // [splits, M, N] fp32 when splits > 1
+    uint32_t* err;
+    NF4Tables tb;
+};
+
+struct DecodeArgs {
+    const qlora_nf4_weight* w;
+    const void* X;          // [M, K] bf16
+    const void* U2;         // [M, 2*Rpad] bf16 hi/lo of s*U
+    const void* B2;         // [N, 2*Rpad] bf16
+    int32_t Rpad;
+    int64_t M;
+    void* out;
+    int32_t out_f32;
+    float* partial;
+    int32_t splits;
+};
+
+constexpr int64_t kDecodeMaxM = 16;
+int decode_splits(int64_t N, int ksteps0, int sms);
+qlora_status launch_tc_decode(const DecodeArgs& a, cudaStream_t stream);
+
 // LoRA-side GEMM (gemm_lora_tc.cu): partial[split][rows][R] = sum over the
 // split's share of the reduction of A-operand rows times B-operand rows.
 struct LoraGemmParams {

@@ -20,8 +20,21 @@ struct NF4Tables {
     float t[15];
 };
 
+// Bucketed code search for the quantize kernel.  For fp32 x in [-1, 1] with
+// bits b, the bucket index is
+//     k = max(((b & 0x7FFFFFFF) >> 20) - 0x3CF, 0) + 42 * (b >> 31)
+// (bucket 0 of each sign holds |x| < 2^-5; the others split each binade of
+// |x| in [2^-5, 1] into 8 equal parts).  No bucket contains more than one
+// decision threshold, so code(x) = base[k] + (x > thr[k]) with thr[k] = +inf
+// for buckets without a threshold.
+constexpr int kCodeBuckets = 84;
+struct QuantBuckets {
+    float2 e[kCodeBuckets];   // (.x = threshold, .y = base code as int bits)
+};
+
 // Host side: the library's tables, built once (codebook.cu).
 const NF4Tables& host_tables();
+const QuantBuckets& host_buckets();
 
 // Host side: count of kernels launched by this library (api.cu).
 void note_launches(int n);

@@ -4,17 +4,19 @@
 // 8-bit floats with second-level block 256).
 //
 // Kernels, in launch order:
-//   nf4_quantize_blocks  one pass over W: per 64-block absmax (4 threads per
-//                        block, warp shuffles), IEEE division, 15-threshold
-//                        code count, nibble packing; writes the packed codes,
-//                        the fp32 absmax c1 per block, and the fp64 sum of the
-//                        CTA's 64 c1 values over a fixed pairwise tree.
+//   nf4_quantize_blocks  one pass over W: per 64-block absmax (2 threads per
+//                        block, packed 16-bit max), correctly rounded
+//                        division, bucketed code search with one compare,
+//                        nibble packing; writes the packed codes, the fp32
+//                        absmax c1 per block, and the fp64 sum of each chunk
+//                        of 128 c1 values over a fixed pairwise tree.
 //   tree_sum_pass        fp64 pairwise-tree sums of 1024 partials per CTA,
 //                        repeated until one value is left.
 //   dq_blocks            per group of 256 blocks: mu from the tree sum,
 //                        d = c1 - mu, c2 = max|d|, E4M3 code of d / c2.
 // Every tree is over aligned power-of-two ranges with zero padding, so the
 // total equals a pairwise tree over all c1 padded to a power of two.
+#include <algorithm>
 #include <mutex>
 
 #include "qlora_internal.cuh"
@@ -40,76 +42,114 @@ uint32_t* device_error_word() {
 
 namespace {
 
-constexpr int kQuantThreads = 256;                   // 64 blocks of 64 weights per CTA
-constexpr int kBlocksPerCta = kQuantThreads / 4;
+constexpr int kQuantThreads = 256;                   // 2 threads per block of 64 weights
+constexpr int kBlocksPerCta = kQuantThreads / 2;     // 128 blocks per chunk (one CTA iteration)
+constexpr int kCtasPerSm = 3;
+constexpr int kTableEntries = 4096;                  // every 12-bit index (bits >> 20) is in range
 constexpr int kTreeThreads = 1024;
 constexpr int kDqThreads = 256;                      // one group of 256 blocks per CTA
 
-__device__ __forceinline__ uint32_t nf4_code(float x, const NF4Tables& tb) {
-    uint32_t c = 0;
-#pragma unroll
-    for (int j = 0; j < 15; ++j) c += (x > tb.t[j]) ? 1u : 0u;
-    return c;
+// x = fp32(w / m), correctly rounded, for |w| <= m with m in [2^-100, 2^100]:
+// Markstein's division (P. Markstein, "Computation of elementary functions on
+// the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990): with
+// y = RN(1/m) and q0 = RN(w*y), the remainder r = w - m*q0 is exact in one
+// FMA and RN(q0 + r*y) is the correctly rounded quotient.  Outside that scale
+// range the IEEE division intrinsic is used.
+__device__ __forceinline__ float div_markstein(float w, float m, float y) {
+    const float q0 = __fmul_rn(w, y);
+    const float r = __fmaf_rn(-m, q0, w);
+    return __fmaf_rn(r, y, q0);
 }
 
-__global__ void __launch_bounds__(kQuantThreads)
-nf4_quantize_blocks(const uint4* __restrict__ W, int64_t nb1, uint2* __restrict__ codes,
-                    float* __restrict__ c1_out, double* __restrict__ cta_sums, NF4Tables tb) {
-    const int64_t blk = (int64_t)blockIdx.x * kBlocksPerCta + (threadIdx.x >> 2);
-    const int sub = threadIdx.x & 3;
-    const bool valid = blk < nb1;
+// NF4 code of x in [-1, 1]: the table is indexed by the top 12 bits of x
+// (sign, exponent, 3 mantissa bits), i.e. by bucket; one compare finishes.
+__device__ __forceinline__ uint32_t nf4_code(float x, const float2* __restrict__ table) {
+    const float2 e = table[__float_as_uint(x) >> 20];
+    return (uint32_t)__float_as_int(e.y) + (x > e.x ? 1u : 0u);
+}
 
-    uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    if (valid) {
-        const uint4 a = W[(blk * 64 + sub * 16) / 8];
-        const uint4 b = W[(blk * 64 + sub * 16) / 8 + 1];
-        w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
-        w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
-    }
-    float v[16];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        v[2 * i] = bf16_bits_to_f32(w[i] & 0xFFFFu);
-        v[2 * i + 1] = bf16_bits_to_f32(w[i] >> 16);
-    }
-    float m = 0.f;
-    bool finite = true;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const float a = fabsf(v[i]);
-        finite &= (a <= 3.402823466e38f);
-        m = fmaxf(m, a);
-    }
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-    if (!finite) atomicOr(&g_error_flags, ERR_FLAG_NONFINITE);
-
-    if (valid) {
-        uint32_t lo = 0, hi = 0;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float x = (m > 0.f) ? __fdiv_rn(v[i], m) : 0.f;
-            const uint32_t c = nf4_code(x, tb);
-            const int byte = i >> 1;
-            const int shift = 8 * (byte & 3) + ((i & 1) ? 0 : 4);   // element 2j -> high nibble
-            if (byte < 4) lo |= c << shift; else hi |= c << shift;
-        }
-        codes[blk * 4 + sub] = make_uint2(lo, hi);
-        if (sub == 0) c1_out[blk] = m;
-    }
-
-    // fp64 tree over the CTA's 64 block constants: lanes 0,4,...,28 hold blocks
-    // 8w..8w+7 of warp w; xor-shuffles by 4, 8, 16 pair neighbours level by level.
-    double s = valid ? (double)m : 0.0;
-    s += __shfl_xor_sync(0xffffffffu, s, 4);
-    s += __shfl_xor_sync(0xffffffffu, s, 8);
-    s += __shfl_xor_sync(0xffffffffu, s, 16);
+// One pass over W.  Persistent CTAs loop over chunks of 128 consecutive NF4
+// blocks; two threads share a block (32 weights each).  Per chunk: packed
+// codes, fp32 block absmax, and the chunk's fp64 pairwise-tree sum of c1.
+__global__ void __launch_bounds__(kQuantThreads, kCtasPerSm)
+nf4_quantize_blocks(const uint4* __restrict__ W, int64_t nb1, uint4* __restrict__ codes,
+                    float* __restrict__ c1_out, double* __restrict__ chunk_sums, int64_t n_chunks,
+                    QuantBuckets qb) {
+    __shared__ float2 table[kTableEntries];
     __shared__ double warp_sums[kQuantThreads / 32];
-    if ((threadIdx.x & 31) == 0) warp_sums[threadIdx.x >> 5] = s;
+    for (int i = threadIdx.x; i < kTableEntries; i += kQuantThreads) {
+        const int key = min(max((i & 0x7FF) - 0x3CF, 0), 41);
+        table[i] = qb.e[key + 42 * (i >> 11)];
+    }
     __syncthreads();
-    if (threadIdx.x == 0) {
-        const double* ws = warp_sums;
-        cta_sums[blockIdx.x] = ((ws[0] + ws[1]) + (ws[2] + ws[3])) + ((ws[4] + ws[5]) + (ws[6] + ws[7]));
+    const int sub = threadIdx.x & 1;
+    for (int64_t chunk = blockIdx.x; chunk < n_chunks; chunk += gridDim.x) {
+        const int64_t blk = chunk * kBlocksPerCta + (threadIdx.x >> 1);
+        const bool valid = blk < nb1;
+        uint4 v4[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v4[j] = valid ? W[blk * 8 + sub * 4 + j] : make_uint4(0, 0, 0, 0);
+        const uint32_t w[16] = {v4[0].x, v4[0].y, v4[0].z, v4[0].w, v4[1].x, v4[1].y, v4[1].z, v4[1].w,
+                                v4[2].x, v4[2].y, v4[2].z, v4[2].w, v4[3].x, v4[3].y, v4[3].z, v4[3].w};
+        // block absmax on the bf16 bit patterns: |w| orders like the unsigned 15-bit magnitude
+        uint32_t mx = 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) mx = __vmaxu2(mx, w[i] & 0x7FFF7FFFu);
+        uint32_t mbits = max(mx & 0xFFFFu, mx >> 16);
+        mbits = max(mbits, (uint32_t)__shfl_xor_sync(0xffffffffu, mbits, 1));
+        const float m = bf16_bits_to_f32(mbits);
+        if (mbits >= 0x7F80u) atomicOr(&g_error_flags, ERR_FLAG_NONFINITE);
+
+        if (valid) {
+            uint32_t out[4] = {0x77777777u, 0x77777777u, 0x77777777u, 0x77777777u};  // all-zero block: code 7
+            if (m > 0.f && mbits < 0x7F80u) {
+                if ((m >= 7.8886091e-31f) && (m <= 1.2676506e30f)) {   // 2^-100 .. 2^100: Markstein division
+                    const float y = __frcp_rn(m);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t word = 0;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {     // weights 8q .. 8q+7 of this thread
+                            const uint32_t pair = w[4 * q + (i >> 1)];
+                            const float v = __uint_as_float((i & 1) ? (pair & 0xFFFF0000u) : (pair << 16));
+                            const uint32_t c = nf4_code(div_markstein(v, m, y), table);
+                            word |= c << (8 * (i >> 1) + ((i & 1) ? 0 : 4));   // weight 2j -> high nibble
+                        }
+                        out[q] = word;
+                    }
+                } else {                                                // extreme scales: IEEE division
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t word = 0;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const uint32_t pair = w[4 * q + (i >> 1)];
+                            const float v = __uint_as_float((i & 1) ? (pair & 0xFFFF0000u) : (pair << 16));
+                            const uint32_t c = nf4_code(__fdiv_rn(v, m), table);
+                            word |= c << (8 * (i >> 1) + ((i & 1) ? 0 : 4));
+                        }
+                        out[q] = word;
+                    }
+                }
+            }
+            codes[blk * 2 + sub] = make_uint4(out[0], out[1], out[2], out[3]);
+            if (sub == 0) c1_out[blk] = m;
+        }
+
+        // fp64 pairwise tree over the chunk's 128 block constants: even lanes hold the
+        // blocks of the warp in order; xor-shuffles by 2..16 pair neighbours level by level.
+        double s = valid ? (double)m : 0.0;
+        s += __shfl_xor_sync(0xffffffffu, s, 2);
+        s += __shfl_xor_sync(0xffffffffu, s, 4);
+        s += __shfl_xor_sync(0xffffffffu, s, 8);
+        s += __shfl_xor_sync(0xffffffffu, s, 16);
+        if ((threadIdx.x & 31) == 0) warp_sums[threadIdx.x >> 5] = s;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            const double* ws = warp_sums;
+            chunk_sums[chunk] = ((ws[0] + ws[1]) + (ws[2] + ws[3])) + ((ws[4] + ws[5]) + (ws[6] + ws[7]));
+        }
+        __syncthreads();
     }
 }
 
@@ -161,7 +201,7 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 }  // namespace
 
 // Scratch layout of the quantize: fp32 c1[nb1], then the fp64 partial sums of
-// every tree level (P1 = ceil(nb1/64), then ceil(P/1024) until 1).
+// every tree level (P1 = ceil(nb1/128), then ceil(P/1024) until 1).
 size_t quantize_workspace_bytes(int64_t nb1) {
     size_t bytes = align_up((size_t)nb1 * sizeof(float), 256);
     int64_t p = (nb1 + kBlocksPerCta - 1) / kBlocksPerCta;
@@ -176,7 +216,6 @@ size_t quantize_workspace_bytes(int64_t nb1) {
 qlora_status launch_quantize(const void* W, int64_t N, int64_t K, const qlora_nf4_weight* out,
                              void* workspace, cudaStream_t stream) {
     const int64_t nb1 = N * K / 64;
-    const NF4Tables& tb = host_tables();
     char* ws = static_cast<char*>(workspace);
     float* c1 = reinterpret_cast<float*>(ws);
     ws += align_up((size_t)nb1 * sizeof(float), 256);
@@ -184,8 +223,11 @@ qlora_status launch_quantize(const void* W, int64_t N, int64_t K, const qlora_nf
     double* level = reinterpret_cast<double*>(ws);
     ws += align_up((size_t)p * sizeof(double), 256);
 
-    nf4_quantize_blocks<<<(unsigned)p, kQuantThreads, 0, stream>>>(
-        static_cast<const uint4*>(W), nb1, reinterpret_cast<uint2*>(out->codes), c1, level, tb);
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t grid = std::min<int64_t>(p, (int64_t)sms * kCtasPerSm);
+    nf4_quantize_blocks<<<(unsigned)grid, kQuantThreads, 0, stream>>>(
+        static_cast<const uint4*>(W), nb1, reinterpret_cast<uint4*>(out->codes), c1, level, p, host_buckets());
     QLORA_CHECK_LAUNCH();
     while (p > 1) {
         const int64_t np = (p + kTreeThreads - 1) / kTreeThreads;

@@ -101,6 +101,30 @@ def test_quantize_decision_boundaries_bit_exact():
     check_dequantize_exact(w, check_quantize_exact(W, w))
 
 
+def test_quantize_every_scale_at_every_decision_boundary():
+    """Every positive finite bf16 block absmax c (subnormals included), each with
+    the bf16 values within +-2 ulps of t_j * c for all 15 decision thresholds."""
+    g = np.random.default_rng(11)
+    q = o.nf4_codebook().astype(np.float64)
+    mids = (q[:-1] + q[1:]) / 2
+    scales = np.arange(1, 0x7F80, dtype=np.uint32).astype(np.uint16)         # all positive finite bf16
+    c = o.bf16_bits_to_f32(scales).astype(np.float64)
+    centre = o.f32_to_bf16_bits((c[:, None] * mids[None, :]).astype(np.float32)).astype(np.int64)
+    cand = np.concatenate([centre + d for d in (-2, -1, 0, 1, 2)], axis=1)   # [n_scales, 75]
+    cand = np.where((cand & 0x7F80) == 0x7F80, 0, cand)                        # keep finite patterns
+    mag = o.bf16_bits_to_f32(cand.astype(np.uint16)).astype(np.float64)
+    cand = np.where(np.abs(mag) <= c[:, None], cand, 0).astype(np.uint16)     # |value| <= absmax
+    filler = g.integers(0, 0x7F80, size=(scales.size, 126 - 75)).astype(np.uint16)
+    fmag = o.bf16_bits_to_f32(filler).astype(np.float64)
+    filler = np.where(fmag <= c[:, None], filler, 0).astype(np.uint16)
+    body = np.concatenate([cand, filler], axis=1)
+    blocks = np.concatenate([scales[:, None], body[:, :63], scales[:, None], body[:, 63:]], axis=1)
+    bits = np.ascontiguousarray(blocks.reshape(-1, 128))               # one row = the two blocks of a scale
+    W = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+    w = quantize_on_gpu(W)
+    check_dequantize_exact(w, check_quantize_exact(W, w))
+
+
 def test_quantize_every_finite_bf16_value():
     g = np.random.default_rng(1)
     allb = np.arange(65536, dtype=np.uint32).astype(np.uint16)
