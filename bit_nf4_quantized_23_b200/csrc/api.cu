@@ -3,6 +3,8 @@
 #include <algorithm>
 #include <atomic>
 #include <cmath>
+#include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -118,6 +120,20 @@ qlora_status lora_U(const void* X, const void* A2, int64_t M, int64_t K, int32_t
 }  // namespace
 
 void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+bool sync_check_enabled() {
+    static const bool on = std::getenv("QLORA_SYNC_CHECK") != nullptr;
+    return on;
+}
+
+bool sync_check(const char* where) {
+    const cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) {
+        std::fprintf(stderr, "[qlora] kernel launched from %s failed: %s\n", where, cudaGetErrorString(e));
+        return false;
+    }
+    return true;
+}
 
 }  // namespace qlora
 
@@ -389,16 +405,17 @@ qlora_status qlora_read_device_errors(void* stream, int32_t clear, uint32_t* fla
     uint32_t* word = device_error_word();
     if (!word) return QLORA_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    uint32_t h = 0;
-    if (cudaMemcpyAsync(&h, word, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess) return QLORA_ERR_CUDA;
+    uint32_t h[2] = {0, 0};
+    if (cudaMemcpyAsync(h, word, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess) return QLORA_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return QLORA_ERR_CUDA;
-    if (clear && h) {
-        if (cudaMemsetAsync(word, 0, sizeof(uint32_t), s) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (h[1] && sync_check_enabled()) std::fprintf(stderr, "[qlora] device location code 0x%08x\n", h[1]);
+    if (clear && (h[0] || h[1])) {
+        if (cudaMemsetAsync(word, 0, sizeof(h), s) != cudaSuccess) return QLORA_ERR_CUDA;
         if (cudaStreamSynchronize(s) != cudaSuccess) return QLORA_ERR_CUDA;
     }
-    if (flags) *flags = h;
-    if (h & ERR_FLAG_TIMEOUT) return QLORA_ERR_TIMEOUT;
-    if (h & ERR_FLAG_NONFINITE) return QLORA_ERR_NONFINITE;
+    if (flags) *flags = h[0];
+    if (h[0] & ERR_FLAG_TIMEOUT) return QLORA_ERR_TIMEOUT;
+    if (h[0] & ERR_FLAG_NONFINITE) return QLORA_ERR_NONFINITE;
     return QLORA_OK;
 }
 

@@ -74,39 +74,26 @@ NF4Tables build_tables() {
     return tb;
 }
 
-// Bucket table of the quantize kernel (see QuantBuckets): for each sign and
-// bucket, the code of the bucket's lowest x and the one threshold inside it.
+// Bucket table of the quantize kernel (see QuantBuckets).  bucket(x) =
+// RNE(64 x + 64) is monotone in x, so a threshold in a lower bucket lies below
+// every x of bucket k and one in a higher bucket above it.
+int bucket_of(double x) { return (int)std::nearbyint(64.0 * x + 64.0); }   // default mode: ties to even
+
 QuantBuckets build_buckets(const NF4Tables& tb) {
     QuantBuckets qb;
-    for (int sign = 0; sign < 2; ++sign) {
-        for (int k = 0; k < 42; ++k) {
-            float thr = INFINITY;
-            int base = 7;
-            if (k > 0) {
-                const uint32_t lo_bits = (uint32_t)(k - 1 + 0x3D0) << 20;    // |x| range [lo, hi)
-                const uint32_t hi_bits = (uint32_t)(k + 0x3D0) << 20;
-                float lo, hi;
-                std::memcpy(&lo, &lo_bits, 4);
-                std::memcpy(&hi, &hi_bits, 4);
-                base = 0;
-                int inside = 0;
-                for (int j = 0; j < 15; ++j) {
-                    const float t = tb.t[j];
-                    if (sign == 0) {          // x in [lo, hi)
-                        if (t < lo) ++base;
-                        else if (t < hi) { thr = t; ++inside; }
-                    } else {                  // x in (-hi, -lo]
-                        if (t <= -hi) ++base;
-                        else if (t <= -lo) { thr = t; ++inside; }
-                    }
-                }
-                if (inside > 1) std::abort();   // the bucket width is below every threshold gap
-            }
-            int32_t b = base;
-            float bf;
-            std::memcpy(&bf, &b, 4);
-            qb.e[sign * 42 + k] = make_float2(thr, bf);
+    for (int k = 0; k < kCodeBuckets; ++k) {
+        int base = 0, inside = 0;
+        float thr = INFINITY;
+        for (int j = 0; j < 15; ++j) {
+            const int b = bucket_of((double)tb.t[j]);
+            if (b < k) ++base;
+            else if (b == k) { thr = tb.t[j]; ++inside; }
         }
+        if (inside > 1) std::abort();             // bucket narrower than every threshold gap
+        int32_t bb = base;
+        float bf;
+        std::memcpy(&bf, &bb, 4);
+        qb.e[k] = make_float2(thr, bf);
     }
     return qb;
 }

@@ -85,10 +85,12 @@ tc_lora_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
     if (warp == 0) {
         if (lane == 0) {
             const uint32_t b_bytes = MN ? (uint32_t)R * 256u : (uint32_t)R * 128u;
+            int issued = 0;
             for (int i = 0; i < nk; ++i) {
                 const int s = i % kStages;
                 const uint32_t ph = (uint32_t)(i / kStages) & 1u;
                 if (!ptx::mbar_wait(bar_empty + 8 * s, ph ^ 1u, abort, p.err)) break;
+                issued = i + 1;
                 const uint32_t fb = bar_full + 8 * s;
                 const int ks = k_begin + i;
                 const uint32_t a_dst = sA + s * kAStage, b_dst = sB + s * kBStage;
@@ -105,6 +107,10 @@ tc_lora_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                         ptx::tma_load_2d(b_dst + (chunks + c) * 8192, &tmB, R + c * 64, ks * 64, fb);
                     }
                 }
+            }
+            if (*abort) {   // drain this CTA's copies in flight before it exits
+                for (int i = max(0, issued - kStages); i < issued; ++i)
+                    ptx::mbar_wait_drain(bar_full + 8 * (i % kStages), (uint32_t)(i / kStages) & 1u);
             }
         }
     } else if (warp == 1) {
@@ -135,6 +141,7 @@ tc_lora_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                 ptx::mma_commit(bar_empty + 8 * s);
             }
             ptx::mma_commit(bar_acc);
+            if (*abort) ptx::mbar_wait_drain(bar_acc, 0);   // issued MMAs finish before TMEM is freed
         }
     } else {
         const bool acc_ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_acc, 0, abort, p.err));

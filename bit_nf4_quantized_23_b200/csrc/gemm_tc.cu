@@ -183,10 +183,12 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
+            int issued = 0;
             for (int it = 0; it < ktotal; ++it) {
                 const int s = it % kStages;
                 const uint32_t ph = (uint32_t)(it / kStages) & 1u;
                 if (!ptx::mbar_wait(bar_empty + 8 * s, ph ^ 1u, abort, p.err)) break;
+                issued = it + 1;
                 const uint32_t fa = bar_full_a + 8 * s;
                 const uint32_t a_dst = sA + s * L::kAStageBytes;
                 const uint32_t b_dst = sB + s * kBStageBytes;
@@ -207,6 +209,10 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
                             ptx::tma_load_2d(b_dst + c * 8192, &tmB1, (int32_t)(n0 + c * 64), j * 64, fa);
                     }
                 }
+            }
+            if (*abort) {   // drain this CTA's copies in flight before it exits
+                for (int it = max(0, issued - kStages); it < issued; ++it)
+                    ptx::mbar_wait_drain(bar_full_a + 8 * (it % kStages), (uint32_t)(it / kStages) & 1u);
             }
         }
     } else if (warp == 1) {
@@ -236,6 +242,7 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
                 ptx::mma_commit(bar_empty + 8 * s);
             }
             ptx::mma_commit(bar_acc);   // arrives when every issued MMA has completed
+            if (*abort) ptx::mbar_wait_drain(bar_acc, 0);   // issued MMAs finish before TMEM is freed
         }
     } else {
         // ------------------------------------------------------------ dequant producers
@@ -383,12 +390,15 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
 // Y[M,N] for M <= 16 tokens (decode), "swap-AB": D[n, m] = W_hat[n, :] X[m, :]^T
 // with the dequantized weight as the 128-row MMA operand A (K-major image
 // written by the producer warps) and the tokens as a 16-wide operand B (TMA).
-// The codes stream through a deep ring (weight bytes dominate the traffic);
-// the reduction over K is split across CTAs so every SM streams.  Split s
+// The codes stream through a deep TMA ring (weight bytes dominate the
+// traffic); the producer warps also copy the small token tile (loaded one step
+// ahead) into the swizzled B stage; the reduction over K is split across CTAs
+// so every SM streams.  Split s
 // writes fp32 partial[s][m][n] (or Y directly when there is one split); the
 // LoRA steps run in split 0.
-constexpr int kDecCodeStages = 12;              // packed-code ring (the HBM stream)
-constexpr int kDecStages = 3;                   // dequantized-tile / token ring
+constexpr int kDecCodeStages = 8;               // packed-code ring (the HBM stream)
+constexpr int kDecStages = 2;                   // dequantized-tile / token ring
+constexpr int kDecCtasPerSm = 3;                // ~69 KB of shared memory per CTA
 constexpr int kDecPrefetch = 4;                 // block constants are loaded this many K-steps ahead
 constexpr uint32_t kDecAStage = 128 * 128;      // W_hat or B2 tile [128 rows x 64]
 constexpr uint32_t kDecBStage = 16 * 128;       // X or U2 tile [16 tokens x 64]
@@ -396,22 +406,20 @@ constexpr uint32_t kDecCodesStage = 128 * 32;   // packed codes [128 rows x 32 b
 constexpr uint32_t kDecOffB = kDecStages * kDecAStage;
 constexpr uint32_t kDecOffCodes = kDecOffB + kDecStages * kDecBStage;
 constexpr uint32_t kDecOffBars = kDecOffCodes + kDecCodeStages * kDecCodesStage;
-// barriers: cfull[CS], cempty[CS], bfull[S], afull[S], aempty[S], acc
-constexpr uint32_t kDecOffSlot = kDecOffBars + (2 * kDecCodeStages + 3 * kDecStages + 1) * 8;
+// barriers: cfull[CS], cempty[CS], afull[S], aempty[S], acc
+constexpr uint32_t kDecOffSlot = kDecOffBars + (2 * kDecCodeStages + 2 * kDecStages + 1) * 8;
 constexpr uint32_t kDecOffAbort = kDecOffSlot + 4;
 constexpr uint32_t kDecAlloc = kDecOffAbort + 4 + 1024;
 
-__global__ void __launch_bounds__(kThreads, 1)
-tc_decode_nf4(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmCodes,
-              const __grid_constant__ CUtensorMap tmU2, const __grid_constant__ CUtensorMap tmB2, DecodeParams p) {
+__global__ void __launch_bounds__(kThreads, kDecCtasPerSm)
+tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, DecodeParams p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t base = (ptx::smem_addr(smem_raw) + 1023u) & ~1023u;
     uint8_t* gbase = smem_raw + (base - ptx::smem_addr(smem_raw));
     const uint32_t sA = base, sB = base + kDecOffB, sCodes = base + kDecOffCodes;
     const uint32_t bar_cfull = base + kDecOffBars;
     const uint32_t bar_cempty = bar_cfull + 8 * kDecCodeStages;
-    const uint32_t bar_bfull = bar_cempty + 8 * kDecCodeStages;
-    const uint32_t bar_afull = bar_bfull + 8 * kDecStages;
+    const uint32_t bar_afull = bar_cempty + 8 * kDecCodeStages;
     const uint32_t bar_aempty = bar_afull + 8 * kDecStages;
     const uint32_t bar_acc = bar_aempty + 8 * kDecStages;
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gbase + kDecOffSlot);
@@ -431,7 +439,6 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             ptx::mbar_init(bar_cempty + 8 * s, 4);
         }
         for (int s = 0; s < kDecStages; ++s) {
-            ptx::mbar_init(bar_bfull + 8 * s, 1);
             ptx::mbar_init(bar_afull + 8 * s, 4);
             ptx::mbar_init(bar_aempty + 8 * s, 1);
         }
@@ -439,10 +446,7 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
         *abort = 0;
         ptx::fence_barrier_init();
         ptx::fence_proxy_async_smem();
-        ptx::tma_prefetch_map(&tmX);
         ptx::tma_prefetch_map(&tmCodes);
-        ptx::tma_prefetch_map(&tmU2);
-        ptx::tma_prefetch_map(&tmB2);
     }
     if (warp == 1) {
         ptx::tmem_alloc(base + kDecOffSlot, 32);
@@ -455,36 +459,23 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
 
     if (warp == 0) {
         if (lane == 0) {
-            // codes run up to kDecCodeStages steps ahead of the tile ring
-            int next_code = 0;
+            // packed codes run up to kDecCodeStages steps ahead of the producers (cempty is
+            // observed phase by phase, in order); nothing else is loaded by TMA
             bool ok = true;
-            for (int i = 0; i < ntot && ok; ++i) {
-                const int code_limit = min(nk0, i + kDecCodeStages);
-                while (next_code < code_limit && ok) {
-                    const int cs = next_code % kDecCodeStages;
-                    const uint32_t cph = (uint32_t)(next_code / kDecCodeStages) & 1u;
-                    ok = ptx::mbar_wait(bar_cempty + 8 * cs, cph ^ 1u, abort, p.err);
-                    if (!ok) break;
-                    ptx::mbar_arrive_expect_tx(bar_cfull + 8 * cs, kDecCodesStage);
-                    ptx::tma_load_2d(sCodes + cs * kDecCodesStage, &tmCodes, (kbeg + next_code) * 32, (int32_t)n0,
-                                     bar_cfull + 8 * cs);
-                    ++next_code;
-                }
+            int issued = 0;
+            for (int c = 0; c < nk0 && ok; ++c) {
+                const int cs = c % kDecCodeStages;
+                const uint32_t cph = (uint32_t)(c / kDecCodeStages) & 1u;
+                ok = ptx::mbar_wait(bar_cempty + 8 * cs, cph ^ 1u, abort, p.err);
                 if (!ok) break;
-                const int s = i % kDecStages;
-                const uint32_t ph = (uint32_t)(i / kDecStages) & 1u;
-                ok = ptx::mbar_wait(bar_aempty + 8 * s, ph ^ 1u, abort, p.err);
-                if (!ok) break;
-                const uint32_t fb = bar_bfull + 8 * s;
-                if (i < nk0) {
-                    ptx::mbar_arrive_expect_tx(fb, kDecBStage);
-                    ptx::tma_load_2d(sB + s * kDecBStage, &tmX, (kbeg + i) * 64, 0, fb);
-                } else {
-                    const int j = i - nk0;
-                    ptx::mbar_arrive_expect_tx(fb, kDecAStage + kDecBStage);
-                    ptx::tma_load_2d(sA + s * kDecAStage, &tmB2, j * 64, (int32_t)n0, fb);
-                    ptx::tma_load_2d(sB + s * kDecBStage, &tmU2, j * 64, 0, fb);
-                }
+                ptx::mbar_arrive_expect_tx(bar_cfull + 8 * cs, kDecCodesStage);
+                ptx::tma_load_2d(sCodes + cs * kDecCodesStage, &tmCodes, (kbeg + c) * 32, (int32_t)n0,
+                                 bar_cfull + 8 * cs);
+                issued = c + 1;
+            }
+            if (*abort) {   // drain this CTA's copies in flight before it exits
+                for (int c = max(0, issued - kDecCodeStages); c < issued; ++c)
+                    ptx::mbar_wait_drain(bar_cfull + 8 * (c % kDecCodeStages), (uint32_t)(c / kDecCodeStages) & 1u);
             }
         }
     } else if (warp == 1) {
@@ -494,9 +485,8 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             for (int i = 0; i < ntot && ok; ++i) {
                 const int s = i % kDecStages;
                 const uint32_t ph = (uint32_t)(i / kDecStages) & 1u;
-                ok = ptx::mbar_wait(bar_bfull + 8 * s, ph, abort, p.err);
-                if (ok && i < nk0) ok = ptx::mbar_wait(bar_afull + 8 * s, ph, abort, p.err);
-                if (!ok) break;
+                ok = ptx::mbar_wait(bar_afull + 8 * s, ph, abort, p.err);
+                if (!ok) { atomicMax(p.dbg, 0x60000000u | (uint32_t)i); break; }
                 ptx::tc_fence_after();
                 const uint32_t a_base = sA + s * kDecAStage, b_base = sB + s * kDecBStage;
 #pragma unroll
@@ -507,12 +497,27 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                 ptx::mma_commit(bar_aempty + 8 * s);
             }
             ptx::mma_commit(bar_acc);
+            if (*abort) ptx::mbar_wait_drain(bar_acc, 0);   // issued MMAs finish before TMEM is freed
         }
     } else {
-        // producers: thread t expands W row n0 + t for every K-step of this split
+        // producers: thread t expands W row n0 + t for every K-step of this split, and copies
+        // 16 bytes of the token tile (token t >> 3, 16-byte chunk t & 7), loaded one step ahead
         const int t = threadIdx.x - 64;
         const int64_t n = n0 + t;
         const bool row_ok = n < p.N;
+        const int xm = t >> 3, xc = t & 7;
+        const bool x_ok = xm < p.M;
+        const uint4* xsrc = static_cast<const uint4*>(p.X) + (int64_t)xm * (p.K / 8) + xc;
+        uint4 xnext = make_uint4(0, 0, 0, 0);
+        const int64_t nb1 = p.N * (p.K / 64);
+        // bounds self-check of the token loads: column (step*64 + xc*8 .. +7) of token xm < M
+        auto x_in_bounds = [&](int step) -> bool {
+            const int64_t col = (int64_t)step * 64 + xc * 8;
+            const bool in = xm < p.M && col + 8 <= p.K && step >= 0;
+            if (!in) { atomicOr(p.err, ERR_FLAG_BOUNDS); atomicMax(p.dbg, 0x10000000u | (uint32_t)step); }
+            return in;
+        };
+        if (x_ok && nk0 > 0 && x_in_bounds(kbeg)) xnext = __ldg(xsrc + (int64_t)kbeg * 8);
         const float mu = *p.mu;
         const int64_t blk0 = n * (p.K / 64) + kbeg;
         // block constants of steps i .. i+kDecPrefetch-1 (register queue, shifted each step)
@@ -523,30 +528,66 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             qcode[d] = 0;
             qc2[d] = 0.f;
             if (row_ok && d < nk0) {
+                if (blk0 + d >= nb1) { atomicOr(p.err, ERR_FLAG_BOUNDS); atomicMax(p.dbg, 0x20000000u); continue; }
                 qcode[d] = __ldg(p.c1_codes + blk0 + d);
                 qc2[d] = __ldg(p.c2 + ((blk0 + d) >> 8));
             }
         }
         bool ok = true;
-        for (int i = 0; i < nk0 && ok; ++i) {
+        for (int i = 0; i < ntot && ok; ++i) {
+            if (i >= nk0) {
+                // LoRA step: copy B2[n0 + t, j*64 .. +63] into the A stage and 16 bytes of
+                // U2[token, j*64 ..] into the B stage (zero outside the matrices)
+                const int s = i % kDecStages;
+                const uint32_t ph = (uint32_t)(i / kDecStages) & 1u;
+                const int j = i - nk0;
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_aempty + 8 * s, ph ^ 1u, abort, p.err));
+                if (!ok) break;
+                const int64_t R2 = 2 * (int64_t)p.Rpad;
+                const uint32_t row_addr = sA + s * kDecAStage + (uint32_t)t * 128u;
+                if (row_ok) {
+                    const uint4* src = static_cast<const uint4*>(p.B2) + (n * R2 + (int64_t)j * 64) / 8;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) st_shared_v4(row_addr + ((c ^ (t & 7)) << 4), __ldg(src + c));
+                } else {
+                    zero_row(row_addr);
+                }
+                uint4 u = make_uint4(0, 0, 0, 0);
+                if (x_ok) u = __ldg(static_cast<const uint4*>(p.U2) + ((int64_t)xm * R2 + (int64_t)j * 64) / 8 + xc);
+                st_shared_v4(sB + s * kDecBStage + (uint32_t)xm * 128u + ((uint32_t)(xc ^ (xm & 7)) << 4), u);
+                ptx::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(bar_afull + 8 * s);
+                continue;
+            }
             const int cs = i % kDecCodeStages;
             const uint32_t cph = (uint32_t)(i / kDecCodeStages) & 1u;
             const int s = i % kDecStages;
             const uint32_t ph = (uint32_t)(i / kDecStages) & 1u;
             const float c1p = rebuild_c1(qcode[0], qc2[0], mu);
+            const uint4 xcur = xnext;
+            if (x_ok && i + 1 < nk0 && x_in_bounds(kbeg + i + 1)) xnext = __ldg(xsrc + (int64_t)(kbeg + i + 1) * 8);
 #pragma unroll
             for (int d = 0; d + 1 < kDecPrefetch; ++d) {
                 qcode[d] = qcode[d + 1];
                 qc2[d] = qc2[d + 1];
             }
             if (row_ok && i + kDecPrefetch < nk0) {
-                qcode[kDecPrefetch - 1] = __ldg(p.c1_codes + blk0 + i + kDecPrefetch);
-                qc2[kDecPrefetch - 1] = __ldg(p.c2 + ((blk0 + i + kDecPrefetch) >> 8));
+                if (blk0 + i + kDecPrefetch < nb1) {
+                    qcode[kDecPrefetch - 1] = __ldg(p.c1_codes + blk0 + i + kDecPrefetch);
+                    qc2[kDecPrefetch - 1] = __ldg(p.c2 + ((blk0 + i + kDecPrefetch) >> 8));
+                } else {
+                    atomicOr(p.err, ERR_FLAG_BOUNDS);
+                    atomicMax(p.dbg, 0x30000000u | (uint32_t)i);
+                }
             }
             bool w_ok = ptx::mbar_wait(bar_cfull + 8 * cs, cph, abort, p.err);
+            if (!w_ok) atomicMax(p.dbg, 0x40000000u | (uint32_t)i);
             w_ok = w_ok && ptx::mbar_wait(bar_aempty + 8 * s, ph ^ 1u, abort, p.err);
+            if (!w_ok) atomicMax(p.dbg, 0x50000000u | (uint32_t)i);
             ok = __all_sync(0xffffffffu, w_ok);
             if (!ok) break;
+            st_shared_v4(sB + s * kDecBStage + (uint32_t)xm * 128u + ((uint32_t)(xc ^ (xm & 7)) << 4), xcur);
             const uint32_t row_addr = sA + s * kDecAStage + (uint32_t)t * 128u;
             if (!row_ok) {
                 zero_row(row_addr);
@@ -660,10 +701,10 @@ static qlora_status launch_one(const TcGemmArgs& a, cudaStream_t stream) {
     return QLORA_OK;
 }
 
-// Splits of the reduction so that tiles x splits fills one wave of CTAs (two per SM).
+// Splits of the reduction so that tiles x splits fills one wave of CTAs.
 int decode_splits(int64_t N, int ksteps0, int sms) {
     const int64_t tiles = (N + 127) / 128;
-    const int64_t slots = 2 * (int64_t)sms;
+    const int64_t slots = kDecCtasPerSm * (int64_t)sms;
     int64_t sp = slots / tiles;
     if (sp > 16) sp = 16;
     if (sp > ksteps0) sp = ksteps0;
@@ -674,13 +715,11 @@ qlora_status launch_tc_decode(const DecodeArgs& a, cudaStream_t stream) {
     const qlora_nf4_weight* w = a.w;
     const int64_t N = w->N, K = w->K;
     const int64_t R2 = 2 * (int64_t)a.Rpad;
-    CUtensorMap tmX, tmCodes, tmU2, tmB2;
-    if (!make_tmap_2d(&tmX, true, a.X, K, a.M, K * 2, 64, 16, true)) return QLORA_ERR_CUDA;
+    CUtensorMap tmCodes;
     if (!make_tmap_2d(&tmCodes, false, w->codes, K / 2, N, K / 2, 32, 128, false)) return QLORA_ERR_CUDA;
-    if (!make_tmap_2d(&tmU2, true, a.U2, R2, a.M, R2 * 2, 64, 16, true)) return QLORA_ERR_CUDA;
-    if (!make_tmap_2d(&tmB2, true, a.B2, R2, N, R2 * 2, 64, 128, true)) return QLORA_ERR_CUDA;
     DecodeParams p{};
-    p.M = a.M; p.N = N; p.K = K;
+    p.M = a.M; p.N = N; p.K = K; p.X = a.X; p.U2 = a.U2; p.B2 = a.B2; p.Rpad = a.Rpad;
+    p.dbg = device_error_word() ? device_error_word() + 1 : nullptr;
     p.ksteps0 = (int)(K / 64);
     p.ksteps1 = (int)(R2 / 64);
     p.kps = (p.ksteps0 + a.splits - 1) / a.splits;
@@ -698,7 +737,7 @@ qlora_status launch_tc_decode(const DecodeArgs& a, cudaStream_t stream) {
         configured = true;
     }
     const dim3 grid((unsigned)((N + 127) / 128), (unsigned)p.splits);
-    tc_decode_nf4<<<grid, kThreads, kDecAlloc, stream>>>(tmX, tmCodes, tmU2, tmB2, p);
+    tc_decode_nf4<<<grid, kThreads, kDecAlloc, stream>>>(tmCodes, p);
     QLORA_CHECK_LAUNCH();
     if (p.splits > 1) {
         const int64_t MN = a.M * N;

@@ -39,6 +39,10 @@ qlora_status launch_tc_gemm_nf4(TcGemmArgs& a, bool dx, cudaStream_t stream);
 // Small-M forward (M <= 16): swap-AB fused dequant-GEMM with split-K.
 struct DecodeParams {
     int64_t M, N, K;
+    const void* X;          // [M, K] bf16 (read by the producer warps)
+    const void* U2;         // [M, 2*Rpad] bf16 (LoRA steps, read by the producer warps)
+    const void* B2;         // [N, 2*Rpad] bf16
+    int32_t Rpad;
     int32_t ksteps0, ksteps1, kps, splits;
     const uint8_t* c1_codes;
     const float* c2;
@@ -47,6 +51,7 @@ struct DecodeParams {
     int32_t out_f32;
     float* partial;         // [splits, M, N] fp32 when splits > 1
     uint32_t* err;
+    uint32_t* dbg;          // second device word: where a self-check or a wait gave up
     NF4Tables tb;
 };
 

@@ -20,14 +20,12 @@ struct NF4Tables {
     float t[15];
 };
 
-// Bucketed code search for the quantize kernel.  For fp32 x in [-1, 1] with
-// bits b, the bucket index is
-//     k = max(((b & 0x7FFFFFFF) >> 20) - 0x3CF, 0) + 42 * (b >> 31)
-// (bucket 0 of each sign holds |x| < 2^-5; the others split each binade of
-// |x| in [2^-5, 1] into 8 equal parts).  No bucket contains more than one
-// decision threshold, so code(x) = base[k] + (x > thr[k]) with thr[k] = +inf
-// for buckets without a threshold.
-constexpr int kCodeBuckets = 84;
+// Bucketed code search for the quantize kernel.  For x in [-1, 1] the bucket
+// is k = RNE(64*x + 64) in [0, 128] (one FMA with a round-to-integer magic
+// constant).  Every gap between decision thresholds exceeds the bucket width
+// 1/64, so a bucket holds at most one threshold and
+//     code(x) = base[k] + (x > thr[k]),   thr[k] = +inf when the bucket has none.
+constexpr int kCodeBuckets = 129;
 struct QuantBuckets {
     float2 e[kCodeBuckets];   // (.x = threshold, .y = base code as int bits)
 };
@@ -41,7 +39,13 @@ void note_launches(int n);
 
 // Device error flag word (one per device that loaded the library).  Kernels in
 // quantize.cu set it directly; other kernels get its address as an argument.
-enum : uint32_t { ERR_FLAG_TIMEOUT = 1u, ERR_FLAG_NONFINITE = 2u };
+enum : uint32_t { ERR_FLAG_TIMEOUT = 1u, ERR_FLAG_NONFINITE = 2u, ERR_FLAG_BOUNDS = 4u };
+
+// Host side: when the environment variable QLORA_SYNC_CHECK is set, every
+// library launch is followed by a device synchronization and a failing kernel
+// is named on stderr (debugging aid; off by default).
+bool sync_check_enabled();
+bool sync_check(const char* kernel);
 
 // Host side: device address of the error word of the current device (cached
 // per device; nullptr on failure).
@@ -103,6 +107,7 @@ __device__ __forceinline__ uint32_t dequant_bits(float q, float c1p) {
             (void)cudaGetLastError();                          \
             return QLORA_ERR_CUDA;                             \
         }                                                      \
+        if (qlora::sync_check_enabled() && !qlora::sync_check(__func__)) return QLORA_ERR_CUDA; \
     } while (0)
 
 #define QLORA_TRY(expr)                                        \

@@ -23,8 +23,9 @@
 
 namespace qlora {
 
-// The device error word of this library (zero-initialised at module load).
-__device__ uint32_t g_error_flags = 0;
+// The device error words of this library (zero-initialised at module load):
+// [0] error flags, [1] location code of the last failed self-check or wait.
+__device__ uint32_t g_error_flags[2] = {0, 0};
 
 uint32_t* device_error_word() {
     static std::mutex mu;
@@ -45,7 +46,7 @@ namespace {
 constexpr int kQuantThreads = 256;                   // 2 threads per block of 64 weights
 constexpr int kBlocksPerCta = kQuantThreads / 2;     // 128 blocks per chunk (one CTA iteration)
 constexpr int kCtasPerSm = 3;
-constexpr int kTableEntries = 4096;                  // every 12-bit index (bits >> 20) is in range
+constexpr int kTableWords = kCodeBuckets * 32;       // bank-private copies: entry e of lane l at e*32 + l
 constexpr int kTreeThreads = 1024;
 constexpr int kDqThreads = 256;                      // one group of 256 blocks per CTA
 
@@ -61,10 +62,14 @@ __device__ __forceinline__ float div_markstein(float w, float m, float y) {
     return __fmaf_rn(r, y, q0);
 }
 
-// NF4 code of x in [-1, 1]: the table is indexed by the top 12 bits of x
-// (sign, exponent, 3 mantissa bits), i.e. by bucket; one compare finishes.
-__device__ __forceinline__ uint32_t nf4_code(float x, const float2* __restrict__ table) {
-    const float2 e = table[__float_as_uint(x) >> 20];
+// NF4 code of x in [-1, 1].  bucket k = RNE(64x + 64) comes from one FMA that
+// rounds to an integer (1.5 * 2^23 makes the fp32 ulp 1); the table keeps one
+// copy of every entry per lane (entry k of lane l at k*32 + l), so the 32 lanes
+// of a warp never meet in a shared-memory bank.
+__device__ __forceinline__ uint32_t nf4_code(float x, const float2* __restrict__ lane_table) {
+    const float y = __fmaf_rn(x, 64.f, 12582976.f);               // 1.5 * 2^23 + 64
+    const uint32_t k = __float_as_uint(y) - 0x4B400000u;          // RNE(64x + 64), 0..128
+    const float2 e = lane_table[k * 32u];
     return (uint32_t)__float_as_int(e.y) + (x > e.x ? 1u : 0u);
 }
 
@@ -75,13 +80,11 @@ __global__ void __launch_bounds__(kQuantThreads, kCtasPerSm)
 nf4_quantize_blocks(const uint4* __restrict__ W, int64_t nb1, uint4* __restrict__ codes,
                     float* __restrict__ c1_out, double* __restrict__ chunk_sums, int64_t n_chunks,
                     QuantBuckets qb) {
-    __shared__ float2 table[kTableEntries];
+    __shared__ float2 table[kTableWords];
     __shared__ double warp_sums[kQuantThreads / 32];
-    for (int i = threadIdx.x; i < kTableEntries; i += kQuantThreads) {
-        const int key = min(max((i & 0x7FF) - 0x3CF, 0), 41);
-        table[i] = qb.e[key + 42 * (i >> 11)];
-    }
+    for (int i = threadIdx.x; i < kTableWords; i += kQuantThreads) table[i] = qb.e[i >> 5];
     __syncthreads();
+    const float2* lane_table = table + (threadIdx.x & 31);
     const int sub = threadIdx.x & 1;
     for (int64_t chunk = blockIdx.x; chunk < n_chunks; chunk += gridDim.x) {
         const int64_t blk = chunk * kBlocksPerCta + (threadIdx.x >> 1);
@@ -98,7 +101,7 @@ nf4_quantize_blocks(const uint4* __restrict__ W, int64_t nb1, uint4* __restrict_
         uint32_t mbits = max(mx & 0xFFFFu, mx >> 16);
         mbits = max(mbits, (uint32_t)__shfl_xor_sync(0xffffffffu, mbits, 1));
         const float m = bf16_bits_to_f32(mbits);
-        if (mbits >= 0x7F80u) atomicOr(&g_error_flags, ERR_FLAG_NONFINITE);
+        if (mbits >= 0x7F80u) atomicOr(&g_error_flags[0], ERR_FLAG_NONFINITE);
 
         if (valid) {
             uint32_t out[4] = {0x77777777u, 0x77777777u, 0x77777777u, 0x77777777u};  // all-zero block: code 7
@@ -112,7 +115,7 @@ nf4_quantize_blocks(const uint4* __restrict__ W, int64_t nb1, uint4* __restrict_
                         for (int i = 0; i < 8; ++i) {     // weights 8q .. 8q+7 of this thread
                             const uint32_t pair = w[4 * q + (i >> 1)];
                             const float v = __uint_as_float((i & 1) ? (pair & 0xFFFF0000u) : (pair << 16));
-                            const uint32_t c = nf4_code(div_markstein(v, m, y), table);
+                            const uint32_t c = nf4_code(div_markstein(v, m, y), lane_table);
                             word |= c << (8 * (i >> 1) + ((i & 1) ? 0 : 4));   // weight 2j -> high nibble
                         }
                         out[q] = word;
@@ -125,7 +128,7 @@ nf4_quantize_blocks(const uint4* __restrict__ W, int64_t nb1, uint4* __restrict_
                         for (int i = 0; i < 8; ++i) {
                             const uint32_t pair = w[4 * q + (i >> 1)];
                             const float v = __uint_as_float((i & 1) ? (pair & 0xFFFF0000u) : (pair << 16));
-                            const uint32_t c = nf4_code(__fdiv_rn(v, m), table);
+                            const uint32_t c = nf4_code(__fdiv_rn(v, m), lane_table);
                             word |= c << (8 * (i >> 1) + ((i & 1) ? 0 : 4));
                         }
                         out[q] = word;
