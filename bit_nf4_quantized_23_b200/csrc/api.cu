@@ -100,7 +100,7 @@ LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int32_t r) {
     part = std::max(part, lora_partial_bytes(M, N, (int)R));
     part = std::max(part, lora_partial_bytes(K, M, (int)R));
     part = std::max(part, lora_partial_bytes(N, M, (int)R));
-    if (M <= kDecodeMaxM) part = std::max(part, (size_t)16 * M * N * sizeof(float));   // decode split-K partials
+    if (M <= kDecodeMaxM) part = std::max(part, decode_partial_bytes(N, K));   // decode partial tiles
     l.part_off = o; o += align_up(part, 256);
     l.total = o;
     return l;
@@ -234,27 +234,20 @@ qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const void* X, int64_t 
     void* B2 = ws + lw.b2_off;
     void* A2 = ws + lw.a2_off;
     float* partial = reinterpret_cast<float*>(ws + lw.part_off);
+    if (M <= kDecodeMaxM) {
+        // decode: U = X A^T and the LoRA term are computed in fp32 around the dequant GEMM
+        DecodeArgs d{};
+        d.w = w; d.X = X; d.A = A; d.B = B; d.r = r; d.scale = scale; d.M = M; d.out = Y;
+        d.out_f32 = (y_dtype == QLORA_DTYPE_F32); d.U = U; d.partial = partial;
+        TimerScope t(QLORA_TIMER_DECODE, s);
+        return launch_tc_decode(d, s);
+    }
     {
         TimerScope t(QLORA_TIMER_LORA, s);
         QLORA_TRY(launch_dup_rows(A, r, R, K, A2, s));
         QLORA_TRY(launch_dup_cols(B, N, r, R, B2, s));
     }
     QLORA_TRY(lora_U(X, A2, M, K, r, R, scale, U, U2, partial, s));
-    if (M <= kDecodeMaxM) {
-        static int sms = 0;
-        if (sms == 0) {
-            int dev = 0;
-            if (cudaGetDevice(&dev) != cudaSuccess ||
-                cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-                return QLORA_ERR_CUDA;
-        }
-        DecodeArgs d{};
-        d.w = w; d.X = X; d.U2 = U2; d.B2 = B2; d.Rpad = R; d.M = M; d.out = Y;
-        d.out_f32 = (y_dtype == QLORA_DTYPE_F32); d.partial = partial;
-        d.splits = decode_splits(N, (int)(K / 64), sms);
-        TimerScope t(QLORA_TIMER_DECODE, s);
-        return launch_tc_decode(d, s);
-    }
     TcGemmArgs a{};
     a.w = w; a.A0 = X; a.A1 = U2; a.B1 = B2; a.Rpad = R;
     a.p.M = M; a.p.Nout = N; a.p.out = Y; a.p.ldo = N; a.p.out_f32 = (y_dtype == QLORA_DTYPE_F32);

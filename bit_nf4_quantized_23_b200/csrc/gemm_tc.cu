@@ -27,6 +27,8 @@
 // table held in byte-split registers and selected with byte permutes), then
 // run the epilogue (TMEM -> registers -> global, bf16 or fp32).
 // No TMA multicast is used anywhere.
+#include <algorithm>
+
 #include <cuda.h>
 
 #include "qlora_internal.cuh"
@@ -38,7 +40,6 @@ namespace {
 
 constexpr int kBN = 256;
 constexpr int kStages = 3;
-constexpr int kThreads = 192;                 // decode kernel: TMA warp, MMA warp, 4 producer/epilogue warps
 constexpr int kProducerWarps = 8;             // fused GEMM: 8 producer/epilogue warps
 constexpr int kGemmThreads = 64 + 32 * kProducerWarps;
 constexpr int kGemmPrefetch = 2;              // block constants are loaded this many K-steps ahead
@@ -92,10 +93,11 @@ __device__ __forceinline__ void build_lut(Lut& t, float c1p, const NF4Tables& tb
 // it.  Bytes whose code is >= 8 take entries 8-15 (sign-replicated bit 3).
 __device__ __forceinline__ uint4 expand8(uint32_t w, const Lut& t) {
     const uint32_t u = w << 4;             // bit 3 of the low nibble of each byte -> that byte's bit 7
+    const uint32_t wm = w & 0x77777777u;   // table index of every code; prmt reads selector bits 0-15
     uint32_t o[4];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-        const uint32_t sel = (w >> (16 * h)) & 0x7777u;
+        const uint32_t sel = h == 0 ? wm : (wm >> 16);
         const uint32_t mask = prmt(u, w, h == 0 ? 0xD9C8u : 0xFBEAu);
         const uint32_t la = prmt(t.L[0], t.L[1], sel);
         const uint32_t lb = prmt(t.L[2], t.L[3], sel);
@@ -389,29 +391,42 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
 //
 // Y[M,N] for M <= 16 tokens (decode), "swap-AB": D[n, m] = W_hat[n, :] X[m, :]^T
 // with the dequantized weight as the 128-row MMA operand A (K-major image
-// written by the producer warps) and the tokens as a 16-wide operand B (TMA).
-// The codes stream through a deep TMA ring (weight bytes dominate the
-// traffic); the producer warps also copy the small token tile (loaded one step
-// ahead) into the swizzled B stage; the reduction over K is split across CTAs
-// so every SM streams.  Split s
-// writes fp32 partial[s][m][n] (or Y directly when there is one split); the
-// LoRA steps run in split 0.
-constexpr int kDecCodeStages = 8;               // packed-code ring (the HBM stream)
-constexpr int kDecStages = 2;                   // dequantized-tile / token ring
-constexpr int kDecCtasPerSm = 3;                // ~69 KB of shared memory per CTA
-constexpr int kDecPrefetch = 4;                 // block constants are loaded this many K-steps ahead
-constexpr uint32_t kDecAStage = 128 * 128;      // W_hat or B2 tile [128 rows x 64]
-constexpr uint32_t kDecBStage = 16 * 128;       // X or U2 tile [16 tokens x 64]
+// written by the producer warps) and the tokens as a 16-wide operand B.
+// The work is the sequence of (tile of 128 W rows, K-step of 64) units, tile
+// major; it is cut into G equal contiguous ranges, one per persistent CTA
+// (stream-K), so every SM streams the same number of weight bytes whatever
+// the shape.  A CTA's range crosses tiles: each (tile, CTA) piece is a
+// segment, accumulated in one of two TMEM accumulators and written as an fp32
+// partial tile to slot tile + CTA; decode_fixup then sums each tile's slots in
+// CTA order (deterministic) and adds the LoRA term s U B^T in fp32.
+// Warp roles (320 threads): warp 0 lane 0 streams the packed codes through a
+// TMA ring; warp 1 owns TMEM and issues tcgen05.mma; warps 2-9 are two
+// producer groups of 4 warps that take alternate units (one W row of 64
+// weights per thread per unit, plus the token tile), and each group runs the
+// epilogue of the segments that use its accumulator.
+constexpr int kDecThreads = 320;
+constexpr int kDecCtasPerSm = 2;                // ~105 KB of shared memory per CTA
+constexpr int kDecMaxCtas = 1024;
+constexpr int kDecCodeStages = 8;               // packed-code ring (the HBM stream); stage parity = group
+constexpr int kDecStages = 4;                   // dequantized-tile / token ring; stage parity = group
+constexpr int kDecPrefetch = 4;                 // block constants are loaded this many units (of the group) ahead
+constexpr uint32_t kDecAStage = 128 * 128;      // W_hat tile [128 rows x 64]
+constexpr uint32_t kDecBStage = 16 * 128;       // X tile [16 tokens x 64]
 constexpr uint32_t kDecCodesStage = 128 * 32;   // packed codes [128 rows x 32 bytes]
 constexpr uint32_t kDecOffB = kDecStages * kDecAStage;
 constexpr uint32_t kDecOffCodes = kDecOffB + kDecStages * kDecBStage;
 constexpr uint32_t kDecOffBars = kDecOffCodes + kDecCodeStages * kDecCodesStage;
-// barriers: cfull[CS], cempty[CS], afull[S], aempty[S], acc
-constexpr uint32_t kDecOffSlot = kDecOffBars + (2 * kDecCodeStages + 2 * kDecStages + 1) * 8;
+// barriers: cfull[CS], cempty[CS], afull[S], aempty[S], accfull[2], accempty[2], drain
+constexpr uint32_t kDecNumBars = 2 * kDecCodeStages + 2 * kDecStages + 5;
+constexpr uint32_t kDecOffSlot = kDecOffBars + kDecNumBars * 8;
 constexpr uint32_t kDecOffAbort = kDecOffSlot + 4;
 constexpr uint32_t kDecAlloc = kDecOffAbort + 4 + 1024;
+constexpr uint32_t kDecSlotFloats = 16 * 128;   // one partial tile: [16 tokens][128 rows] fp32
 
-__global__ void __launch_bounds__(kThreads, kDecCtasPerSm)
+// First unit of CTA b when U units are cut into G ranges.
+__host__ __device__ __forceinline__ int64_t dec_range_begin(int64_t b, int64_t U, int64_t G) { return b * U / G; }
+
+__global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm)
 tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, DecodeParams p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t base = (ptx::smem_addr(smem_raw) + 1023u) & ~1023u;
@@ -421,17 +436,18 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, DecodeParams p) {
     const uint32_t bar_cempty = bar_cfull + 8 * kDecCodeStages;
     const uint32_t bar_afull = bar_cempty + 8 * kDecCodeStages;
     const uint32_t bar_aempty = bar_afull + 8 * kDecStages;
-    const uint32_t bar_acc = bar_aempty + 8 * kDecStages;
+    const uint32_t bar_accfull = bar_aempty + 8 * kDecStages;
+    const uint32_t bar_accempty = bar_accfull + 16;
+    const uint32_t bar_drain = bar_accempty + 16;
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gbase + kDecOffSlot);
     volatile int* abort = reinterpret_cast<volatile int*>(gbase + kDecOffAbort);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t n0 = (int64_t)blockIdx.x * 128;
-    const int split = blockIdx.y;
-    const int kbeg = split * p.kps;
-    const int nk0 = max(0, min(p.ksteps0, kbeg + p.kps) - kbeg);
-    const int nk1 = split == 0 ? p.ksteps1 : 0;
-    const int ntot = nk0 + nk1;
+    const int S = p.ksteps;                                   // units per tile
+    const int64_t u0 = dec_range_begin(blockIdx.x, p.units, p.grid);
+    const int n = (int)(dec_range_begin(blockIdx.x + 1, p.units, p.grid) - u0);   // units of this CTA
+    const int64_t t0 = u0 / S;                                // tile of the first segment
+    const int step0 = (int)(u0 - t0 * S);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kDecCodeStages; ++s) {
@@ -442,7 +458,11 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, DecodeParams p) {
             ptx::mbar_init(bar_afull + 8 * s, 4);
             ptx::mbar_init(bar_aempty + 8 * s, 1);
         }
-        ptx::mbar_init(bar_acc, 1);
+        for (int a = 0; a < 2; ++a) {
+            ptx::mbar_init(bar_accfull + 8 * a, 1);
+            ptx::mbar_init(bar_accempty + 8 * a, 4);
+        }
+        ptx::mbar_init(bar_drain, 1);
         *abort = 0;
         ptx::fence_barrier_init();
         ptx::fence_proxy_async_smem();
@@ -459,19 +479,21 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, DecodeParams p) {
 
     if (warp == 0) {
         if (lane == 0) {
-            // packed codes run up to kDecCodeStages steps ahead of the producers (cempty is
-            // observed phase by phase, in order); nothing else is loaded by TMA
+            // codes of unit i go to stage i % kDecCodeStages; cempty is observed phase by phase
             bool ok = true;
             int issued = 0;
-            for (int c = 0; c < nk0 && ok; ++c) {
-                const int cs = c % kDecCodeStages;
-                const uint32_t cph = (uint32_t)(c / kDecCodeStages) & 1u;
+            int64_t tile = t0;
+            int step = step0;
+            for (int i = 0; i < n && ok; ++i) {
+                const int cs = i % kDecCodeStages;
+                const uint32_t cph = (uint32_t)(i / kDecCodeStages) & 1u;
                 ok = ptx::mbar_wait(bar_cempty + 8 * cs, cph ^ 1u, abort, p.err);
                 if (!ok) break;
                 ptx::mbar_arrive_expect_tx(bar_cfull + 8 * cs, kDecCodesStage);
-                ptx::tma_load_2d(sCodes + cs * kDecCodesStage, &tmCodes, (kbeg + c) * 32, (int32_t)n0,
+                ptx::tma_load_2d(sCodes + cs * kDecCodesStage, &tmCodes, step * 32, (int32_t)(tile * 128),
                                  bar_cfull + 8 * cs);
-                issued = c + 1;
+                issued = i + 1;
+                if (++step == S) { step = 0; ++tile; }
             }
             if (*abort) {   // drain this CTA's copies in flight before it exits
                 for (int c = max(0, issued - kDecCodeStages); c < issued; ++c)
@@ -482,7 +504,15 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, DecodeParams p) {
         if (lane == 0) {
             constexpr uint32_t idesc = ptx::idesc_bf16_f32_ab(128, 16, 0, 0);
             bool ok = true;
-            for (int i = 0; i < ntot && ok; ++i) {
+            int step = step0, seg = 0;
+            bool fresh = true;                                // first unit of a segment: overwrite
+            for (int i = 0; i < n && ok; ++i) {
+                const int a = seg & 1;
+                if (fresh && seg >= 2) {                      // accumulator a drained by segment seg-2's epilogue
+                    ok = ptx::mbar_wait(bar_accempty + 8 * a, (uint32_t)((seg - 2) >> 1) & 1u, abort, p.err);
+                    if (!ok) { atomicMax(p.dbg, 0x61000000u | (uint32_t)i); break; }
+                    ptx::tc_fence_after();
+                }
                 const int s = i % kDecStages;
                 const uint32_t ph = (uint32_t)(i / kDecStages) & 1u;
                 ok = ptx::mbar_wait(bar_afull + 8 * s, ph, abort, p.err);
@@ -491,96 +521,112 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, DecodeParams p) {
                 const uint32_t a_base = sA + s * kDecAStage, b_base = sB + s * kDecBStage;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    ptx::mma_bf16_ss(tmem, ptx::smem_desc_sw128(a_base + kk * 32, 16, 1024),
+                    ptx::mma_bf16_ss(tmem + 16u * (uint32_t)a, ptx::smem_desc_sw128(a_base + kk * 32, 16, 1024),
                                      ptx::smem_desc_sw128(b_base + kk * 32, 16, 1024), idesc,
-                                     (i | kk) != 0 ? 1u : 0u);
+                                     (!fresh || kk != 0) ? 1u : 0u);
                 ptx::mma_commit(bar_aempty + 8 * s);
+                fresh = false;
+                if (++step == S || i == n - 1) {              // segment ends: hand the accumulator over
+                    ptx::mma_commit(bar_accfull + 8 * a);
+                    step = step == S ? 0 : step;
+                    ++seg;
+                    fresh = true;
+                }
             }
-            ptx::mma_commit(bar_acc);
-            if (*abort) ptx::mbar_wait_drain(bar_acc, 0);   // issued MMAs finish before TMEM is freed
+            ptx::mma_commit(bar_drain);
+            if (*abort) ptx::mbar_wait_drain(bar_drain, 0);   // issued MMAs finish before TMEM is freed
         }
     } else {
-        // producers: thread t expands W row n0 + t for every K-step of this split, and copies
-        // 16 bytes of the token tile (token t >> 3, 16-byte chunk t & 7), loaded one step ahead
-        const int t = threadIdx.x - 64;
-        const int64_t n = n0 + t;
-        const bool row_ok = n < p.N;
+        // producer group g takes units g, g + 2, ...; thread t expands W row tile*128 + t of each
+        // and copies 16 bytes of its token tile (token t >> 3, 16-byte chunk t & 7)
+        const int g = (warp - 2) >> 2;
+        const int t = threadIdx.x - 64 - 128 * g;
         const int xm = t >> 3, xc = t & 7;
         const bool x_ok = xm < p.M;
-        const uint4* xsrc = static_cast<const uint4*>(p.X) + (int64_t)xm * (p.K / 8) + xc;
-        uint4 xnext = make_uint4(0, 0, 0, 0);
+        const uint4* xrow = static_cast<const uint4*>(p.X) + (int64_t)xm * (p.K / 8) + xc;
         const int64_t nb1 = p.N * (p.K / 64);
-        // bounds self-check of the token loads: column (step*64 + xc*8 .. +7) of token xm < M
-        auto x_in_bounds = [&](int step) -> bool {
-            const int64_t col = (int64_t)step * 64 + xc * 8;
-            const bool in = xm < p.M && col + 8 <= p.K && step >= 0;
-            if (!in) { atomicOr(p.err, ERR_FLAG_BOUNDS); atomicMax(p.dbg, 0x10000000u | (uint32_t)step); }
-            return in;
-        };
-        if (x_ok && nk0 > 0 && x_in_bounds(kbeg)) xnext = __ldg(xsrc + (int64_t)kbeg * 8);
+        const int64_t kb = p.K / 64;
         const float mu = *p.mu;
-        const int64_t blk0 = n * (p.K / 64) + kbeg;
-        // block constants of steps i .. i+kDecPrefetch-1 (register queue, shifted each step)
+        // unit cursors: (tile, step) of the current unit, of the next one (token tile) and of the
+        // prefetch head (block constants); each moves by 2 units
+        auto advance = [S](int64_t& tile, int& step, int by) {
+            step += by;
+            while (step >= S) { step -= S; ++tile; }
+        };
+        int64_t cur_tile = t0; int cur_step = step0;
+        advance(cur_tile, cur_step, g);
+        auto x_load = [&](int64_t step) -> uint4 {
+            const int64_t col = step * 64 + xc * 8;
+            if (!(x_ok && col + 8 <= p.K)) {
+                if (x_ok) { atomicOr(p.err, ERR_FLAG_BOUNDS); atomicMax(p.dbg, 0x10000000u | (uint32_t)step); }
+                return make_uint4(0, 0, 0, 0);
+            }
+            return __ldg(xrow + step * 8);
+        };
+        auto const_load = [&](int64_t tile, int step, uint32_t& code, float& c2) {
+            code = 0; c2 = 0.f;
+            const int64_t row = tile * 128 + t;
+            if (row >= p.N) return;
+            const int64_t blk = row * kb + step;
+            if (blk >= nb1 || step >= kb) { atomicOr(p.err, ERR_FLAG_BOUNDS); atomicMax(p.dbg, 0x20000000u); return; }
+            code = __ldg(p.c1_codes + blk);
+            c2 = __ldg(p.c2 + (blk >> 8));
+        };
+        uint4 xnext = make_uint4(0, 0, 0, 0);
+        if (g < n) xnext = x_load(cur_step);
         uint32_t qcode[kDecPrefetch];
         float qc2[kDecPrefetch];
+        int64_t pf_tile = cur_tile; int pf_step = cur_step;
 #pragma unroll
         for (int d = 0; d < kDecPrefetch; ++d) {
-            qcode[d] = 0;
-            qc2[d] = 0.f;
-            if (row_ok && d < nk0) {
-                if (blk0 + d >= nb1) { atomicOr(p.err, ERR_FLAG_BOUNDS); atomicMax(p.dbg, 0x20000000u); continue; }
-                qcode[d] = __ldg(p.c1_codes + blk0 + d);
-                qc2[d] = __ldg(p.c2 + ((blk0 + d) >> 8));
-            }
+            qcode[d] = 0; qc2[d] = 0.f;
+            if (g + 2 * d < n) const_load(pf_tile, pf_step, qcode[d], qc2[d]);
+            advance(pf_tile, pf_step, 2);
         }
-        bool ok = true;
-        for (int i = 0; i < ntot && ok; ++i) {
-            if (i >= nk0) {
-                // LoRA step: copy B2[n0 + t, j*64 .. +63] into the A stage and 16 bytes of
-                // U2[token, j*64 ..] into the B stage (zero outside the matrices)
-                const int s = i % kDecStages;
-                const uint32_t ph = (uint32_t)(i / kDecStages) & 1u;
-                const int j = i - nk0;
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_aempty + 8 * s, ph ^ 1u, abort, p.err));
-                if (!ok) break;
-                const int64_t R2 = 2 * (int64_t)p.Rpad;
-                const uint32_t row_addr = sA + s * kDecAStage + (uint32_t)t * 128u;
-                if (row_ok) {
-                    const uint4* src = static_cast<const uint4*>(p.B2) + (n * R2 + (int64_t)j * 64) / 8;
+        int64_t nx_tile = cur_tile; int nx_step = cur_step;
+        advance(nx_tile, nx_step, 2);
+
+        int epi_seg = g;                                      // next segment whose epilogue is ours
+        const int last_seg = (int)((u0 + n - 1) / S - t0);
+        auto epilogue = [&](int seg) -> bool {
+            const int a = seg & 1;
+            const bool ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_accfull + 8 * a, (uint32_t)(seg >> 1) & 1u,
+                                                                    abort, p.err));
+            if (!ok) { if (lane == 0) atomicMax(p.dbg, 0x70000000u | (uint32_t)seg); return false; }
+            ptx::tc_fence_after();
+            const uint32_t quad = (uint32_t)(warp & 3);
+            uint32_t v[16];
+            ptx::tmem_ld_32x32b_x16(tmem + ((quad * 32u) << 16) + 16u * (uint32_t)a, v);
+            ptx::tmem_ld_wait();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar_accempty + 8 * a);
+            float* dst = p.partial + (t0 + seg + (int64_t)blockIdx.x) * kDecSlotFloats + quad * 32 + lane;
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) st_shared_v4(row_addr + ((c ^ (t & 7)) << 4), __ldg(src + c));
-                } else {
-                    zero_row(row_addr);
-                }
-                uint4 u = make_uint4(0, 0, 0, 0);
-                if (x_ok) u = __ldg(static_cast<const uint4*>(p.U2) + ((int64_t)xm * R2 + (int64_t)j * 64) / 8 + xc);
-                st_shared_v4(sB + s * kDecBStage + (uint32_t)xm * 128u + ((uint32_t)(xc ^ (xm & 7)) << 4), u);
-                ptx::fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(bar_afull + 8 * s);
-                continue;
-            }
+            for (int m = 0; m < 16; ++m)
+                if (m < p.M) dst[m * 128] = __uint_as_float(v[m]);
+            return true;
+        };
+
+        bool ok = true;
+        for (int i = g; i < n && ok; i += 2) {
+            const int seg = (int)(cur_tile - t0);
+            while (epi_seg < seg && ok) { ok = epilogue(epi_seg); epi_seg += 2; }
+            if (!ok) break;
             const int cs = i % kDecCodeStages;
             const uint32_t cph = (uint32_t)(i / kDecCodeStages) & 1u;
             const int s = i % kDecStages;
             const uint32_t ph = (uint32_t)(i / kDecStages) & 1u;
             const float c1p = rebuild_c1(qcode[0], qc2[0], mu);
             const uint4 xcur = xnext;
-            if (x_ok && i + 1 < nk0 && x_in_bounds(kbeg + i + 1)) xnext = __ldg(xsrc + (int64_t)(kbeg + i + 1) * 8);
+            if (i + 2 < n) xnext = x_load(nx_step);
 #pragma unroll
             for (int d = 0; d + 1 < kDecPrefetch; ++d) {
                 qcode[d] = qcode[d + 1];
                 qc2[d] = qc2[d + 1];
             }
-            if (row_ok && i + kDecPrefetch < nk0) {
-                if (blk0 + i + kDecPrefetch < nb1) {
-                    qcode[kDecPrefetch - 1] = __ldg(p.c1_codes + blk0 + i + kDecPrefetch);
-                    qc2[kDecPrefetch - 1] = __ldg(p.c2 + ((blk0 + i + kDecPrefetch) >> 8));
-                } else {
-                    atomicOr(p.err, ERR_FLAG_BOUNDS);
-                    atomicMax(p.dbg, 0x30000000u | (uint32_t)i);
-                }
-            }
+            qcode[kDecPrefetch - 1] = 0; qc2[kDecPrefetch - 1] = 0.f;
+            if (i + 2 * kDecPrefetch < n) const_load(pf_tile, pf_step, qcode[kDecPrefetch - 1], qc2[kDecPrefetch - 1]);
             bool w_ok = ptx::mbar_wait(bar_cfull + 8 * cs, cph, abort, p.err);
             if (!w_ok) atomicMax(p.dbg, 0x40000000u | (uint32_t)i);
             w_ok = w_ok && ptx::mbar_wait(bar_aempty + 8 * s, ph ^ 1u, abort, p.err);
@@ -589,7 +635,7 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, DecodeParams p) {
             if (!ok) break;
             st_shared_v4(sB + s * kDecBStage + (uint32_t)xm * 128u + ((uint32_t)(xc ^ (xm & 7)) << 4), xcur);
             const uint32_t row_addr = sA + s * kDecAStage + (uint32_t)t * 128u;
-            if (!row_ok) {
+            if (cur_tile * 128 + t >= p.N) {
                 zero_row(row_addr);
             } else {
                 const uint32_t src = sCodes + cs * kDecCodesStage + (uint32_t)t * 32u;
@@ -606,31 +652,11 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, DecodeParams p) {
                 ptx::mbar_arrive(bar_cempty + 8 * cs);
                 ptx::mbar_arrive(bar_afull + 8 * s);
             }
+            advance(cur_tile, cur_step, 2);
+            advance(nx_tile, nx_step, 2);
+            advance(pf_tile, pf_step, 2);
         }
-        // epilogue: lane quadrant (warp & 3) holds W rows n0 + 32*quad + lane, columns = tokens
-        const bool acc_ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_acc, 0, abort, p.err));
-        ptx::tc_fence_after();
-        if (acc_ok && ntot > 0) {
-            const uint32_t quad = (uint32_t)(warp & 3);
-            uint32_t v[16];
-            ptx::tmem_ld_32x32b_x16(tmem + ((quad * 32u) << 16), v);
-            ptx::tmem_ld_wait();
-            const int64_t nn = n0 + quad * 32 + lane;
-            if (nn < p.N) {
-#pragma unroll
-                for (int m = 0; m < 16; ++m) {
-                    if (m >= p.M) break;
-                    const float val = __uint_as_float(v[m]);
-                    if (p.splits > 1) {
-                        p.partial[((int64_t)split * p.M + m) * p.N + nn] = val;
-                    } else if (p.out_f32) {
-                        static_cast<float*>(p.out)[(int64_t)m * p.N + nn] = val;
-                    } else {
-                        static_cast<uint16_t*>(p.out)[(int64_t)m * p.N + nn] = (uint16_t)f32_to_bf16_bits_rn(val);
-                    }
-                }
-            }
-        }
+        while (ok && epi_seg <= last_seg) { ok = epilogue(epi_seg); epi_seg += 2; }
     }
 
     ptx::tc_fence_before();
@@ -641,14 +667,107 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, DecodeParams p) {
     }
 }
 
-// out[m, n] = sum over splits of partial[s][m][n] (fixed order), converted to the output type.
-__global__ void decode_reduce(const float* __restrict__ partial, int splits, int64_t MN, void* out, int out_f32) {
-    const int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x;
-    if (i >= MN) return;
+// U[m, j] = sum_k X[m, k] A[j, k] in fp32 (one CTA per (j, m); fixed reduction order).
+__global__ void __launch_bounds__(256)
+decode_lora_u(const uint4* __restrict__ X, const uint4* __restrict__ A, int64_t K8, int r, float* __restrict__ U) {
+    const int j = blockIdx.x, m = blockIdx.y;
+    const uint4* xr = X + (int64_t)m * K8;
+    const uint4* ar = A + (int64_t)j * K8;
     float acc = 0.f;
-    for (int s = 0; s < splits; ++s) acc = __fadd_rn(acc, partial[(int64_t)s * MN + i]);
-    if (out_f32) static_cast<float*>(out)[i] = acc;
-    else static_cast<uint16_t*>(out)[i] = (uint16_t)f32_to_bf16_bits_rn(acc);
+    for (int64_t c0 = threadIdx.x; c0 < K8; c0 += 4 * 256) {
+        uint4 xv[4], av[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {                         // four 16-byte chunks in flight per thread
+            const int64_t c = c0 + q * 256;
+            xv[q] = c < K8 ? __ldg(xr + c) : make_uint4(0, 0, 0, 0);
+            av[q] = c < K8 ? __ldg(ar + c) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t xw[4] = {xv[q].x, xv[q].y, xv[q].z, xv[q].w};
+            const uint32_t aw[4] = {av[q].x, av[q].y, av[q].z, av[q].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                acc = __fmaf_rn(bf16_bits_to_f32(xw[e] & 0xFFFFu), bf16_bits_to_f32(aw[e] & 0xFFFFu), acc);
+                acc = __fmaf_rn(bf16_bits_to_f32(xw[e] >> 16), bf16_bits_to_f32(aw[e] >> 16), acc);
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, o));
+    __shared__ float ws[8];
+    if ((threadIdx.x & 31) == 0) ws[threadIdx.x >> 5] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float s = 0.f;
+        for (int w = 0; w < 8; ++w) s = __fadd_rn(s, ws[w]);
+        U[(int64_t)m * r + j] = s;
+    }
+}
+
+// Y[m, n] = sum over the CTAs b covering tile n / 128 of partial[tile + b][m][n % 128] (in b
+// order) + scale * sum_j U[m, j] B[n, j], converted to the output type.  One CTA per tile;
+// every group of loads is issued back to back (the kernel is latency-bound, not bandwidth-bound).
+__global__ void __launch_bounds__(128)
+decode_fixup(const float* __restrict__ partial, int64_t units, int64_t G, int S, int64_t M, int64_t N,
+             const float* __restrict__ U, const uint16_t* __restrict__ B, int r, float scale, void* out, int out_f32) {
+    extern __shared__ float us[];                             // us[j * 16 + m] = U[m, j]
+    for (int i = threadIdx.x; i < r * 16; i += 128) {
+        const int j = i >> 4, m = i & 15;
+        us[i] = m < M ? U[(int64_t)m * r + j] : 0.f;
+    }
+    __syncthreads();
+    const int64_t tile = blockIdx.x;
+    const int64_t n = tile * 128 + threadIdx.x;
+    if (n >= N) return;
+    auto cta_of = [&](int64_t u) {                            // the CTA whose range holds unit u
+        int64_t b = u * G / units;
+        while (b + 1 < G && dec_range_begin(b + 1, units, G) <= u) ++b;
+        while (b > 0 && dec_range_begin(b, units, G) > u) --b;
+        return b;
+    };
+    const int64_t ba = cta_of(tile * S), bz = cta_of(tile * S + S - 1);
+    float acc[16];
+#pragma unroll
+    for (int m = 0; m < 16; ++m) acc[m] = 0.f;
+    for (int64_t b = ba; b <= bz; ++b) {
+        const float* pp = partial + (tile + b) * kDecSlotFloats + threadIdx.x;
+        float v[16];
+#pragma unroll
+        for (int m = 0; m < 16; ++m) v[m] = m < M ? pp[m * 128] : 0.f;
+#pragma unroll
+        for (int m = 0; m < 16; ++m) acc[m] = __fadd_rn(acc[m], v[m]);
+    }
+    float lora[16];
+#pragma unroll
+    for (int m = 0; m < 16; ++m) lora[m] = 0.f;
+    const uint16_t* brow = B + n * r;
+    for (int j0 = 0; j0 < r; j0 += 8) {
+        float bv[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) bv[q] = j0 + q < r ? bf16_bits_to_f32(brow[j0 + q]) : 0.f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            if (j0 + q >= r) continue;
+            const float4* uj = reinterpret_cast<const float4*>(us + (j0 + q) * 16);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float4 u4 = uj[c];
+                lora[4 * c + 0] = __fmaf_rn(u4.x, bv[q], lora[4 * c + 0]);
+                lora[4 * c + 1] = __fmaf_rn(u4.y, bv[q], lora[4 * c + 1]);
+                lora[4 * c + 2] = __fmaf_rn(u4.z, bv[q], lora[4 * c + 2]);
+                lora[4 * c + 3] = __fmaf_rn(u4.w, bv[q], lora[4 * c + 3]);
+            }
+        }
+    }
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+        if (m < M) {
+            const float y = __fmaf_rn(scale, lora[m], acc[m]);
+            if (out_f32) static_cast<float*>(out)[m * N + n] = y;
+            else static_cast<uint16_t*>(out)[m * N + n] = (uint16_t)f32_to_bf16_bits_rn(y);
+        }
+    }
 }
 
 // ---------------------------------------------------------------------------- host
@@ -702,33 +821,40 @@ static qlora_status launch_one(const TcGemmArgs& a, cudaStream_t stream) {
 }
 
 // Splits of the reduction so that tiles x splits fills one wave of CTAs.
-int decode_splits(int64_t N, int ksteps0, int sms) {
-    const int64_t tiles = (N + 127) / 128;
-    const int64_t slots = kDecCtasPerSm * (int64_t)sms;
-    int64_t sp = slots / tiles;
-    if (sp > 16) sp = 16;
-    if (sp > ksteps0) sp = ksteps0;
-    return sp < 1 ? 1 : (int)sp;
+static int64_t decode_grid(int64_t units, int sms) {
+    return std::max<int64_t>(1, std::min<int64_t>({units, (int64_t)kDecCtasPerSm * sms, (int64_t)kDecMaxCtas}));
+}
+
+size_t decode_partial_bytes(int64_t N, int64_t K) {
+    const int64_t tiles = (N + 127) / 128, units = tiles * (K / 64);
+    const int64_t slots = tiles + std::min<int64_t>(units, kDecMaxCtas);
+    return (size_t)slots * kDecSlotFloats * sizeof(float);
 }
 
 qlora_status launch_tc_decode(const DecodeArgs& a, cudaStream_t stream) {
     const qlora_nf4_weight* w = a.w;
     const int64_t N = w->N, K = w->K;
-    const int64_t R2 = 2 * (int64_t)a.Rpad;
+    static int sms = 0;
+    if (sms == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return QLORA_ERR_CUDA;
+    }
     CUtensorMap tmCodes;
     if (!make_tmap_2d(&tmCodes, false, w->codes, K / 2, N, K / 2, 32, 128, false)) return QLORA_ERR_CUDA;
     DecodeParams p{};
-    p.M = a.M; p.N = N; p.K = K; p.X = a.X; p.U2 = a.U2; p.B2 = a.B2; p.Rpad = a.Rpad;
-    p.dbg = device_error_word() ? device_error_word() + 1 : nullptr;
-    p.ksteps0 = (int)(K / 64);
-    p.ksteps1 = (int)(R2 / 64);
-    p.kps = (p.ksteps0 + a.splits - 1) / a.splits;
-    p.splits = (p.ksteps0 + p.kps - 1) / p.kps;          // every split gets at least one K-step
+    p.M = a.M; p.N = N; p.K = K; p.X = a.X;
+    p.ksteps = (int32_t)(K / 64);
+    const int64_t tiles = (N + 127) / 128;
+    p.units = tiles * p.ksteps;
+    p.grid = decode_grid(p.units, sms);
     p.c1_codes = w->c1_codes; p.c2 = w->c2; p.mu = w->mu;
-    p.out = a.out; p.out_f32 = a.out_f32; p.partial = a.partial;
+    p.partial = a.partial;
     p.tb = host_tables();
     p.err = device_error_word();
     if (!p.err) return QLORA_ERR_CUDA;
+    p.dbg = p.err + 1;
     static bool configured = false;
     if (!configured) {
         if (cudaFuncSetAttribute(tc_decode_nf4, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDecAlloc) !=
@@ -736,14 +862,15 @@ qlora_status launch_tc_decode(const DecodeArgs& a, cudaStream_t stream) {
             return QLORA_ERR_CUDA;
         configured = true;
     }
-    const dim3 grid((unsigned)((N + 127) / 128), (unsigned)p.splits);
-    tc_decode_nf4<<<grid, kThreads, kDecAlloc, stream>>>(tmCodes, p);
+    decode_lora_u<<<dim3((unsigned)a.r, (unsigned)a.M), 256, 0, stream>>>(
+        static_cast<const uint4*>(a.X), static_cast<const uint4*>(a.A), K / 8, a.r, a.U);
     QLORA_CHECK_LAUNCH();
-    if (p.splits > 1) {
-        const int64_t MN = a.M * N;
-        decode_reduce<<<(unsigned)((MN + 255) / 256), 256, 0, stream>>>(a.partial, p.splits, MN, a.out, a.out_f32);
-        QLORA_CHECK_LAUNCH();
-    }
+    tc_decode_nf4<<<(unsigned)p.grid, kDecThreads, kDecAlloc, stream>>>(tmCodes, p);
+    QLORA_CHECK_LAUNCH();
+    decode_fixup<<<(unsigned)tiles, 128, (size_t)a.r * 16 * sizeof(float), stream>>>(
+        a.partial, p.units, p.grid, p.ksteps, a.M, N, a.U, static_cast<const uint16_t*>(a.B), a.r, a.scale, a.out,
+        a.out_f32);
+    QLORA_CHECK_LAUNCH();
     return QLORA_OK;
 }
 

@@ -36,20 +36,18 @@ struct TcGemmArgs {
 // Encodes the tensor maps and launches the forward (dx = false) or dX kernel.
 qlora_status launch_tc_gemm_nf4(TcGemmArgs& a, bool dx, cudaStream_t stream);
 
-// Small-M forward (M <= 16): swap-AB fused dequant-GEMM with split-K.
+// Small-M forward (M <= 16): swap-AB fused dequant-GEMM, stream-K over
+// (tile, K-step) units with fp32 partial tiles and a fixup that adds the LoRA term.
 struct DecodeParams {
     int64_t M, N, K;
     const void* X;          // [M, K] bf16 (read by the producer warps)
-    const void* U2;         // [M, 2*Rpad] bf16 (LoRA steps, read by the producer warps)
-    const void* B2;         // [N, 2*Rpad] bf16
-    int32_t Rpad;
-    int32_t ksteps0, ksteps1, kps, splits;
+    int32_t ksteps;         // K / 64: units per tile of 128 W rows
+    int64_t units;          // tiles * ksteps
+    int64_t grid;           // persistent CTAs; CTA b takes units [b*units/grid, (b+1)*units/grid)
     const uint8_t* c1_codes;
     const float* c2;
     const float* mu;
-    void* out;
-    int32_t out_f32;
-    float* partial;         // [splits, M, N] fp32 when splits > 1
+    float* partial;         // [tiles + grid][16][128] fp32 partial tiles, slot = tile + CTA
     uint32_t* err;
     uint32_t* dbg;          // second device word: where a self-check or a wait gave up
     NF4Tables tb;
@@ -58,18 +56,19 @@ struct DecodeParams {
 struct DecodeArgs {
     const qlora_nf4_weight* w;
     const void* X;          // [M, K] bf16
-    const void* U2;         // [M, 2*Rpad] bf16 hi/lo of s*U
-    const void* B2;         // [N, 2*Rpad] bf16
-    int32_t Rpad;
+    const void* A;          // [r, K] bf16
+    const void* B;          // [N, r] bf16
+    int32_t r;
+    float scale;            // alpha / r
     int64_t M;
     void* out;
     int32_t out_f32;
-    float* partial;
-    int32_t splits;
+    float* U;               // [M, r] fp32, written (X A^T)
+    float* partial;         // decode_partial_bytes(N, K)
 };
 
 constexpr int64_t kDecodeMaxM = 16;
-int decode_splits(int64_t N, int ksteps0, int sms);
+size_t decode_partial_bytes(int64_t N, int64_t K);
 qlora_status launch_tc_decode(const DecodeArgs& a, cudaStream_t stream);
 
 // LoRA-side GEMM (gemm_lora_tc.cu): partial[split][rows][R] = sum over the

@@ -8,8 +8,8 @@
 //                        block, packed 16-bit max), correctly rounded
 //                        division, bucketed code search with one compare,
 //                        nibble packing; writes the packed codes, the fp32
-//                        absmax c1 per block, and the fp64 sum of each chunk
-//                        of 128 c1 values over a fixed pairwise tree.
+//                        absmax c1 per block, and the fp64 sum of each
+//                        warp's 16 c1 values over a fixed pairwise tree.
 //   tree_sum_pass        fp64 pairwise-tree sums of 1024 partials per CTA,
 //                        repeated until one value is left.
 //   dq_blocks            per group of 256 blocks: mu from the tree sum,
@@ -74,26 +74,34 @@ __device__ __forceinline__ uint32_t nf4_code(float x, const float2* __restrict__
 }
 
 // One pass over W.  Persistent CTAs loop over chunks of 128 consecutive NF4
-// blocks; two threads share a block (32 weights each).  Per chunk: packed
-// codes, fp32 block absmax, and the chunk's fp64 pairwise-tree sum of c1.
+// blocks (the next chunk's weights are loaded while the current one is coded);
+// two threads share a block (32 weights each).  Per chunk: packed codes, fp32
+// block absmax, and per warp the fp64 pairwise-tree sum of its 16 blocks' c1
+// (aligned subtrees of the global tree, combined by tree_sum_pass).
 __global__ void __launch_bounds__(kQuantThreads, kCtasPerSm)
 nf4_quantize_blocks(const uint4* __restrict__ W, int64_t nb1, uint4* __restrict__ codes,
-                    float* __restrict__ c1_out, double* __restrict__ chunk_sums, int64_t n_chunks,
+                    float* __restrict__ c1_out, double* __restrict__ warp_sums_out, int64_t n_chunks,
                     QuantBuckets qb) {
     __shared__ float2 table[kTableWords];
-    __shared__ double warp_sums[kQuantThreads / 32];
     for (int i = threadIdx.x; i < kTableWords; i += kQuantThreads) table[i] = qb.e[i >> 5];
     __syncthreads();
     const float2* lane_table = table + (threadIdx.x & 31);
     const int sub = threadIdx.x & 1;
+
+    uint4 nxt[4];
+    auto load_chunk = [&](int64_t chunk) {
+        const int64_t blk = chunk * kBlocksPerCta + (threadIdx.x >> 1);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            nxt[j] = (chunk < n_chunks && blk < nb1) ? W[blk * 8 + sub * 4 + j] : make_uint4(0, 0, 0, 0);
+    };
+    load_chunk(blockIdx.x);
     for (int64_t chunk = blockIdx.x; chunk < n_chunks; chunk += gridDim.x) {
         const int64_t blk = chunk * kBlocksPerCta + (threadIdx.x >> 1);
         const bool valid = blk < nb1;
-        uint4 v4[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) v4[j] = valid ? W[blk * 8 + sub * 4 + j] : make_uint4(0, 0, 0, 0);
-        const uint32_t w[16] = {v4[0].x, v4[0].y, v4[0].z, v4[0].w, v4[1].x, v4[1].y, v4[1].z, v4[1].w,
-                                v4[2].x, v4[2].y, v4[2].z, v4[2].w, v4[3].x, v4[3].y, v4[3].z, v4[3].w};
+        const uint32_t w[16] = {nxt[0].x, nxt[0].y, nxt[0].z, nxt[0].w, nxt[1].x, nxt[1].y, nxt[1].z, nxt[1].w,
+                                nxt[2].x, nxt[2].y, nxt[2].z, nxt[2].w, nxt[3].x, nxt[3].y, nxt[3].z, nxt[3].w};
+        load_chunk(chunk + gridDim.x);
         // block absmax on the bf16 bit patterns: |w| orders like the unsigned 15-bit magnitude
         uint32_t mx = 0;
 #pragma unroll
@@ -106,17 +114,19 @@ nf4_quantize_blocks(const uint4* __restrict__ W, int64_t nb1, uint4* __restrict_
         if (valid) {
             uint32_t out[4] = {0x77777777u, 0x77777777u, 0x77777777u, 0x77777777u};  // all-zero block: code 7
             if (m > 0.f && mbits < 0x7F80u) {
+                // weights are coded in the order 6,7,4,5,2,3,0,1 of each group of 8 so that
+                // word = 16 * word + code leaves weight 2j in the high nibble of byte j
                 if ((m >= 7.8886091e-31f) && (m <= 1.2676506e30f)) {   // 2^-100 .. 2^100: Markstein division
                     const float y = __frcp_rn(m);
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         uint32_t word = 0;
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {     // weights 8q .. 8q+7 of this thread
+                        for (int jj = 0; jj < 8; ++jj) {
+                            const int i = (6 - 2 * (jj >> 1)) + (jj & 1);
                             const uint32_t pair = w[4 * q + (i >> 1)];
                             const float v = __uint_as_float((i & 1) ? (pair & 0xFFFF0000u) : (pair << 16));
-                            const uint32_t c = nf4_code(div_markstein(v, m, y), lane_table);
-                            word |= c << (8 * (i >> 1) + ((i & 1) ? 0 : 4));   // weight 2j -> high nibble
+                            word = word * 16u + nf4_code(div_markstein(v, m, y), lane_table);
                         }
                         out[q] = word;
                     }
@@ -125,11 +135,11 @@ nf4_quantize_blocks(const uint4* __restrict__ W, int64_t nb1, uint4* __restrict_
                     for (int q = 0; q < 4; ++q) {
                         uint32_t word = 0;
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
+                        for (int jj = 0; jj < 8; ++jj) {
+                            const int i = (6 - 2 * (jj >> 1)) + (jj & 1);
                             const uint32_t pair = w[4 * q + (i >> 1)];
                             const float v = __uint_as_float((i & 1) ? (pair & 0xFFFF0000u) : (pair << 16));
-                            const uint32_t c = nf4_code(__fdiv_rn(v, m), lane_table);
-                            word |= c << (8 * (i >> 1) + ((i & 1) ? 0 : 4));
+                            word = word * 16u + nf4_code(__fdiv_rn(v, m), lane_table);
                         }
                         out[q] = word;
                     }
@@ -139,20 +149,14 @@ nf4_quantize_blocks(const uint4* __restrict__ W, int64_t nb1, uint4* __restrict_
             if (sub == 0) c1_out[blk] = m;
         }
 
-        // fp64 pairwise tree over the chunk's 128 block constants: even lanes hold the
-        // blocks of the warp in order; xor-shuffles by 2..16 pair neighbours level by level.
+        // fp64 pairwise tree over the warp's 16 blocks (even lanes, in order): xor-shuffles
+        // by 2..16 pair neighbours level by level; one sum per warp
         double s = valid ? (double)m : 0.0;
         s += __shfl_xor_sync(0xffffffffu, s, 2);
         s += __shfl_xor_sync(0xffffffffu, s, 4);
         s += __shfl_xor_sync(0xffffffffu, s, 8);
         s += __shfl_xor_sync(0xffffffffu, s, 16);
-        if ((threadIdx.x & 31) == 0) warp_sums[threadIdx.x >> 5] = s;
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            const double* ws = warp_sums;
-            chunk_sums[chunk] = ((ws[0] + ws[1]) + (ws[2] + ws[3])) + ((ws[4] + ws[5]) + (ws[6] + ws[7]));
-        }
-        __syncthreads();
+        if ((threadIdx.x & 31) == 0) warp_sums_out[chunk * (kQuantThreads / 32) + (threadIdx.x >> 5)] = s;
     }
 }
 
@@ -207,7 +211,7 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // every tree level (P1 = ceil(nb1/128), then ceil(P/1024) until 1).
 size_t quantize_workspace_bytes(int64_t nb1) {
     size_t bytes = align_up((size_t)nb1 * sizeof(float), 256);
-    int64_t p = (nb1 + kBlocksPerCta - 1) / kBlocksPerCta;
+    int64_t p = (nb1 + kBlocksPerCta - 1) / kBlocksPerCta * (kQuantThreads / 32);   // one sum per warp (16 blocks)
     bytes += align_up((size_t)p * sizeof(double), 256);
     while (p > 1) {
         p = (p + kTreeThreads - 1) / kTreeThreads;
@@ -222,15 +226,17 @@ qlora_status launch_quantize(const void* W, int64_t N, int64_t K, const qlora_nf
     char* ws = static_cast<char*>(workspace);
     float* c1 = reinterpret_cast<float*>(ws);
     ws += align_up((size_t)nb1 * sizeof(float), 256);
-    int64_t p = (nb1 + kBlocksPerCta - 1) / kBlocksPerCta;
+    const int64_t n_chunks = (nb1 + kBlocksPerCta - 1) / kBlocksPerCta;
+    int64_t p = n_chunks * (kQuantThreads / 32);                 // first tree level: one sum per 16 blocks
     double* level = reinterpret_cast<double*>(ws);
     ws += align_up((size_t)p * sizeof(double), 256);
 
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t grid = std::min<int64_t>(p, (int64_t)sms * kCtasPerSm);
+    const int64_t grid = std::min<int64_t>(n_chunks, (int64_t)sms * kCtasPerSm);
     nf4_quantize_blocks<<<(unsigned)grid, kQuantThreads, 0, stream>>>(
-        static_cast<const uint4*>(W), nb1, reinterpret_cast<uint4*>(out->codes), c1, level, p, host_buckets());
+        static_cast<const uint4*>(W), nb1, reinterpret_cast<uint4*>(out->codes), c1, level, n_chunks,
+        host_buckets());
     QLORA_CHECK_LAUNCH();
     while (p > 1) {
         const int64_t np = (p + kTreeThreads - 1) / kTreeThreads;

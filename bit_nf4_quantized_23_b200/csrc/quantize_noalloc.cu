@@ -34,7 +34,7 @@ qlora_status launch_quantize(const void* W, int64_t N, int64_t K, const qlora_nf
 namespace {
 
 constexpr int64_t kNoAllocMaxWeights = int64_t(1) << 26;          // 67,108,864
-constexpr size_t kNoAllocScratchBytes = (size_t(1) << 22) + (size_t(1) << 18);   // 4.25 MiB
+constexpr size_t kNoAllocScratchBytes = (size_t(1) << 22) + (size_t(3) << 18);   // 4.75 MiB
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 

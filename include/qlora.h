@@ -146,7 +146,7 @@ qlora_status qlora_quantize_nf4_dq(const void* W, int64_t N, int64_t K,
  * pointers, or a latency-critical path that must not call cudaMalloc/cudaFree,
  * which may synchronize the device).  The pages have no counterpart: this is a
  * deployment variant of the same operation with the same bit-exact results.
- *   Scratch: a static array of 4.25 MiB in the library's device image, held by
+ *   Scratch: a static array of 4.75 MiB in the library's device image, held by
  *   every GPU that loads the library until the process exits.  Tensors of more
  *   than 67,108,864 weights (e.g. larger than W[8192,8192]) return
  *   QLORA_ERR_TOO_LARGE before anything is launched.

@@ -204,6 +204,19 @@ def test_ragged_linear(M, N, K, r):
     check_linear_full(W, X, A, B, dY, r, alpha=2.0 * r)
 
 
+# Small-M forward (M <= 16): the work is cut into equal ranges of (128-row tile, 64-wide
+# K-step) units, one per persistent CTA.  These shapes give one unit per CTA (every tile
+# summed from many partials), CTAs that cross several tile boundaries, a tile split over
+# ~300 CTAs, ragged N, the largest rank, and both output types.
+@pytest.mark.parametrize("M,N,K,r,y_f32", [(16, 1000, 640, 16, False), (7, 2600, 64, 8, True),
+                                           (16, 40000, 64, 16, False), (2, 300, 4096, 256, False),
+                                           (16, 9000, 1024, 16, True), (1, 128, 19200, 4, False)])
+def test_decode_stream_k_layouts(M, N, K, r, y_f32):
+    W, X, A, B, dY = si.custom_linear(N, K, M, r, seed=3 * M + N + K + r)
+    dt = torch.float32 if y_f32 else torch.bfloat16
+    check_linear_full(W, X, A, B, dY, r, alpha=2.0 * r, y_dtype=dt, dx_dtype=dt)
+
+
 def test_recompute_U_and_no_dX():
     W, X, A, B, dY = si.custom_linear(128, 256, 24, 8, seed=77)
     w = quantize_on_gpu(W)
