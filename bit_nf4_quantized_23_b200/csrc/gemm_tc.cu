@@ -391,7 +391,7 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
 //
 // Y[M,N] for M <= 16 tokens (decode), "swap-AB": D[n, m] = W_hat[n, :] X[m, :]^T
 // with the dequantized weight as the 128-row MMA operand A (K-major image
-// written by the producer warps) and the tokens as a 16-wide operand B.
+// written by the producer warps) and the token tile as a 16-wide operand B.
 // The work is the sequence of (tile of 128 W rows, K-step of 64) units, tile
 // major; it is cut into G equal contiguous ranges, one per persistent CTA
 // (stream-K), so every SM streams the same number of weight bytes whatever
@@ -399,39 +399,45 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
 // segment, accumulated in one of two TMEM accumulators and written as an fp32
 // partial tile to slot tile + CTA; decode_fixup then sums each tile's slots in
 // CTA order (deterministic) and adds the LoRA term s U B^T in fp32.
-// Warp roles (320 threads): warp 0 lane 0 streams the packed codes through a
-// TMA ring; warp 1 owns TMEM and issues tcgen05.mma; warps 2-9 are two
-// producer groups of 4 warps that take alternate units (one W row of 64
-// weights per thread per unit, plus the token tile), and each group runs the
-// epilogue of the segments that use its accumulator.
+// Warp roles (320 threads): warp 0 lane 0 streams each unit's packed codes and
+// token tile through a TMA ring (a ring slot is freed by the MMA that read it);
+// warp 1 owns TMEM and issues tcgen05.mma; warps 2-9 are two producer groups of
+// 4 warps that take alternate units (one W row of 64 weights per thread per
+// unit), and each group runs the epilogue of the segments that use its
+// accumulator.  The dequant is ALU-bound (byte-permute table lookups), so the
+// producers do nothing else per unit.
 constexpr int kDecThreads = 320;
-constexpr int kDecCtasPerSm = 2;                // ~105 KB of shared memory per CTA
+constexpr int kDecCtasPerSm = 2;                // ~103 KB of shared memory per CTA
 constexpr int kDecMaxCtas = 1024;
-constexpr int kDecCodeStages = 8;               // packed-code ring (the HBM stream); stage parity = group
-constexpr int kDecStages = 4;                   // dequantized-tile / token ring; stage parity = group
+constexpr int kDecCodeStages = 6;               // codes + token ring (the HBM stream); even: stage parity = group
+constexpr int kDecStages = 4;                   // dequantized-tile ring; stage parity = group
 constexpr int kDecPrefetch = 4;                 // block constants are loaded this many units (of the group) ahead
 constexpr uint32_t kDecAStage = 128 * 128;      // W_hat tile [128 rows x 64]
-constexpr uint32_t kDecBStage = 16 * 128;       // X tile [16 tokens x 64]
+constexpr uint32_t kDecXStage = 16 * 128;       // X tile [16 tokens x 64], 128-byte swizzled rows (TMA)
 constexpr uint32_t kDecCodesStage = 128 * 32;   // packed codes [128 rows x 32 bytes]
-constexpr uint32_t kDecOffB = kDecStages * kDecAStage;
-constexpr uint32_t kDecOffCodes = kDecOffB + kDecStages * kDecBStage;
-constexpr uint32_t kDecOffBars = kDecOffCodes + kDecCodeStages * kDecCodesStage;
+constexpr uint32_t kDecOffX = kDecStages * kDecAStage;
+constexpr uint32_t kDecOffCodes = kDecOffX + kDecCodeStages * kDecXStage;
+constexpr uint32_t kDecOffE4 = kDecOffCodes + kDecCodeStages * kDecCodesStage;   // E4M3 value table [256] fp32
+constexpr uint32_t kDecOffBars = kDecOffE4 + 256 * 4;
 // barriers: cfull[CS], cempty[CS], afull[S], aempty[S], accfull[2], accempty[2], drain
 constexpr uint32_t kDecNumBars = 2 * kDecCodeStages + 2 * kDecStages + 5;
 constexpr uint32_t kDecOffSlot = kDecOffBars + kDecNumBars * 8;
 constexpr uint32_t kDecOffAbort = kDecOffSlot + 4;
 constexpr uint32_t kDecAlloc = kDecOffAbort + 4 + 1024;
 constexpr uint32_t kDecSlotFloats = 16 * 128;   // one partial tile: [16 tokens][128 rows] fp32
+static_assert(kDecCodeStages % 2 == 0 && kDecStages % 2 == 0, "ring stages alternate between the two groups");
+static_assert(2 * (kDecAlloc + 1024) <= 233472, "two CTAs per SM");
 
 // First unit of CTA b when U units are cut into G ranges.
 __host__ __device__ __forceinline__ int64_t dec_range_begin(int64_t b, int64_t U, int64_t G) { return b * U / G; }
 
 __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm)
-tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, DecodeParams p) {
+tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, const __grid_constant__ CUtensorMap tmX, DecodeParams p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t base = (ptx::smem_addr(smem_raw) + 1023u) & ~1023u;
     uint8_t* gbase = smem_raw + (base - ptx::smem_addr(smem_raw));
-    const uint32_t sA = base, sB = base + kDecOffB, sCodes = base + kDecOffCodes;
+    const uint32_t sA = base, sX = base + kDecOffX, sCodes = base + kDecOffCodes;
+    float* e4tab = reinterpret_cast<float*>(gbase + kDecOffE4);
     const uint32_t bar_cfull = base + kDecOffBars;
     const uint32_t bar_cempty = bar_cfull + 8 * kDecCodeStages;
     const uint32_t bar_afull = bar_cempty + 8 * kDecCodeStages;
@@ -449,10 +455,11 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, DecodeParams p) {
     const int64_t t0 = u0 / S;                                // tile of the first segment
     const int step0 = (int)(u0 - t0 * S);
 
+    if (threadIdx.x < 256) e4tab[threadIdx.x] = e4m3_to_f32(threadIdx.x);
     if (threadIdx.x == 0) {
         for (int s = 0; s < kDecCodeStages; ++s) {
             ptx::mbar_init(bar_cfull + 8 * s, 1);
-            ptx::mbar_init(bar_cempty + 8 * s, 4);
+            ptx::mbar_init(bar_cempty + 8 * s, 1);
         }
         for (int s = 0; s < kDecStages; ++s) {
             ptx::mbar_init(bar_afull + 8 * s, 4);
@@ -467,6 +474,7 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, DecodeParams p) {
         ptx::fence_barrier_init();
         ptx::fence_proxy_async_smem();
         ptx::tma_prefetch_map(&tmCodes);
+        ptx::tma_prefetch_map(&tmX);
     }
     if (warp == 1) {
         ptx::tmem_alloc(base + kDecOffSlot, 32);
@@ -479,7 +487,8 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, DecodeParams p) {
 
     if (warp == 0) {
         if (lane == 0) {
-            // codes of unit i go to stage i % kDecCodeStages; cempty is observed phase by phase
+            // unit i: codes and token tile into ring slot i % kDecCodeStages, once the MMA
+            // that read the slot's previous contents has completed (cempty, phase by phase)
             bool ok = true;
             int issued = 0;
             int64_t tile = t0;
@@ -489,9 +498,10 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, DecodeParams p) {
                 const uint32_t cph = (uint32_t)(i / kDecCodeStages) & 1u;
                 ok = ptx::mbar_wait(bar_cempty + 8 * cs, cph ^ 1u, abort, p.err);
                 if (!ok) break;
-                ptx::mbar_arrive_expect_tx(bar_cfull + 8 * cs, kDecCodesStage);
+                ptx::mbar_arrive_expect_tx(bar_cfull + 8 * cs, kDecCodesStage + kDecXStage);
                 ptx::tma_load_2d(sCodes + cs * kDecCodesStage, &tmCodes, step * 32, (int32_t)(tile * 128),
                                  bar_cfull + 8 * cs);
+                ptx::tma_load_2d(sX + cs * kDecXStage, &tmX, step * 64, 0, bar_cfull + 8 * cs);
                 issued = i + 1;
                 if (++step == S) { step = 0; ++tile; }
             }
@@ -511,20 +521,21 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, DecodeParams p) {
                 if (fresh && seg >= 2) {                      // accumulator a drained by segment seg-2's epilogue
                     ok = ptx::mbar_wait(bar_accempty + 8 * a, (uint32_t)((seg - 2) >> 1) & 1u, abort, p.err);
                     if (!ok) { atomicMax(p.dbg, 0x61000000u | (uint32_t)i); break; }
-                    ptx::tc_fence_after();
                 }
                 const int s = i % kDecStages;
-                const uint32_t ph = (uint32_t)(i / kDecStages) & 1u;
-                ok = ptx::mbar_wait(bar_afull + 8 * s, ph, abort, p.err);
+                const int cs = i % kDecCodeStages;
+                ok = ptx::mbar_wait(bar_afull + 8 * s, (uint32_t)(i / kDecStages) & 1u, abort, p.err) &&
+                     ptx::mbar_wait(bar_cfull + 8 * cs, (uint32_t)(i / kDecCodeStages) & 1u, abort, p.err);
                 if (!ok) { atomicMax(p.dbg, 0x60000000u | (uint32_t)i); break; }
                 ptx::tc_fence_after();
-                const uint32_t a_base = sA + s * kDecAStage, b_base = sB + s * kDecBStage;
+                const uint32_t a_base = sA + s * kDecAStage, b_base = sX + cs * kDecXStage;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     ptx::mma_bf16_ss(tmem + 16u * (uint32_t)a, ptx::smem_desc_sw128(a_base + kk * 32, 16, 1024),
                                      ptx::smem_desc_sw128(b_base + kk * 32, 16, 1024), idesc,
                                      (!fresh || kk != 0) ? 1u : 0u);
                 ptx::mma_commit(bar_aempty + 8 * s);
+                ptx::mma_commit(bar_cempty + 8 * cs);
                 fresh = false;
                 if (++step == S || i == n - 1) {              // segment ends: hand the accumulator over
                     ptx::mma_commit(bar_accfull + 8 * a);
@@ -537,54 +548,37 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, DecodeParams p) {
             if (*abort) ptx::mbar_wait_drain(bar_drain, 0);   // issued MMAs finish before TMEM is freed
         }
     } else {
-        // producer group g takes units g, g + 2, ...; thread t expands W row tile*128 + t of each
-        // and copies 16 bytes of its token tile (token t >> 3, 16-byte chunk t & 7)
+        // producer group g takes units g, g + 2, ...; thread t expands W row tile*128 + t
         const int g = (warp - 2) >> 2;
         const int t = threadIdx.x - 64 - 128 * g;
-        const int xm = t >> 3, xc = t & 7;
-        const bool x_ok = xm < p.M;
-        const uint4* xrow = static_cast<const uint4*>(p.X) + (int64_t)xm * (p.K / 8) + xc;
         const int64_t nb1 = p.N * (p.K / 64);
         const int64_t kb = p.K / 64;
         const float mu = *p.mu;
-        // unit cursors: (tile, step) of the current unit, of the next one (token tile) and of the
-        // prefetch head (block constants); each moves by 2 units
-        auto advance = [S](int64_t& tile, int& step, int by) {
-            step += by;
-            while (step >= S) { step -= S; ++tile; }
+        // a unit cursor: tile, step and the first-level block index of row tile*128 + t at step 0
+        struct Cursor { int64_t tile, rowblk; int step; };
+        auto advance = [&](Cursor& c, int by) {
+            c.step += by;
+            while (c.step >= S) { c.step -= S; ++c.tile; c.rowblk += 128 * kb; }
         };
-        int64_t cur_tile = t0; int cur_step = step0;
-        advance(cur_tile, cur_step, g);
-        auto x_load = [&](int64_t step) -> uint4 {
-            const int64_t col = step * 64 + xc * 8;
-            if (!(x_ok && col + 8 <= p.K)) {
-                if (x_ok) { atomicOr(p.err, ERR_FLAG_BOUNDS); atomicMax(p.dbg, 0x10000000u | (uint32_t)step); }
-                return make_uint4(0, 0, 0, 0);
-            }
-            return __ldg(xrow + step * 8);
-        };
-        auto const_load = [&](int64_t tile, int step, uint32_t& code, float& c2) {
+        Cursor cur{t0, (t0 * 128 + t) * kb, step0};
+        advance(cur, g);
+        auto const_load = [&](const Cursor& c, uint32_t& code, float& c2) {
             code = 0; c2 = 0.f;
-            const int64_t row = tile * 128 + t;
-            if (row >= p.N) return;
-            const int64_t blk = row * kb + step;
-            if (blk >= nb1 || step >= kb) { atomicOr(p.err, ERR_FLAG_BOUNDS); atomicMax(p.dbg, 0x20000000u); return; }
+            if (c.tile * 128 + t >= p.N) return;
+            const int64_t blk = c.rowblk + c.step;
+            if (blk >= nb1) { atomicOr(p.err, ERR_FLAG_BOUNDS); atomicMax(p.dbg, 0x20000000u); return; }
             code = __ldg(p.c1_codes + blk);
             c2 = __ldg(p.c2 + (blk >> 8));
         };
-        uint4 xnext = make_uint4(0, 0, 0, 0);
-        if (g < n) xnext = x_load(cur_step);
         uint32_t qcode[kDecPrefetch];
         float qc2[kDecPrefetch];
-        int64_t pf_tile = cur_tile; int pf_step = cur_step;
+        Cursor pf = cur;
 #pragma unroll
         for (int d = 0; d < kDecPrefetch; ++d) {
             qcode[d] = 0; qc2[d] = 0.f;
-            if (g + 2 * d < n) const_load(pf_tile, pf_step, qcode[d], qc2[d]);
-            advance(pf_tile, pf_step, 2);
+            if (g + 2 * d < n) const_load(pf, qcode[d], qc2[d]);
+            advance(pf, 2);
         }
-        int64_t nx_tile = cur_tile; int nx_step = cur_step;
-        advance(nx_tile, nx_step, 2);
 
         int epi_seg = g;                                      // next segment whose epilogue is ours
         const int last_seg = (int)((u0 + n - 1) / S - t0);
@@ -610,51 +604,41 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, DecodeParams p) {
 
         bool ok = true;
         for (int i = g; i < n && ok; i += 2) {
-            const int seg = (int)(cur_tile - t0);
+            const int seg = (int)(cur.tile - t0);
             while (epi_seg < seg && ok) { ok = epilogue(epi_seg); epi_seg += 2; }
             if (!ok) break;
             const int cs = i % kDecCodeStages;
-            const uint32_t cph = (uint32_t)(i / kDecCodeStages) & 1u;
             const int s = i % kDecStages;
-            const uint32_t ph = (uint32_t)(i / kDecStages) & 1u;
-            const float c1p = rebuild_c1(qcode[0], qc2[0], mu);
-            const uint4 xcur = xnext;
-            if (i + 2 < n) xnext = x_load(nx_step);
+            const float c1p = __fadd_rn(__fmul_rn(e4tab[qcode[0]], qc2[0]), mu);   // c1' = fp32(fp32(v8 c2) + mu)
 #pragma unroll
             for (int d = 0; d + 1 < kDecPrefetch; ++d) {
                 qcode[d] = qcode[d + 1];
                 qc2[d] = qc2[d + 1];
             }
             qcode[kDecPrefetch - 1] = 0; qc2[kDecPrefetch - 1] = 0.f;
-            if (i + 2 * kDecPrefetch < n) const_load(pf_tile, pf_step, qcode[kDecPrefetch - 1], qc2[kDecPrefetch - 1]);
-            bool w_ok = ptx::mbar_wait(bar_cfull + 8 * cs, cph, abort, p.err);
+            if (i + 2 * kDecPrefetch < n) const_load(pf, qcode[kDecPrefetch - 1], qc2[kDecPrefetch - 1]);
+            bool w_ok = ptx::mbar_wait(bar_cfull + 8 * cs, (uint32_t)(i / kDecCodeStages) & 1u, abort, p.err);
             if (!w_ok) atomicMax(p.dbg, 0x40000000u | (uint32_t)i);
-            w_ok = w_ok && ptx::mbar_wait(bar_aempty + 8 * s, ph ^ 1u, abort, p.err);
+            w_ok = w_ok && ptx::mbar_wait(bar_aempty + 8 * s, ((uint32_t)(i / kDecStages) & 1u) ^ 1u, abort, p.err);
             if (!w_ok) atomicMax(p.dbg, 0x50000000u | (uint32_t)i);
             ok = __all_sync(0xffffffffu, w_ok);
             if (!ok) break;
-            st_shared_v4(sB + s * kDecBStage + (uint32_t)xm * 128u + ((uint32_t)(xc ^ (xm & 7)) << 4), xcur);
             const uint32_t row_addr = sA + s * kDecAStage + (uint32_t)t * 128u;
-            if (cur_tile * 128 + t >= p.N) {
+            if (cur.tile * 128 + t >= p.N) {
                 zero_row(row_addr);
             } else {
                 const uint32_t src = sCodes + cs * kDecCodesStage + (uint32_t)t * 32u;
-                const uint32_t first = ((uint32_t)t >> 2) & 1u;
-                const uint4 x = ld_shared_v4(src + first * 16u);
-                const uint4 y = ld_shared_v4(src + (first ^ 1u) * 16u);
+                const uint4 x = ld_shared_v4(src);
+                const uint4 y = ld_shared_v4(src + 16u);
                 Lut lut;
                 build_lut(lut, c1p, p.tb);
-                expand_block_row(row_addr, (uint32_t)t & 7u, first ? y : x, first ? x : y, lut);
+                expand_block_row(row_addr, (uint32_t)t & 7u, x, y, lut);
             }
             ptx::fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) {
-                ptx::mbar_arrive(bar_cempty + 8 * cs);
-                ptx::mbar_arrive(bar_afull + 8 * s);
-            }
-            advance(cur_tile, cur_step, 2);
-            advance(nx_tile, nx_step, 2);
-            advance(pf_tile, pf_step, 2);
+            if (lane == 0) ptx::mbar_arrive(bar_afull + 8 * s);
+            advance(cur, 2);
+            advance(pf, 2);
         }
         while (ok && epi_seg <= last_seg) { ok = epilogue(epi_seg); epi_seg += 2; }
     }
@@ -841,10 +825,11 @@ qlora_status launch_tc_decode(const DecodeArgs& a, cudaStream_t stream) {
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return QLORA_ERR_CUDA;
     }
-    CUtensorMap tmCodes;
+    CUtensorMap tmCodes, tmX;
     if (!make_tmap_2d(&tmCodes, false, w->codes, K / 2, N, K / 2, 32, 128, false)) return QLORA_ERR_CUDA;
+    if (!make_tmap_2d(&tmX, true, a.X, K, a.M, K * 2, 64, 16, true)) return QLORA_ERR_CUDA;
     DecodeParams p{};
-    p.M = a.M; p.N = N; p.K = K; p.X = a.X;
+    p.M = a.M; p.N = N; p.K = K;
     p.ksteps = (int32_t)(K / 64);
     const int64_t tiles = (N + 127) / 128;
     p.units = tiles * p.ksteps;
@@ -865,7 +850,7 @@ qlora_status launch_tc_decode(const DecodeArgs& a, cudaStream_t stream) {
     decode_lora_u<<<dim3((unsigned)a.r, (unsigned)a.M), 256, 0, stream>>>(
         static_cast<const uint4*>(a.X), static_cast<const uint4*>(a.A), K / 8, a.r, a.U);
     QLORA_CHECK_LAUNCH();
-    tc_decode_nf4<<<(unsigned)p.grid, kDecThreads, kDecAlloc, stream>>>(tmCodes, p);
+    tc_decode_nf4<<<(unsigned)p.grid, kDecThreads, kDecAlloc, stream>>>(tmCodes, tmX, p);
     QLORA_CHECK_LAUNCH();
     decode_fixup<<<(unsigned)tiles, 128, (size_t)a.r * 16 * sizeof(float), stream>>>(
         a.partial, p.units, p.grid, p.ksteps, a.M, N, a.U, static_cast<const uint16_t*>(a.B), a.r, a.scale, a.out,

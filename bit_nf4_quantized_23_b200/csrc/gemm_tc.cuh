@@ -40,7 +40,6 @@ qlora_status launch_tc_gemm_nf4(TcGemmArgs& a, bool dx, cudaStream_t stream);
 // (tile, K-step) units with fp32 partial tiles and a fixup that adds the LoRA term.
 struct DecodeParams {
     int64_t M, N, K;
-    const void* X;          // [M, K] bf16 (read by the producer warps)
     int32_t ksteps;         // K / 64: units per tile of 128 W rows
     int64_t units;          // tiles * ksteps
     int64_t grid;           // persistent CTAs; CTA b takes units [b*units/grid, (b+1)*units/grid)
