@@ -83,14 +83,15 @@ tc_lora_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        if (lane == 0) {
-            const uint32_t b_bytes = MN ? (uint32_t)R * 256u : (uint32_t)R * 128u;
-            int issued = 0;
-            for (int i = 0; i < nk; ++i) {
-                const int s = i % kStages;
-                const uint32_t ph = (uint32_t)(i / kStages) & 1u;
-                if (!ptx::mbar_wait(bar_empty + 8 * s, ph ^ 1u, abort, p.err)) break;
-                issued = i + 1;
+        // TMA issuer: the whole warp runs the loop, one elected lane issues the copies
+        const uint32_t b_bytes = MN ? (uint32_t)R * 256u : (uint32_t)R * 128u;
+        int issued = 0;
+        for (int i = 0; i < nk; ++i) {
+            const int s = i % kStages;
+            const uint32_t ph = (uint32_t)(i / kStages) & 1u;
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_empty + 8 * s, ph ^ 1u, abort, p.err))) break;
+            issued = i + 1;
+            if (ptx::elect_one_sync()) {
                 const uint32_t fb = bar_full + 8 * s;
                 const int ks = k_begin + i;
                 const uint32_t a_dst = sA + s * kAStage, b_dst = sB + s * kBStage;
@@ -108,21 +109,23 @@ tc_lora_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                     }
                 }
             }
-            if (*abort) {   // drain this CTA's copies in flight before it exits
-                for (int i = max(0, issued - kStages); i < issued; ++i)
-                    ptx::mbar_wait_drain(bar_full + 8 * (i % kStages), (uint32_t)(i / kStages) & 1u);
-            }
+            __syncwarp();
+        }
+        if (*abort) {   // drain this CTA's copies in flight before it exits
+            for (int i = max(0, issued - kStages); i < issued; ++i)
+                ptx::mbar_wait_drain(bar_full + 8 * (i % kStages), (uint32_t)(i / kStages) & 1u);
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            const uint32_t idesc = ptx::idesc_bf16_f32_ab(128, R, MN ? 1 : 0, MN ? 1 : 0);
-            bool ok = true;
-            for (int i = 0; i < nk && ok; ++i) {
-                const int s = i % kStages;
-                const uint32_t ph = (uint32_t)(i / kStages) & 1u;
-                ok = ptx::mbar_wait(bar_full + 8 * s, ph, abort, p.err);
-                if (!ok) break;
-                ptx::tc_fence_after();
+        // MMA issuer: the whole warp runs the loop, one elected lane issues the MMAs and commits
+        const uint32_t idesc = ptx::idesc_bf16_f32_ab(128, R, MN ? 1 : 0, MN ? 1 : 0);
+        bool ok = true;
+        for (int i = 0; i < nk && ok; ++i) {
+            const int s = i % kStages;
+            const uint32_t ph = (uint32_t)(i / kStages) & 1u;
+            ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_full + 8 * s, ph, abort, p.err));
+            if (!ok) break;
+            ptx::tc_fence_after();
+            if (ptx::elect_one_sync()) {
                 const uint32_t a_base = sA + s * kAStage, b_base = sB + s * kBStage;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
@@ -132,7 +135,8 @@ tc_lora_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                                          ptx::smem_desc_sw128(b_base + kk * 32, 16, 1024), idesc, acc);
                     } else {
                         const uint64_t ad = ptx::smem_desc_sw128(a_base + kk * 2048, 8192, 1024);
-                        ptx::mma_bf16_ss(tmem, ad, ptx::smem_desc_sw128(b_base + kk * 2048, 8192, 1024), idesc, acc);
+                        ptx::mma_bf16_ss(tmem, ad, ptx::smem_desc_sw128(b_base + kk * 2048, 8192, 1024), idesc,
+                                         acc);
                         ptx::mma_bf16_ss(tmem, ad,
                                          ptx::smem_desc_sw128(b_base + (R / 64) * 8192 + kk * 2048, 8192, 1024),
                                          idesc, 1u);
@@ -140,9 +144,13 @@ tc_lora_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                 }
                 ptx::mma_commit(bar_empty + 8 * s);
             }
+            __syncwarp();
+        }
+        if (ptx::elect_one_sync()) {
             ptx::mma_commit(bar_acc);
             if (*abort) ptx::mbar_wait_drain(bar_acc, 0);   // issued MMAs finish before TMEM is freed
         }
+        __syncwarp();
     } else {
         const bool acc_ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_acc, 0, abort, p.err));
         ptx::tc_fence_after();

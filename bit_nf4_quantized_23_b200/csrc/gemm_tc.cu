@@ -184,13 +184,14 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            int issued = 0;
-            for (int it = 0; it < ktotal; ++it) {
-                const int s = it % kStages;
-                const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-                if (!ptx::mbar_wait(bar_empty + 8 * s, ph ^ 1u, abort, p.err)) break;
-                issued = it + 1;
+        // (the whole warp runs the loop; one elected lane issues the copies)
+        int issued = 0;
+        int s = 0;
+        uint32_t ph = 0;
+        for (int it = 0; it < ktotal; ++it) {
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_empty + 8 * s, ph ^ 1u, abort, p.err))) break;
+            issued = it + 1;
+            if (ptx::elect_one_sync()) {
                 const uint32_t fa = bar_full_a + 8 * s;
                 const uint32_t a_dst = sA + s * L::kAStageBytes;
                 const uint32_t b_dst = sB + s * kBStageBytes;
@@ -212,40 +213,51 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
                     }
                 }
             }
-            if (*abort) {   // drain this CTA's copies in flight before it exits
-                for (int it = max(0, issued - kStages); it < issued; ++it)
-                    ptx::mbar_wait_drain(bar_full_a + 8 * (it % kStages), (uint32_t)(it / kStages) & 1u);
-            }
+            __syncwarp();
+            if (++s == kStages) { s = 0; ph ^= 1u; }
+        }
+        if (*abort) {   // drain this CTA's copies in flight before it exits
+            for (int it = max(0, issued - kStages); it < issued; ++it)
+                ptx::mbar_wait_drain(bar_full_a + 8 * (it % kStages), (uint32_t)(it / kStages) & 1u);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc = ptx::idesc_bf16_f32(128, kBN, DX ? 1 : 0);
-            bool ok = true;
-            for (int it = 0; it < ktotal && ok; ++it) {
-                const int s = it % kStages;
-                const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-                ok = ptx::mbar_wait(bar_full_a + 8 * s, ph, abort, p.err);
-                if (ok && it < ks0) ok = ptx::mbar_wait(bar_full_b + 8 * s, ph, abort, p.err);
-                if (!ok) break;
-                ptx::tc_fence_after();
-                const uint32_t a_base = sA + s * L::kAStageBytes;
-                const uint32_t b_base = sB + s * kBStageBytes;
+        // (the whole warp runs the loop; one elected lane issues the MMAs and their commits;
+        // descriptors are built once and advanced by stage offsets: start address >> 4 in
+        // the low 14 bits, every shared address is below 256 KiB, so no carry leaves them)
+        constexpr uint32_t idesc = ptx::idesc_bf16_f32(128, kBN, DX ? 1 : 0);
+        const uint64_t adesc0 = ptx::smem_desc_sw128(sA, 16, 1024);
+        const uint64_t bdesc0 = DX ? ptx::smem_desc_sw128(sB, 8192, 1024) : ptx::smem_desc_sw128(sB, 16, 1024);
+        bool ok = true;
+        int s = 0;
+        uint32_t ph = 0;
+        for (int it = 0; it < ktotal && ok; ++it) {
+            bool w = ptx::mbar_wait(bar_full_a + 8 * s, ph, abort, p.err);
+            if (w && it < ks0) w = ptx::mbar_wait(bar_full_b + 8 * s, ph, abort, p.err);
+            ok = __all_sync(0xffffffffu, w);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            if (ptx::elect_one_sync()) {
+                const uint64_t ad = adesc0 + ((uint32_t)s * (L::kAStageBytes >> 4));
+                const uint64_t bd = bdesc0 + ((uint32_t)s * (kBStageBytes >> 4));
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t bdesc = DX ? ptx::smem_desc_sw128(b_base + kk * 2048, 8192, 1024)
-                                              : ptx::smem_desc_sw128(b_base + kk * 32, 16, 1024);
+                    const uint64_t bdesc = bd + (DX ? kk * (2048 >> 4) : kk * (32 >> 4));
 #pragma unroll
-                    for (int h = 0; h < NUM_ACC; ++h) {
-                        const uint64_t adesc = ptx::smem_desc_sw128(a_base + h * 16384 + kk * 32, 16, 1024);
-                        ptx::mma_bf16_ss(tmem + h * 256, adesc, bdesc, idesc, (it | kk) != 0 ? 1u : 0u);
-                    }
+                    for (int h = 0; h < NUM_ACC; ++h)
+                        ptx::mma_bf16_ss(tmem + h * 256, ad + h * (16384 >> 4) + kk * (32 >> 4), bdesc, idesc,
+                                         (it | kk) != 0 ? 1u : 0u);
                 }
                 ptx::mma_commit(bar_empty + 8 * s);
             }
+            __syncwarp();
+            if (++s == kStages) { s = 0; ph ^= 1u; }
+        }
+        if (ptx::elect_one_sync()) {
             ptx::mma_commit(bar_acc);   // arrives when every issued MMA has completed
             if (*abort) ptx::mbar_wait_drain(bar_acc, 0);   // issued MMAs finish before TMEM is freed
         }
+        __syncwarp();
     } else {
         // ------------------------------------------------------------ dequant producers
         // Thread t (0..255) owns one unit per K-step: forward: B row t = W row n0 + t, K-block it;
@@ -486,67 +498,81 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, const __grid_constant
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        if (lane == 0) {
-            // unit i: codes and token tile into ring slot i % kDecCodeStages, once the MMA
-            // that read the slot's previous contents has completed (cempty, phase by phase)
-            bool ok = true;
-            int issued = 0;
-            int64_t tile = t0;
-            int step = step0;
-            for (int i = 0; i < n && ok; ++i) {
-                const int cs = i % kDecCodeStages;
-                const uint32_t cph = (uint32_t)(i / kDecCodeStages) & 1u;
-                ok = ptx::mbar_wait(bar_cempty + 8 * cs, cph ^ 1u, abort, p.err);
-                if (!ok) break;
+        // unit i: codes and token tile into ring slot i % kDecCodeStages, once the MMA that
+        // read the slot's previous contents has completed (cempty, phase by phase); the whole
+        // warp runs the loop and one elected lane issues the copies
+        bool ok = true;
+        int issued = 0;
+        int64_t tile = t0;
+        int step = step0;
+        int cs = 0;
+        uint32_t cph = 0;
+        for (int i = 0; i < n && ok; ++i) {
+            ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_cempty + 8 * cs, cph ^ 1u, abort, p.err));
+            if (!ok) break;
+            if (ptx::elect_one_sync()) {
                 ptx::mbar_arrive_expect_tx(bar_cfull + 8 * cs, kDecCodesStage + kDecXStage);
                 ptx::tma_load_2d(sCodes + cs * kDecCodesStage, &tmCodes, step * 32, (int32_t)(tile * 128),
                                  bar_cfull + 8 * cs);
                 ptx::tma_load_2d(sX + cs * kDecXStage, &tmX, step * 64, 0, bar_cfull + 8 * cs);
-                issued = i + 1;
-                if (++step == S) { step = 0; ++tile; }
             }
-            if (*abort) {   // drain this CTA's copies in flight before it exits
-                for (int c = max(0, issued - kDecCodeStages); c < issued; ++c)
-                    ptx::mbar_wait_drain(bar_cfull + 8 * (c % kDecCodeStages), (uint32_t)(c / kDecCodeStages) & 1u);
-            }
+            __syncwarp();
+            issued = i + 1;
+            if (++step == S) { step = 0; ++tile; }
+            if (++cs == kDecCodeStages) { cs = 0; cph ^= 1u; }
+        }
+        if (*abort) {   // drain this CTA's copies in flight before it exits
+            for (int c = max(0, issued - kDecCodeStages); c < issued; ++c)
+                ptx::mbar_wait_drain(bar_cfull + 8 * (c % kDecCodeStages), (uint32_t)(c / kDecCodeStages) & 1u);
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            constexpr uint32_t idesc = ptx::idesc_bf16_f32_ab(128, 16, 0, 0);
-            bool ok = true;
-            int step = step0, seg = 0;
-            bool fresh = true;                                // first unit of a segment: overwrite
-            for (int i = 0; i < n && ok; ++i) {
-                const int a = seg & 1;
-                if (fresh && seg >= 2) {                      // accumulator a drained by segment seg-2's epilogue
-                    ok = ptx::mbar_wait(bar_accempty + 8 * a, (uint32_t)((seg - 2) >> 1) & 1u, abort, p.err);
-                    if (!ok) { atomicMax(p.dbg, 0x61000000u | (uint32_t)i); break; }
-                }
-                const int s = i % kDecStages;
-                const int cs = i % kDecCodeStages;
-                ok = ptx::mbar_wait(bar_afull + 8 * s, (uint32_t)(i / kDecStages) & 1u, abort, p.err) &&
-                     ptx::mbar_wait(bar_cfull + 8 * cs, (uint32_t)(i / kDecCodeStages) & 1u, abort, p.err);
-                if (!ok) { atomicMax(p.dbg, 0x60000000u | (uint32_t)i); break; }
-                ptx::tc_fence_after();
-                const uint32_t a_base = sA + s * kDecAStage, b_base = sX + cs * kDecXStage;
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    ptx::mma_bf16_ss(tmem + 16u * (uint32_t)a, ptx::smem_desc_sw128(a_base + kk * 32, 16, 1024),
-                                     ptx::smem_desc_sw128(b_base + kk * 32, 16, 1024), idesc,
-                                     (!fresh || kk != 0) ? 1u : 0u);
+        // MMA issuer: the whole warp runs the loop, one elected lane issues.  Descriptors are
+        // built once and advanced by stage offsets (start address >> 4 in the low 14 bits;
+        // every shared address here is below 256 KiB, so no carry leaves them).
+        constexpr uint32_t idesc = ptx::idesc_bf16_f32_ab(128, 16, 0, 0);
+        const uint64_t adesc0 = ptx::smem_desc_sw128(sA, 16, 1024);
+        const uint64_t bdesc0 = ptx::smem_desc_sw128(sX, 16, 1024);
+        bool ok = true;
+        int step = step0, seg = 0;
+        int s = 0, cs = 0;                                    // ring slots of unit i, and their phase bits
+        uint32_t ph = 0, cph = 0;
+        bool fresh = true;                                    // first unit of a segment: overwrite
+        for (int i = 0; i < n && ok; ++i) {
+            const int a = seg & 1;
+            if (fresh && seg >= 2) {                          // accumulator a drained by segment seg-2's epilogue
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_accempty + 8 * a, (uint32_t)((seg - 2) >> 1) & 1u,
+                                                             abort, p.err));
+                if (!ok) { if (lane == 0) atomicMax(p.dbg, 0x61000000u | (uint32_t)i); break; }
+            }
+            ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_afull + 8 * s, ph, abort, p.err) &&
+                                             ptx::mbar_wait(bar_cfull + 8 * cs, cph, abort, p.err));
+            if (!ok) { if (lane == 0) atomicMax(p.dbg, 0x60000000u | (uint32_t)i); break; }
+            ptx::tc_fence_after();
+            const bool last = (step + 1 == S) || (i == n - 1);
+            if (ptx::elect_one_sync()) {
+                const uint64_t ad = adesc0 + ((uint32_t)s * (kDecAStage >> 4));
+                const uint64_t bd = bdesc0 + ((uint32_t)cs * (kDecXStage >> 4));
+                const uint32_t d = tmem + 16u * (uint32_t)a;
+                ptx::mma_bf16_ss(d, ad, bd, idesc, fresh ? 0u : 1u);
+                ptx::mma_bf16_ss(d, ad + 2, bd + 2, idesc, 1u);
+                ptx::mma_bf16_ss(d, ad + 4, bd + 4, idesc, 1u);
+                ptx::mma_bf16_ss(d, ad + 6, bd + 6, idesc, 1u);
                 ptx::mma_commit(bar_aempty + 8 * s);
                 ptx::mma_commit(bar_cempty + 8 * cs);
-                fresh = false;
-                if (++step == S || i == n - 1) {              // segment ends: hand the accumulator over
-                    ptx::mma_commit(bar_accfull + 8 * a);
-                    step = step == S ? 0 : step;
-                    ++seg;
-                    fresh = true;
-                }
+                if (last) ptx::mma_commit(bar_accfull + 8 * a);   // segment ends: hand the accumulator over
             }
+            __syncwarp();
+            if (++s == kDecStages) { s = 0; ph ^= 1u; }
+            if (++cs == kDecCodeStages) { cs = 0; cph ^= 1u; }
+            fresh = last;
+            if (++step == S) step = 0;
+            if (last) ++seg;
+        }
+        if (ptx::elect_one_sync()) {
             ptx::mma_commit(bar_drain);
             if (*abort) ptx::mbar_wait_drain(bar_drain, 0);   // issued MMAs finish before TMEM is freed
         }
+        __syncwarp();
     } else {
         // producer group g takes units g, g + 2, ...; thread t expands W row tile*128 + t
         const int g = (warp - 2) >> 2;
@@ -603,12 +629,12 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, const __grid_constant
         };
 
         bool ok = true;
+        int cs = g, s = g;                                    // ring slots of unit i (parity g), phase bits
+        uint32_t cph = 0, ph = 0;
         for (int i = g; i < n && ok; i += 2) {
             const int seg = (int)(cur.tile - t0);
             while (epi_seg < seg && ok) { ok = epilogue(epi_seg); epi_seg += 2; }
             if (!ok) break;
-            const int cs = i % kDecCodeStages;
-            const int s = i % kDecStages;
             const float c1p = __fadd_rn(__fmul_rn(e4tab[qcode[0]], qc2[0]), mu);   // c1' = fp32(fp32(v8 c2) + mu)
 #pragma unroll
             for (int d = 0; d + 1 < kDecPrefetch; ++d) {
@@ -617,9 +643,9 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, const __grid_constant
             }
             qcode[kDecPrefetch - 1] = 0; qc2[kDecPrefetch - 1] = 0.f;
             if (i + 2 * kDecPrefetch < n) const_load(pf, qcode[kDecPrefetch - 1], qc2[kDecPrefetch - 1]);
-            bool w_ok = ptx::mbar_wait(bar_cfull + 8 * cs, (uint32_t)(i / kDecCodeStages) & 1u, abort, p.err);
+            bool w_ok = ptx::mbar_wait(bar_cfull + 8 * cs, cph, abort, p.err);
             if (!w_ok) atomicMax(p.dbg, 0x40000000u | (uint32_t)i);
-            w_ok = w_ok && ptx::mbar_wait(bar_aempty + 8 * s, ((uint32_t)(i / kDecStages) & 1u) ^ 1u, abort, p.err);
+            w_ok = w_ok && ptx::mbar_wait(bar_aempty + 8 * s, ph ^ 1u, abort, p.err);
             if (!w_ok) atomicMax(p.dbg, 0x50000000u | (uint32_t)i);
             ok = __all_sync(0xffffffffu, w_ok);
             if (!ok) break;
@@ -639,6 +665,8 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, const __grid_constant
             if (lane == 0) ptx::mbar_arrive(bar_afull + 8 * s);
             advance(cur, 2);
             advance(pf, 2);
+            if ((cs += 2) >= kDecCodeStages) { cs -= kDecCodeStages; cph ^= 1u; }
+            if ((s += 2) >= kDecStages) { s -= kDecStages; ph ^= 1u; }
         }
         while (ok && epi_seg <= last_seg) { ok = epilogue(epi_seg); epi_seg += 2; }
     }

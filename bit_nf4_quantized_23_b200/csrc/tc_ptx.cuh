@@ -45,32 +45,50 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
-// One try_wait with a suspend-time hint: a thread whose phase is not complete
-// sleeps (up to kSuspendNs) until it completes instead of spinning, so waiting
-// warps leave the issue slots to the working ones.
+// One try_wait.  With a suspend-time hint (SLEEP) a thread whose phase is not
+// complete may sleep (up to kSuspendNs) instead of spinning, which leaves the
+// issue slots to the working warps.  Measured on the decode and fused GEMM
+// kernels, polling without the hint was no faster for the issuer warps.
 constexpr uint32_t kSuspendNs = 100000;
 
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+template <bool SLEEP>
+__device__ __forceinline__ bool mbar_try_wait_t(uint32_t bar, uint32_t parity) {
     uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity), "n"(kSuspendNs)
-        : "memory");
+    if constexpr (SLEEP) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity), "n"(kSuspendNs)
+            : "memory");
+    } else {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity)
+            : "memory");
+    }
     return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    return mbar_try_wait_t<true>(bar, parity);
 }
 
 // Wait until the phase with the given parity has completed.  Gives up after
 // `limit_ns` of wall time or when another thread of the CTA has already given
-// up (*abort != 0); then raises the TIMEOUT flag and returns false.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort, uint32_t* err,
-                                          uint64_t limit_ns = 2000000000ull) {
-    if (mbar_try_wait(bar, parity)) return true;
+// up (*abort != 0); then raises the TIMEOUT flag and returns false.  The
+// bounded polling loop is out of line so the common case (phase already
+// complete, or completed within one suspended try_wait) stays one instruction.
+template <bool SLEEP>
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort, uint32_t* err,
+                                                   uint64_t limit_ns) {
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_t<SLEEP>(bar, parity)) return true;
         if ((i & 15u) == 0u) {
             if (*abort) return false;
             if (globaltimer_ns() - t0 > limit_ns) {
@@ -82,6 +100,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     }
 }
 
+template <bool SLEEP = true>
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort, uint32_t* err,
+                                          uint64_t limit_ns = 2000000000ull) {
+    if (mbar_try_wait_t<SLEEP>(bar, parity)) return true;
+    return mbar_wait_slow<SLEEP>(bar, parity, abort, err, limit_ns);
+}
+
 // Wait for a phase regardless of the abort flag (used to drain this CTA's own
 // copies in flight before it exits after an abort); bounded by `limit_ns`.
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns = 200000000ull) {
@@ -91,6 +116,21 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, u
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 15u) == 0u && globaltimer_ns() - t0 > limit_ns) return false;
     }
+}
+
+// One lane of the (fully active) warp is elected; it returns true there.  Issue
+// loops run on the whole warp so their state stays warp-uniform (uniform
+// registers, no per-issue register-to-uniform moves) and only the elected
+// lane issues the TMA / tcgen05 instruction.  With every lane active the
+// elected lane is the same each time, so its commits cover its own MMAs.
+__device__ __forceinline__ bool elect_one_sync() {
+    uint32_t pred = 0;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t.reg .b32 R;\n\t"
+        "elect.sync R|P, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, P;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
 }
 
 // ---------------------------------------------------------------- TMA
