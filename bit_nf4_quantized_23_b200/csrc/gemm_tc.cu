@@ -467,6 +467,7 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, const __grid_constant
     const int64_t t0 = u0 / S;                                // tile of the first segment
     const int step0 = (int)(u0 - t0 * S);
 
+    allow_dependents();                                       // the fixup may be scheduled now
     if (threadIdx.x < 256) e4tab[threadIdx.x] = e4m3_to_f32(threadIdx.x);
     if (threadIdx.x == 0) {
         for (int s = 0; s < kDecCodeStages; ++s) {
@@ -677,11 +678,15 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, const __grid_constant
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, 32);
     }
+    // U (the previous kernel) is not read here, but the fixup that follows reads it: this
+    // grid completes only after U's grid has
+    if (threadIdx.x == 0) grid_dependency_wait();
 }
 
 // U[m, j] = sum_k X[m, k] A[j, k] in fp32 (one CTA per (j, m); fixed reduction order).
 __global__ void __launch_bounds__(256)
 decode_lora_u(const uint4* __restrict__ X, const uint4* __restrict__ A, int64_t K8, int r, float* __restrict__ U) {
+    allow_dependents();                                       // the dequant GEMM does not read U
     const int j = blockIdx.x, m = blockIdx.y;
     const uint4* xr = X + (int64_t)m * K8;
     const uint4* ar = A + (int64_t)j * K8;
@@ -724,6 +729,7 @@ __global__ void __launch_bounds__(128)
 decode_fixup(const float* __restrict__ partial, int64_t units, int64_t G, int S, int64_t M, int64_t N,
              const float* __restrict__ U, const uint16_t* __restrict__ B, int r, float scale, void* out, int out_f32) {
     extern __shared__ float us[];                             // us[j * 16 + m] = U[m, j]
+    grid_dependency_wait();                                   // partial tiles and U are complete
     for (int i = threadIdx.x; i < r * 16; i += 128) {
         const int j = i >> 4, m = i & 15;
         us[i] = m < M ? U[(int64_t)m * r + j] : 0.f;
@@ -878,11 +884,14 @@ qlora_status launch_tc_decode(const DecodeArgs& a, cudaStream_t stream) {
     decode_lora_u<<<dim3((unsigned)a.r, (unsigned)a.M), 256, 0, stream>>>(
         static_cast<const uint4*>(a.X), static_cast<const uint4*>(a.A), K / 8, a.r, a.U);
     QLORA_CHECK_LAUNCH();
-    tc_decode_nf4<<<(unsigned)p.grid, kDecThreads, kDecAlloc, stream>>>(tmCodes, tmX, p);
+    // the three kernels are chained with programmatic dependent launch (the dequant GEMM
+    // overlaps the U kernel and the launch gaps; see grid_dependency_wait in each)
+    (void)launch_dependent(tc_decode_nf4, dim3((unsigned)p.grid), dim3(kDecThreads), kDecAlloc, stream, tmCodes,
+                           tmX, p);
     QLORA_CHECK_LAUNCH();
-    decode_fixup<<<(unsigned)tiles, 128, (size_t)a.r * 16 * sizeof(float), stream>>>(
-        a.partial, p.units, p.grid, p.ksteps, a.M, N, a.U, static_cast<const uint16_t*>(a.B), a.r, a.scale, a.out,
-        a.out_f32);
+    (void)launch_dependent(decode_fixup, dim3((unsigned)tiles), dim3(128), (size_t)a.r * 16 * sizeof(float), stream,
+                           (const float*)a.partial, p.units, p.grid, (int)p.ksteps, a.M, N, (const float*)a.U,
+                           static_cast<const uint16_t*>(a.B), a.r, a.scale, a.out, (int)a.out_f32);
     QLORA_CHECK_LAUNCH();
     return QLORA_OK;
 }

@@ -9,6 +9,8 @@
 #include <cuda_fp8.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/qlora.h"
 
 namespace qlora {
@@ -109,6 +111,34 @@ __device__ __forceinline__ uint32_t dequant_bits(float q, float c1p) {
         }                                                      \
         if (qlora::sync_check_enabled() && !qlora::sync_check(__func__)) return QLORA_ERR_CUDA; \
     } while (0)
+
+// Programmatic dependent launch.  A kernel launched with launch_dependent()
+// may start while the previous kernel on the stream still runs; it calls
+// grid_dependency_wait() before it touches anything the previous kernel
+// writes (or, when it reads nothing of it, before it exits, so that its own
+// completion still implies the previous kernel's).  A kernel calls
+// allow_dependents() once the next kernel may be scheduled.  Both are no-ops
+// when the kernel was launched normally.
+namespace qlora {
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                             Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+}  // namespace qlora
 
 #define QLORA_TRY(expr)                                        \
     do {                                                       \
