@@ -31,27 +31,41 @@ namespace qlora {
 namespace {
 
 constexpr int kThreads = 192;
-constexpr int kStages = 2;
 constexpr uint32_t kAStage = 128 * 128;           // 128 rows x 64 bf16
-constexpr uint32_t kBStage = 64 * 1024;           // up to R=256 hi+lo MN-major images
-constexpr uint32_t kOffB = kStages * kAStage;
-constexpr uint32_t kOffBars = kOffB + kStages * kBStage;
-constexpr uint32_t kOffSlot = kOffBars + (2 * kStages + 1) * 8;
-constexpr uint32_t kOffAbort = kOffSlot + 4;
-constexpr uint32_t kSmemAlloc = kOffAbort + 4 + 1024;
+constexpr uint32_t kMaxSmem = 227 * 1024;
+
+// Shared-memory layout for a given B stage size and stage count: A stages, B stages, then
+// barriers full[S], empty[S], acc, the TMEM slot and the abort flag (1 KiB slack for alignment).
+struct LoraLayout {
+    uint32_t stages, b_stage, off_b, off_bars, off_slot, off_abort, alloc;
+};
+__host__ __device__ inline LoraLayout lora_layout(uint32_t stages, uint32_t b_stage) {
+    LoraLayout l;
+    l.stages = stages;
+    l.b_stage = b_stage;
+    l.off_b = stages * kAStage;
+    l.off_bars = l.off_b + stages * b_stage;
+    l.off_slot = l.off_bars + (2 * stages + 1) * 8;
+    l.off_abort = l.off_slot + 4;
+    l.alloc = l.off_abort + 4 + 1024;
+    return l;
+}
 
 template <bool MN>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 tc_lora_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, LoraGemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t base = (ptx::smem_addr(smem_raw) + 1023u) & ~1023u;
     uint8_t* gbase = smem_raw + (base - ptx::smem_addr(smem_raw));
-    const uint32_t sA = base, sB = base + kOffB;
-    const uint32_t bar_full = base + kOffBars;
+    const LoraLayout lay = lora_layout(p.stages, p.b_stage);
+    const int kStages = (int)lay.stages;
+    const uint32_t kBStage = lay.b_stage;
+    const uint32_t sA = base, sB = base + lay.off_b;
+    const uint32_t bar_full = base + lay.off_bars;
     const uint32_t bar_empty = bar_full + 8 * kStages;
     const uint32_t bar_acc = bar_empty + 8 * kStages;
-    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gbase + kOffSlot);
-    volatile int* abort = reinterpret_cast<volatile int*>(gbase + kOffAbort);
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gbase + lay.off_slot);
+    volatile int* abort = reinterpret_cast<volatile int*>(gbase + lay.off_abort);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int R = p.R;
@@ -74,7 +88,7 @@ tc_lora_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
         ptx::tma_prefetch_map(&tmB);
     }
     if (warp == 1) {
-        ptx::tmem_alloc(base + kOffSlot, tmem_cols);
+        ptx::tmem_alloc(base + lay.off_slot, tmem_cols);
         ptx::tmem_relinquish();
     }
     ptx::tc_fence_before();
@@ -186,12 +200,24 @@ qlora_status launch_lora(const CUtensorMap& tmA, const CUtensorMap& tmB, LoraGem
     static bool configured = false;
     auto kern = tc_lora_gemm<MN>;
     if (!configured) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemAlloc) != cudaSuccess)
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaxSmem) != cudaSuccess)
             return QLORA_ERR_CUDA;
         configured = true;
     }
+    // B stage: K-major R rows x 128 B, or the hi and lo MN-major images (2 x R/64 chunks of 8 KiB).
+    // Two CTAs per SM (one's epilogue overlaps the other's main loop) when three or more stages
+    // fit in half of the shared memory, else one CTA with up to six stages.
+    const uint32_t b_stage = MN ? (uint32_t)p.R * 256u : (uint32_t)p.R * 128u;
+    const uint32_t stage = kAStage + b_stage;
+    uint32_t stages = (kMaxSmem / 2 - 2048) / stage;
+    if (stages < 3) stages = (kMaxSmem - 2048) / stage;
+    if (stages > 6) stages = 6;
+    if (stages < 2) return QLORA_ERR_UNSUPPORTED;
+    p.stages = stages;
+    p.b_stage = b_stage;
+    const LoraLayout lay = lora_layout(stages, b_stage);
     const dim3 grid((unsigned)((p.rows + 127) / 128), (unsigned)splits);
-    kern<<<grid, kThreads, kSmemAlloc, stream>>>(tmA, tmB, p);
+    kern<<<grid, kThreads, lay.alloc, stream>>>(tmA, tmB, p);
     QLORA_CHECK_LAUNCH();
     return QLORA_OK;
 }

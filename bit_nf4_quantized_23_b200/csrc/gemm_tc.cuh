@@ -78,6 +78,7 @@ struct LoraGemmParams {
     int32_t ksteps_total;
     int32_t ksteps_per_split;
     uint32_t tmem_cols;
+    uint32_t stages, b_stage;   // pipeline depth and bytes of one B stage (set by the launcher)
     float* partial;
     uint32_t* err;
 };

@@ -41,6 +41,17 @@ __global__ void dup_cols(const uint16_t* __restrict__ B, int64_t N, int r, int R
     B2[n * 2 * R + R + j] = v;
 }
 
+// The same with 8 columns (16 bytes) per thread, for r % 8 == 0 (B rows are then 16-byte aligned).
+__global__ void dup_cols8(const uint4* __restrict__ B, int64_t N, int r8, int R8, uint4* __restrict__ B2) {
+    const int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    if (i >= N * R8) return;
+    const int64_t n = i / R8;
+    const int c = (int)(i - n * R8);
+    const uint4 v = c < r8 ? B[n * r8 + c] : make_uint4(0, 0, 0, 0);
+    B2[n * 2 * R8 + c] = v;
+    B2[n * 2 * R8 + R8 + c] = v;
+}
+
 // A2[j, k] = A2[R + j, k] = A[j, k]; zero rows for r <= j < R.  Moves 8 bf16 per thread.
 __global__ void dup_rows(const uint4* __restrict__ A, int r, int R, int64_t K8, uint4* __restrict__ A2) {
     const int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
@@ -52,20 +63,39 @@ __global__ void dup_rows(const uint4* __restrict__ A, int r, int R, int64_t K8, 
     A2[(R + j) * K8 + k] = v;
 }
 
-// Bt[j, n] = B[n, j] for j < r, zero rows for r <= j < R.
-__global__ void transpose_pad(const uint16_t* __restrict__ B, int64_t N, int r, int R, uint16_t* __restrict__ Bt) {
-    const int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-    if (i >= (int64_t)R * N) return;
-    const int64_t j = i / N;
-    const int64_t n = i - j * N;
-    Bt[i] = j < r ? B[n * r + j] : (uint16_t)0;
+// Bt[j, n] = B[n, j] for j < r, zero rows for r <= j < R.  A CTA moves a [64 n x 32 j] block
+// through shared memory so that reads (along j) and writes (along n) are both coalesced.
+__global__ void __launch_bounds__(256)
+transpose_pad(const uint16_t* __restrict__ B, int64_t N, int r, int R, uint16_t* __restrict__ Bt) {
+    __shared__ uint16_t tile[32][64 + 2];
+    const int64_t n0 = (int64_t)blockIdx.x * 64;
+    const int j0 = blockIdx.y * 32;
+    for (int e = threadIdx.x; e < 64 * 32; e += 256) {
+        const int nn = e >> 5, jj = e & 31;
+        const int64_t n = n0 + nn;
+        tile[jj][nn] = (n < N && j0 + jj < r) ? B[n * r + j0 + jj] : (uint16_t)0;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < 64 * 32; e += 256) {
+        const int jj = e >> 6, nn = e & 63;
+        const int64_t n = n0 + nn;
+        if (n < N && j0 + jj < R) Bt[(int64_t)(j0 + jj) * N + n] = tile[jj][nn];
+    }
 }
 
-// Sum of the split partials partial[s][row][j] (fixed order s = 0, 1, ...).
+// Sum of the split partials partial[s][row][j] in the fixed order s = 0, 1, ...; the loads of
+// four splits are issued together (the kernels are latency-bound, not bandwidth-bound).
 __device__ __forceinline__ float sum_splits(const float* __restrict__ partial, int splits, int64_t rows, int R,
                                             int64_t row, int j) {
+    const int64_t stride = rows * R;
+    const float* p = partial + row * R + j;
     float acc = 0.f;
-    for (int s = 0; s < splits; ++s) acc = __fadd_rn(acc, partial[((int64_t)s * rows + row) * R + j]);
+    int s = 0;
+    for (; s + 4 <= splits; s += 4) {
+        const float a = p[(s + 0) * stride], b = p[(s + 1) * stride], c = p[(s + 2) * stride], d = p[(s + 3) * stride];
+        acc = __fadd_rn(__fadd_rn(__fadd_rn(__fadd_rn(acc, a), b), c), d);
+    }
+    for (; s < splits; ++s) acc = __fadd_rn(acc, p[s * stride]);
     return acc;
 }
 
@@ -89,13 +119,25 @@ __global__ void reduce_rows(const float* __restrict__ partial, int splits, int64
 }
 
 // out[j, row] = S for j < r (the transposed [r, rows] result, e.g. dA from dA^T partials).
-__global__ void reduce_transposed(const float* __restrict__ partial, int splits, int64_t rows, int r, int R,
-                                  float* __restrict__ out) {
-    const int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-    if (i >= rows * (int64_t)r) return;
-    const int64_t j = i / rows;
-    const int64_t row = i - j * rows;
-    out[j * rows + row] = sum_splits(partial, splits, rows, R, row, (int)j);
+// A CTA sums a [32 rows x 64 j] block (reads along j, coalesced) into shared memory and writes
+// it transposed (writes along rows, coalesced).
+constexpr int kTrRows = 32;
+__global__ void __launch_bounds__(256)
+reduce_transposed(const float* __restrict__ partial, int splits, int64_t rows, int r, int R, float* __restrict__ out) {
+    __shared__ float tile[64][kTrRows + 1];
+    const int64_t row0 = (int64_t)blockIdx.x * kTrRows;
+    const int j0 = blockIdx.y * 64;
+    for (int e = threadIdx.x; e < kTrRows * 64; e += 256) {
+        const int rr = e >> 6, jj = e & 63;
+        const int64_t row = row0 + rr;
+        tile[jj][rr] = (row < rows && j0 + jj < R) ? sum_splits(partial, splits, rows, R, row, j0 + jj) : 0.f;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < kTrRows * 64; e += 256) {
+        const int jj = e / kTrRows, rr = e % kTrRows;
+        const int64_t row = row0 + rr;
+        if (row < rows && j0 + jj < r) out[(int64_t)(j0 + jj) * rows + row] = tile[jj][rr];
+    }
 }
 
 inline unsigned blocks(int64_t n) { return (unsigned)((n + kThreads - 1) / kThreads); }
@@ -110,15 +152,19 @@ qlora_status launch_split_hi_lo(const float* V, int64_t M, int r, int R, float s
 }
 
 qlora_status launch_dup_cols(const void* B, int64_t N, int r, int R, void* B2, cudaStream_t s) {
-    dup_cols<<<blocks(N * R), kThreads, 0, s>>>(static_cast<const uint16_t*>(B), N, r, R,
-                                                static_cast<uint16_t*>(B2));
+    if (r % 8 == 0 && (reinterpret_cast<uintptr_t>(B) & 15u) == 0)
+        dup_cols8<<<blocks(N * (R / 8)), kThreads, 0, s>>>(static_cast<const uint4*>(B), N, r / 8, R / 8,
+                                                          static_cast<uint4*>(B2));
+    else
+        dup_cols<<<blocks(N * R), kThreads, 0, s>>>(static_cast<const uint16_t*>(B), N, r, R,
+                                                    static_cast<uint16_t*>(B2));
     QLORA_CHECK_LAUNCH();
     return QLORA_OK;
 }
 
 qlora_status launch_transpose_pad(const void* B, int64_t N, int r, int R, void* Bt, cudaStream_t s) {
-    transpose_pad<<<blocks((int64_t)R * N), kThreads, 0, s>>>(static_cast<const uint16_t*>(B), N, r, R,
-                                                              static_cast<uint16_t*>(Bt));
+    const dim3 grid((unsigned)((N + 63) / 64), (unsigned)((R + 31) / 32));
+    transpose_pad<<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(B), N, r, R, static_cast<uint16_t*>(Bt));
     QLORA_CHECK_LAUNCH();
     return QLORA_OK;
 }
@@ -133,7 +179,8 @@ qlora_status launch_reduce_rows(const float* partial, int splits, int64_t rows, 
 
 qlora_status launch_reduce_transposed(const float* partial, int splits, int64_t rows, int r, int R, float* out,
                                       cudaStream_t s) {
-    reduce_transposed<<<blocks(rows * r), kThreads, 0, s>>>(partial, splits, rows, r, R, out);
+    const dim3 grid((unsigned)((rows + kTrRows - 1) / kTrRows), (unsigned)((R + 63) / 64));
+    reduce_transposed<<<grid, 256, 0, s>>>(partial, splits, rows, r, R, out);
     QLORA_CHECK_LAUNCH();
     return QLORA_OK;
 }
