@@ -48,7 +48,7 @@ constexpr int kBlocksPerCta = kQuantThreads / 2;     // 128 blocks per chunk (on
 constexpr int kCtasPerSm = 3;
 constexpr int kTableWords = kCodeBuckets * 32;       // bank-private copies: entry e of lane l at e*32 + l
 constexpr int kTreeThreads = 1024;
-constexpr int kDqThreads = 256;                      // one group of 256 blocks per CTA
+constexpr int kDqThreads = 256;                      // 8 warps, one group of 256 blocks per warp
 
 // x = fp32(w / m), correctly rounded, for |w| <= m with m in [2^-100, 2^100]:
 // Markstein's division (P. Markstein, "Computation of elementary functions on
@@ -65,43 +65,47 @@ __device__ __forceinline__ float div_markstein(float w, float m, float y) {
 // NF4 code of x in [-1, 1].  bucket k = RNE(64x + 64) comes from one FMA that
 // rounds to an integer (1.5 * 2^23 makes the fp32 ulp 1); the table keeps one
 // copy of every entry per lane (entry k of lane l at k*32 + l), so the 32 lanes
-// of a warp never meet in a shared-memory bank.
-__device__ __forceinline__ uint32_t nf4_code(float x, const float2* __restrict__ lane_table) {
-    const float y = __fmaf_rn(x, 64.f, 12582976.f);               // 1.5 * 2^23 + 64
-    const uint32_t k = __float_as_uint(y) - 0x4B400000u;          // RNE(64x + 64), 0..128
-    const float2 e = lane_table[k * 32u];
-    return (uint32_t)__float_as_int(e.y) + (x > e.x ? 1u : 0u);
+// of a warp never meet in a shared-memory bank.  The shared address of entry k
+// is table + 8*(32k + lane) = 256 * bits(y) + lane_off (mod 2^32) with
+// lane_off = table + 8*lane - 256 * 0x4B400000, one multiply-add.
+__device__ __forceinline__ uint32_t nf4_code(float x, uint32_t lane_off) {
+    const float y = __fmaf_rn(x, 64.f, 12582976.f);               // 1.5 * 2^23 + 64: bits 0x4B400000 + k
+    const uint32_t addr = __float_as_uint(y) * 256u + lane_off;
+    float thr, base;
+    asm("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(thr), "=f"(base) : "r"(addr));
+    return (uint32_t)__float_as_int(base) + (x > thr ? 1u : 0u);
 }
 
 // One pass over W.  Persistent CTAs loop over chunks of 128 consecutive NF4
-// blocks (the next chunk's weights are loaded while the current one is coded);
-// two threads share a block (32 weights each).  Per chunk: packed codes, fp32
-// block absmax, and per warp the fp64 pairwise-tree sum of its 16 blocks' c1
-// (aligned subtrees of the global tree, combined by tree_sum_pass).
+// blocks; two register buffers alternate so the next chunk's weights load
+// while the current one is coded.  Two threads share a block (32 weights
+// each).  Per chunk: packed codes, fp32 block absmax, and per warp the fp64
+// pairwise-tree sum of its 16 blocks' c1 (aligned subtrees of the global
+// tree, combined by tree_sum_pass).
 __global__ void __launch_bounds__(kQuantThreads, kCtasPerSm)
 nf4_quantize_blocks(const uint4* __restrict__ W, int64_t nb1, uint4* __restrict__ codes,
                     float* __restrict__ c1_out, double* __restrict__ warp_sums_out, int64_t n_chunks,
                     QuantBuckets qb) {
+    allow_dependents();                                       // the tree passes may be scheduled now
     __shared__ float2 table[kTableWords];
     for (int i = threadIdx.x; i < kTableWords; i += kQuantThreads) table[i] = qb.e[i >> 5];
     __syncthreads();
-    const float2* lane_table = table + (threadIdx.x & 31);
+    uint32_t table_addr;
+    asm("{ .reg .u64 t; cvta.to.shared.u64 t, %1; cvt.u32.u64 %0, t; }" : "=r"(table_addr) : "l"(table));
+    const uint32_t lane_off = table_addr + 8u * (threadIdx.x & 31) - 0x40000000u;   // 256 * 0x4B400000 mod 2^32
     const int sub = threadIdx.x & 1;
 
-    uint4 nxt[4];
-    auto load_chunk = [&](int64_t chunk) {
+    auto load_chunk = [&](uint4 (&buf)[4], int64_t chunk) {
         const int64_t blk = chunk * kBlocksPerCta + (threadIdx.x >> 1);
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-            nxt[j] = (chunk < n_chunks && blk < nb1) ? W[blk * 8 + sub * 4 + j] : make_uint4(0, 0, 0, 0);
+            buf[j] = (chunk < n_chunks && blk < nb1) ? W[blk * 8 + sub * 4 + j] : make_uint4(0, 0, 0, 0);
     };
-    load_chunk(blockIdx.x);
-    for (int64_t chunk = blockIdx.x; chunk < n_chunks; chunk += gridDim.x) {
+    auto code_chunk = [&](const uint4 (&buf)[4], int64_t chunk) {
         const int64_t blk = chunk * kBlocksPerCta + (threadIdx.x >> 1);
         const bool valid = blk < nb1;
-        const uint32_t w[16] = {nxt[0].x, nxt[0].y, nxt[0].z, nxt[0].w, nxt[1].x, nxt[1].y, nxt[1].z, nxt[1].w,
-                                nxt[2].x, nxt[2].y, nxt[2].z, nxt[2].w, nxt[3].x, nxt[3].y, nxt[3].z, nxt[3].w};
-        load_chunk(chunk + gridDim.x);
+        const uint32_t w[16] = {buf[0].x, buf[0].y, buf[0].z, buf[0].w, buf[1].x, buf[1].y, buf[1].z, buf[1].w,
+                                buf[2].x, buf[2].y, buf[2].z, buf[2].w, buf[3].x, buf[3].y, buf[3].z, buf[3].w};
         // block absmax on the bf16 bit patterns: |w| orders like the unsigned 15-bit magnitude
         uint32_t mx = 0;
 #pragma unroll
@@ -126,7 +130,7 @@ nf4_quantize_blocks(const uint4* __restrict__ W, int64_t nb1, uint4* __restrict_
                             const int i = (6 - 2 * (jj >> 1)) + (jj & 1);
                             const uint32_t pair = w[4 * q + (i >> 1)];
                             const float v = __uint_as_float((i & 1) ? (pair & 0xFFFF0000u) : (pair << 16));
-                            word = word * 16u + nf4_code(div_markstein(v, m, y), lane_table);
+                            word = word * 16u + nf4_code(div_markstein(v, m, y), lane_off);
                         }
                         out[q] = word;
                     }
@@ -139,7 +143,7 @@ nf4_quantize_blocks(const uint4* __restrict__ W, int64_t nb1, uint4* __restrict_
                             const int i = (6 - 2 * (jj >> 1)) + (jj & 1);
                             const uint32_t pair = w[4 * q + (i >> 1)];
                             const float v = __uint_as_float((i & 1) ? (pair & 0xFFFF0000u) : (pair << 16));
-                            word = word * 16u + nf4_code(__fdiv_rn(v, m), lane_table);
+                            word = word * 16u + nf4_code(__fdiv_rn(v, m), lane_off);
                         }
                         out[q] = word;
                     }
@@ -157,11 +161,24 @@ nf4_quantize_blocks(const uint4* __restrict__ W, int64_t nb1, uint4* __restrict_
         s += __shfl_xor_sync(0xffffffffu, s, 8);
         s += __shfl_xor_sync(0xffffffffu, s, 16);
         if ((threadIdx.x & 31) == 0) warp_sums_out[chunk * (kQuantThreads / 32) + (threadIdx.x >> 5)] = s;
+    };
+
+    uint4 bufA[4], bufB[4];
+    load_chunk(bufA, blockIdx.x);
+    for (int64_t chunk = blockIdx.x; chunk < n_chunks; chunk += 2 * (int64_t)gridDim.x) {
+        const int64_t next = chunk + gridDim.x;
+        load_chunk(bufB, next);
+        code_chunk(bufA, chunk);
+        if (next >= n_chunks) break;
+        load_chunk(bufA, next + gridDim.x);
+        code_chunk(bufB, next);
     }
 }
 
 __global__ void __launch_bounds__(kTreeThreads)
 tree_sum_pass(const double* __restrict__ in, int64_t n, double* __restrict__ out) {
+    grid_dependency_wait();                                   // the previous level is complete
+    allow_dependents();
     const int64_t i = (int64_t)blockIdx.x * kTreeThreads + threadIdx.x;
     double s = i < n ? in[i] : 0.0;
 #pragma unroll
@@ -177,29 +194,57 @@ tree_sum_pass(const double* __restrict__ in, int64_t n, double* __restrict__ out
     }
 }
 
+// One warp per group of 256 first-level blocks (8 consecutive c1 per lane):
+// mu from the tree sum, d = fp32(c1 - mu), c2 = max |d| over the group (warp
+// shuffles), x2 = fp32(d / c2) correctly rounded (Markstein as above for c2 in
+// [2^-100, 2^100], IEEE division outside), then its E4M3 code.
 __global__ void __launch_bounds__(kDqThreads)
 dq_blocks(const float* __restrict__ c1, int64_t nb1, const double* __restrict__ total,
           uint8_t* __restrict__ c1_codes, float* __restrict__ c2_out, float* __restrict__ mu_out) {
-    const int64_t i = (int64_t)blockIdx.x * kDqThreads + threadIdx.x;
-    const bool valid = i < nb1;
+    grid_dependency_wait();                                   // c1 and the tree sum are complete
+    const int lane = threadIdx.x & 31;
+    const int64_t g = (int64_t)blockIdx.x * (kDqThreads / 32) + (threadIdx.x >> 5);   // group
+    const int64_t nb2 = (nb1 + 255) / 256;
+    if (g >= nb2) return;
     const float mu = __double2float_rn(__ddiv_rn(*total, (double)nb1));
-    const float d = valid ? __fsub_rn(c1[i], mu) : 0.f;
-    float a = fabsf(d);
+    const int64_t i0 = g * 256 + lane * 8;
+    float d[8];
+    if (i0 + 8 <= nb1) {
+        const float4 a = reinterpret_cast<const float4*>(c1 + i0)[0];
+        const float4 b = reinterpret_cast<const float4*>(c1 + i0)[1];
+        const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
-    __shared__ float wm[kDqThreads / 32];
-    if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = a;
-    __syncthreads();
-    float c2 = wm[0];
+        for (int k = 0; k < 8; ++k) d[k] = __fsub_rn(v[k], mu);
+    } else {
 #pragma unroll
-    for (int k = 1; k < kDqThreads / 32; ++k) c2 = fmaxf(c2, wm[k]);
-    if (valid) {
-        const float x2 = (c2 > 0.f) ? __fdiv_rn(d, c2) : 0.f;
-        c1_codes[i] = (uint8_t)f32_to_e4m3_rn_sat(x2);
+        for (int k = 0; k < 8; ++k) d[k] = i0 + k < nb1 ? __fsub_rn(c1[i0 + k], mu) : 0.f;
     }
-    if (threadIdx.x == 0) {
-        c2_out[blockIdx.x] = c2;
-        if (blockIdx.x == 0) *mu_out = mu;
+    float c2 = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) c2 = fmaxf(c2, fabsf(d[k]));
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) c2 = fmaxf(c2, __shfl_xor_sync(0xffffffffu, c2, off));
+    uint32_t code[8];
+    if (c2 >= 7.8886091e-31f && c2 <= 1.2676506e30f) {
+        const float y = __frcp_rn(c2);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) code[k] = f32_to_e4m3_rn_sat(div_markstein(d[k], c2, y));
+    } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) code[k] = f32_to_e4m3_rn_sat(c2 > 0.f ? __fdiv_rn(d[k], c2) : 0.f);
+    }
+    if (i0 + 8 <= nb1) {
+        const uint2 packed = make_uint2(code[0] | code[1] << 8 | code[2] << 16 | code[3] << 24,
+                                        code[4] | code[5] << 8 | code[6] << 16 | code[7] << 24);
+        reinterpret_cast<uint2*>(c1_codes + i0)[0] = packed;
+    } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            if (i0 + k < nb1) c1_codes[i0 + k] = (uint8_t)code[k];
+    }
+    if (lane == 0) {
+        c2_out[g] = c2;
+        if (g == 0) *mu_out = mu;
     }
 }
 
@@ -242,13 +287,16 @@ qlora_status launch_quantize(const void* W, int64_t N, int64_t K, const qlora_nf
         const int64_t np = (p + kTreeThreads - 1) / kTreeThreads;
         double* next = reinterpret_cast<double*>(ws);
         ws += align_up((size_t)np * sizeof(double), 256);
-        tree_sum_pass<<<(unsigned)np, kTreeThreads, 0, stream>>>(level, p, next);
+        (void)launch_dependent(tree_sum_pass, dim3((unsigned)np), dim3(kTreeThreads), 0, stream,
+                               (const double*)level, p, next);
         QLORA_CHECK_LAUNCH();
         level = next;
         p = np;
     }
     const int64_t nb2 = (nb1 + 255) / 256;
-    dq_blocks<<<(unsigned)nb2, kDqThreads, 0, stream>>>(c1, nb1, level, out->c1_codes, out->c2, out->mu);
+    (void)launch_dependent(dq_blocks, dim3((unsigned)((nb2 + kDqThreads / 32 - 1) / (kDqThreads / 32))),
+                           dim3(kDqThreads), 0, stream, (const float*)c1, nb1, (const double*)level,
+                           out->c1_codes, out->c2, out->mu);
     QLORA_CHECK_LAUNCH();
     return QLORA_OK;
 }
