@@ -36,6 +36,8 @@ METRIC = "QLoRA linear fwd+bwd TFLOP/s and small-M GB/s, as fraction of B200 roo
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
 PACKED_BYTES_PER_WEIGHT = 0.5 + 1 / 64 + 4 / (64 * 256)     # codes + E4M3 constants + c2
+ALU_OPS_PER_WEIGHT = 2.5        # exact bf16 table expansion: 19 permute/logic ops per 8 weights + 8 per 64-weight table
+ALU_OPS_PER_CLK_SM = 62.0       # byte-permute / logic issue rate per SM, measured
 
 
 def parse_args():
@@ -326,8 +328,15 @@ def decode_sweep(device, peaks):
     import bit_nf4_quantized_23_b200 as q4
     import synthetic_inputs as si
     wl = si.WORKLOADS["decode"]
-    l2 = torch.cuda.get_device_properties(device).L2_cache_size
-    out = {}
+    props = torch.cuda.get_device_properties(device)
+    l2 = props.L2_cache_size
+    # ALU roofline of an exact bf16 dequant (every weight through a per-block 16-entry table):
+    # >= 2.5 byte-permute/logic ops per weight on a pipe that issues 62 per clock per SM
+    alu_gbs = (ALU_OPS_PER_CLK_SM * props.multi_processor_count * peaks.get("sm_max_mhz", 1965.0) * 1e6
+               / ALU_OPS_PER_WEIGHT * PACKED_BYTES_PER_WEIGHT / 1e9)
+    out = {"alu_roofline_GB/s": round(alu_gbs, 1),
+           "alu_roofline_basis": f"{ALU_OPS_PER_WEIGHT} ALU ops/weight, {ALU_OPS_PER_CLK_SM} ops/clk/SM (measured "
+                                 "pipe probe), SMs x max SM clock"}
     for i, (N, K) in enumerate(wl.linears):
         W = si.weight(wl, i).to(device)
         A, B = (t.to(device) for t in si.lora(wl, i))
@@ -362,7 +371,8 @@ def decode_sweep(device, peaks):
             out[f"W[{N},{K}] M={M}"] = {
                 "call_us": round(ms * 1e3, 2), "call_GB/s": round(wbytes / (ms * 1e-3) / 1e9, 1),
                 "kernel_us": round(kms * 1e3, 2), "kernel_GB/s": round(wbytes / (kms * 1e-3) / 1e9, 1),
-                "kernel_frac_of_hbm": round(wbytes / (kms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3)}
+                "kernel_frac_of_hbm": round(wbytes / (kms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3),
+                "kernel_frac_of_alu_roofline": round(wbytes / (kms * 1e-3) / 1e9 / alu_gbs, 3)}
         del ws
         torch.cuda.empty_cache()
     return out
