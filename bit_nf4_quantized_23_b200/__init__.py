@@ -18,7 +18,8 @@ import torch
 from ._lib import (QLORA_DTYPE_BF16, QLORA_DTYPE_F32, TIMER_KINDS, NF4WeightC, QloraError, check, lib)
 
 __all__ = [
-    "NF4Weight", "QloraError", "qlora_nf4_sizes", "qlora_nf4_codebook", "qlora_quantize_nf4_dq",
+    "NF4Weight", "QloraError", "CODEBOOKS", "qlora_nf4_sizes", "qlora_nf4_codebook", "qlora_codebook_values",
+    "qlora_quantize_nf4_dq",
     "qlora_quantize_nf4_dq_noalloc",
     "qlora_dequantize", "qlora_linear_workspace_size", "qlora_linear_fwd", "qlora_linear_bwd",
     "qlora_read_device_errors", "qlora_launch_count", "qlora_timing_enable", "qlora_timing_read",
@@ -55,25 +56,41 @@ def _dtype_code(dtype) -> int:
 
 @dataclass
 class NF4Weight:
-    """The four stored buffers of an NF4 + DQ weight (device tensors) and its shape."""
-    codes: torch.Tensor      # uint8 [N*K/2]
-    c1_codes: torch.Tensor   # uint8 [N*K/64]  (FP8 E4M3 bit patterns)
-    c2: torch.Tensor         # fp32 [ceil(N*K/64/256)]
-    mu: torch.Tensor         # fp32 [1]
+    """The stored buffers of a 4-bit quantized weight (device tensors) and its shape.
+
+    With double quantization (the default) the block constants are c1_codes, c2 and mu and
+    `c1` is None; without it `c1` holds the fp32 block absmax values and the other three are
+    None.  `codebook` is "nf4" or "uniform4" (the uniform 4-bit grid NF4 is compared with)."""
+    codes: torch.Tensor                 # uint8 [N*K/2]
+    c1_codes: torch.Tensor | None       # uint8 [N*K/64]  (FP8 E4M3 bit patterns)
+    c2: torch.Tensor | None             # fp32 [ceil(N*K/64/256)]
+    mu: torch.Tensor | None             # fp32 [1]
     N: int
     K: int
+    codebook: str = "nf4"
+    c1: torch.Tensor | None = None      # fp32 [N*K/64] when double quantization is off
 
     def c_struct(self) -> NF4WeightC:
-        return NF4WeightC(self.codes.data_ptr(), self.c1_codes.data_ptr(), self.c2.data_ptr(),
-                          self.mu.data_ptr(), self.N, self.K, 64, 256)
+        p = lambda t: t.data_ptr() if t is not None else None
+        return NF4WeightC(self.codes.data_ptr(), p(self.c1_codes), p(self.c2), p(self.mu), self.N, self.K,
+                          64, 256, CODEBOOKS[self.codebook], 0, p(self.c1))
 
     @staticmethod
-    def empty(N: int, K: int, device="cuda") -> "NF4Weight":
+    def empty(N: int, K: int, device="cuda", codebook: str = "nf4", double_quant: bool = True) -> "NF4Weight":
+        if codebook not in CODEBOOKS:
+            raise ValueError(f"codebook must be one of {sorted(CODEBOOKS)}")
         s = qlora_nf4_sizes(N, K)
-        return NF4Weight(torch.empty(s["codes"], dtype=torch.uint8, device=device),
+        codes = torch.empty(s["codes"], dtype=torch.uint8, device=device)
+        if not double_quant:
+            return NF4Weight(codes, None, None, None, N, K, codebook,
+                             torch.empty(s["c1_codes"], dtype=torch.float32, device=device))
+        return NF4Weight(codes,
                          torch.empty(s["c1_codes"], dtype=torch.uint8, device=device),
                          torch.empty(s["c2"] // 4, dtype=torch.float32, device=device),
-                         torch.empty(1, dtype=torch.float32, device=device), N, K)
+                         torch.empty(1, dtype=torch.float32, device=device), N, K, codebook)
+
+
+CODEBOOKS = {"nf4": 0, "uniform4": 1}
 
 
 def qlora_nf4_sizes(N: int, K: int, blocksize: int = 64, blocksize2: int = 256) -> dict:
@@ -91,16 +108,26 @@ def qlora_nf4_codebook():
     return list(v), list(t)
 
 
+def qlora_codebook_values(codebook: str = "nf4"):
+    """(values[16], thresholds[15]) of a codebook ("nf4" or "uniform4")."""
+    v = (c_float * 16)()
+    t = (c_float * 15)()
+    check(lib().qlora_codebook_values(CODEBOOKS[codebook], v, t), "qlora_codebook_values")
+    return list(v), list(t)
+
+
 def qlora_quantize_nf4_dq(W: torch.Tensor, blocksize: int = 64, blocksize2: int = 256,
                           out: NF4Weight | None = None, workspace: torch.Tensor | None = None,
-                          stream=None) -> NF4Weight:
+                          stream=None, codebook: str = "nf4", double_quant: bool = True) -> NF4Weight:
+    """Quantize W (bf16 [N, K]); `codebook` and `double_quant` apply when `out` is None
+    (otherwise `out` carries them)."""
     _need(W, torch.bfloat16, "W")
     if W.dim() != 2:
         raise ValueError("W must be 2-D [N, K]")
     N, K = W.shape
     sizes = qlora_nf4_sizes(N, K, blocksize, blocksize2)
     if out is None:
-        out = NF4Weight.empty(N, K, W.device)
+        out = NF4Weight.empty(N, K, W.device, codebook, double_quant)
     if workspace is None:
         workspace = torch.empty(sizes["workspace"], dtype=torch.uint8, device=W.device)
     ws = out.c_struct()

@@ -28,7 +28,8 @@ _W = None  # placeholder, replaced by POINTER(NF4WeightC) below
 class NF4WeightC(ctypes.Structure):
     """Mirror of qlora_nf4_weight."""
     _fields_ = [("codes", c_void_p), ("c1_codes", c_void_p), ("c2", c_void_p), ("mu", c_void_p),
-                ("N", c_int64), ("K", c_int64), ("blocksize", c_int32), ("blocksize2", c_int32)]
+                ("N", c_int64), ("K", c_int64), ("blocksize", c_int32), ("blocksize2", c_int32),
+                ("codebook", c_int32), ("reserved", c_int32), ("c1", c_void_p)]
 
 
 _W = POINTER(NF4WeightC)
@@ -38,6 +39,7 @@ SIGNATURES = {
     "qlora_nf4_sizes": (c_int32, [c_int64, c_int64, c_int32, c_int32, POINTER(c_size_t), POINTER(c_size_t),
                                   POINTER(c_size_t), POINTER(c_size_t)]),
     "qlora_nf4_codebook": (c_int32, [POINTER(c_float), POINTER(c_float)]),
+    "qlora_codebook_values": (c_int32, [c_int32, POINTER(c_float), POINTER(c_float)]),
     "qlora_quantize_nf4_dq": (c_int32, [c_void_p, c_int64, c_int64, c_int32, c_int32, _W, c_void_p,
                                         c_size_t, c_void_p]),
     "qlora_quantize_nf4_dq_noalloc": (c_int32, [c_void_p, c_int64, c_int64, c_int32, c_int32, _W, c_void_p]),

@@ -5,6 +5,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstdlib>
+#include <climits>
 #include <cstring>
 #include <mutex>
 
@@ -44,6 +45,7 @@ qlora_status check_blocks(int32_t bs, int32_t bs2) {
 qlora_status check_shape(int64_t N, int64_t K) {
     if (N < 1 || K < 1 || K % 64 != 0) return QLORA_ERR_SHAPE;
     if (N > (int64_t(1) << 40) / K) return QLORA_ERR_SHAPE;   // keeps every flat index in int64 range
+    if (N > INT32_MAX || K > INT32_MAX) return QLORA_ERR_SHAPE;  // tensor-map coordinates are 32-bit
     return QLORA_OK;
 }
 
@@ -51,9 +53,16 @@ qlora_status check_weight(const qlora_nf4_weight* w) {
     if (!w) return QLORA_ERR_INVALID_ARG;
     QLORA_TRY(check_blocks(w->blocksize, w->blocksize2));
     QLORA_TRY(check_shape(w->N, w->K));
-    if (!w->codes || !w->c1_codes || !w->c2 || !w->mu) return QLORA_ERR_INVALID_ARG;
-    if (!aligned16(w->codes) || !aligned16(w->c1_codes) || !aligned16(w->c2) || !aligned16(w->mu))
-        return QLORA_ERR_ALIGN;
+    if (w->codebook != QLORA_CODEBOOK_NF4 && w->codebook != QLORA_CODEBOOK_UNIFORM4) return QLORA_ERR_INVALID_ARG;
+    if (w->reserved != 0) return QLORA_ERR_INVALID_ARG;
+    if (!w->codes) return QLORA_ERR_INVALID_ARG;
+    if (!aligned16(w->codes)) return QLORA_ERR_ALIGN;
+    if (w->c1) {   // double quantization off: fp32 block constants only
+        if (!aligned16(w->c1)) return QLORA_ERR_ALIGN;
+        return QLORA_OK;
+    }
+    if (!w->c1_codes || !w->c2 || !w->mu) return QLORA_ERR_INVALID_ARG;
+    if (!aligned16(w->c1_codes) || !aligned16(w->c2) || !aligned16(w->mu)) return QLORA_ERR_ALIGN;
     return QLORA_OK;
 }
 
@@ -173,11 +182,16 @@ qlora_status qlora_nf4_sizes(int64_t N, int64_t K, int32_t blocksize, int32_t bl
     return QLORA_OK;
 }
 
-qlora_status qlora_nf4_codebook(float values[16], float thresholds[15]) {
-    const NF4Tables& tb = host_tables();
+qlora_status qlora_codebook_values(int32_t codebook, float values[16], float thresholds[15]) {
+    if (codebook != QLORA_CODEBOOK_NF4 && codebook != QLORA_CODEBOOK_UNIFORM4) return QLORA_ERR_INVALID_ARG;
+    const NF4Tables& tb = host_tables(codebook);
     if (values) std::memcpy(values, tb.q, sizeof(tb.q));
     if (thresholds) std::memcpy(thresholds, tb.t, sizeof(tb.t));
     return QLORA_OK;
+}
+
+qlora_status qlora_nf4_codebook(float values[16], float thresholds[15]) {
+    return qlora_codebook_values(QLORA_CODEBOOK_NF4, values, thresholds);
 }
 
 qlora_status qlora_quantize_nf4_dq(const void* W, int64_t N, int64_t K, int32_t blocksize,

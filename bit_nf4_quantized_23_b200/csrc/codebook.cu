@@ -1,5 +1,5 @@
-// Host construction of the NF4 code values and the quantize kernel's decision
-// thresholds.
+// Host construction of the code values (NF4, and the uniform 4-bit grid it is
+// compared with) and the quantize kernel's decision thresholds.
 //
 // The code values are normal quantiles ("Science Depth M5-131: PEFT (LoRA /
 // QLoRA / Prefix Tuning)", section 3, NF4): 16 points with equal probability
@@ -46,22 +46,30 @@ double normal_quantile(double p) {
     return x;
 }
 
-NF4Tables build_tables() {
-    const double delta = 0.5 * ((1.0 - 1.0 / 30.0) + (1.0 - 1.0 / 32.0));
+NF4Tables build_tables(int codebook) {
     double v[16];
-    int n = 0;
-    for (int j = 0; j < 8; ++j) v[n++] = normal_quantile(delta - j * (delta - 0.5) / 8.0);
-    for (int j = 0; j < 7; ++j) v[n++] = -normal_quantile(delta - j * (delta - 0.5) / 7.0);
-    v[n++] = 0.0;
-    // insertion sort, ascending
-    for (int i = 1; i < 16; ++i) {
-        double key = v[i];
-        int j = i - 1;
-        while (j >= 0 && v[j] > key) { v[j + 1] = v[j]; --j; }
-        v[j + 1] = key;
+    double top = 1.0;
+    if (codebook == QLORA_CODEBOOK_UNIFORM4) {
+        // 16 evenly spaced values on [-1, 1]: i * (2/15) - 1 in double, the last exactly 1
+        const double step = 2.0 / 15.0;
+        for (int i = 0; i < 15; ++i) v[i] = (double)i * step + (-1.0);
+        v[15] = 1.0;
+    } else {
+        const double delta = 0.5 * ((1.0 - 1.0 / 30.0) + (1.0 - 1.0 / 32.0));
+        int n = 0;
+        for (int j = 0; j < 8; ++j) v[n++] = normal_quantile(delta - j * (delta - 0.5) / 8.0);
+        for (int j = 0; j < 7; ++j) v[n++] = -normal_quantile(delta - j * (delta - 0.5) / 7.0);
+        v[n++] = 0.0;
+        // insertion sort, ascending
+        for (int i = 1; i < 16; ++i) {
+            double key = v[i];
+            int j = i - 1;
+            while (j >= 0 && v[j] > key) { v[j + 1] = v[j]; --j; }
+            v[j + 1] = key;
+        }
+        top = v[0];
+        for (int i = 1; i < 16; ++i) top = v[i] > top ? v[i] : top;
     }
-    double top = v[0];
-    for (int i = 1; i < 16; ++i) top = v[i] > top ? v[i] : top;
     NF4Tables tb;
     for (int i = 0; i < 16; ++i) tb.q[i] = (float)(v[i] / top);
     for (int j = 0; j < 15; ++j) {
@@ -100,18 +108,20 @@ QuantBuckets build_buckets(const NF4Tables& tb) {
 
 }  // namespace
 
-const QuantBuckets& host_buckets() {
-    static std::once_flag once;
-    static QuantBuckets qb;
-    std::call_once(once, [] { qb = build_buckets(host_tables()); });
-    return qb;
+const QuantBuckets& host_buckets(int codebook) {
+    static std::once_flag once[2];
+    static QuantBuckets qb[2];
+    const int c = codebook == QLORA_CODEBOOK_UNIFORM4 ? 1 : 0;
+    std::call_once(once[c], [c] { qb[c] = build_buckets(host_tables(c)); });
+    return qb[c];
 }
 
-const NF4Tables& host_tables() {
-    static std::once_flag once;
-    static NF4Tables tables;
-    std::call_once(once, [] { tables = build_tables(); });
-    return tables;
+const NF4Tables& host_tables(int codebook) {
+    static std::once_flag once[2];
+    static NF4Tables tables[2];
+    const int c = codebook == QLORA_CODEBOOK_UNIFORM4 ? 1 : 0;
+    std::call_once(once[c], [c] { tables[c] = build_tables(c); });
+    return tables[c];
 }
 
 }  // namespace qlora

@@ -2,7 +2,8 @@
 // PEFT (LoRA / QLoRA / Prefix Tuning)", section 4 (1): W_hat = Dequant(W_NF4) * c1,
 // performed on the fly in forward and backward).
 //
-// W_hat[n,k] = bf16_rn(fp32(q[code] * c1')), c1' = fp32(fp32(e4m3(c1_code) * c2) + mu).
+// W_hat[n,k] = bf16_rn(fp32(q[code] * c1')), c1' = fp32(fp32(e4m3(c1_code) * c2) + mu),
+// or c1' = c1 when double quantization is off (fp32 constants stored).
 // HBM-bound: 0.516 bytes read and 2 bytes written per weight.  Each thread
 // expands 16 weights (8 code bytes -> 32 output bytes, 16-byte stores).
 #include "qlora_internal.cuh"
@@ -14,7 +15,7 @@ constexpr int kDeqThreads = 256;
 
 __global__ void __launch_bounds__(kDeqThreads)
 nf4_dequantize(const uint2* __restrict__ codes, const uint8_t* __restrict__ c1_codes,
-               const float* __restrict__ c2, const float* __restrict__ mu_p,
+               const float* __restrict__ c2, const float* __restrict__ mu_p, const float* __restrict__ c1f,
                int64_t n16, uint4* __restrict__ out, NF4Tables tb) {
     __shared__ float q[16];
     if (threadIdx.x < 16) q[threadIdx.x] = tb.q[threadIdx.x];
@@ -22,7 +23,7 @@ nf4_dequantize(const uint2* __restrict__ codes, const uint8_t* __restrict__ c1_c
     const int64_t i = (int64_t)blockIdx.x * kDeqThreads + threadIdx.x;   // group of 16 weights
     if (i >= n16) return;
     const int64_t blk = i >> 2;
-    const float c1p = rebuild_c1(c1_codes[blk], c2[blk >> 8], *mu_p);
+    const float c1p = c1f ? c1f[blk] : rebuild_c1(c1_codes[blk], c2[blk >> 8], *mu_p);
     const uint2 c = codes[i];
     uint32_t o[8];
 #pragma unroll
@@ -42,8 +43,8 @@ qlora_status launch_dequantize(const qlora_nf4_weight* w, void* W_out, cudaStrea
     const int64_t n16 = w->N * w->K / 16;
     const unsigned grid = (unsigned)((n16 + kDeqThreads - 1) / kDeqThreads);
     nf4_dequantize<<<grid, kDeqThreads, 0, stream>>>(
-        reinterpret_cast<const uint2*>(w->codes), w->c1_codes, w->c2, w->mu, n16,
-        static_cast<uint4*>(W_out), host_tables());
+        reinterpret_cast<const uint2*>(w->codes), w->c1_codes, w->c2, w->mu, w->c1, n16,
+        static_cast<uint4*>(W_out), host_tables(w->codebook));
     QLORA_CHECK_LAUNCH();
     return QLORA_OK;
 }

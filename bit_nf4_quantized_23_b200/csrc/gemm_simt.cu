@@ -30,7 +30,7 @@ __device__ __forceinline__ float load_operand(const SimtOperand& op, int64_t row
             const uint32_t byte = static_cast<const uint8_t*>(op.ptr)[flat >> 1];
             const uint32_t code = (flat & 1) ? (byte & 0xFu) : (byte >> 4);
             const int64_t blk = flat >> 6;
-            const float c1p = rebuild_c1(op.c1_codes[blk], op.c2[blk >> 8], *op.mu);
+            const float c1p = op.c1f ? op.c1f[blk] : rebuild_c1(op.c1_codes[blk], op.c2[blk >> 8], *op.mu);
             return bf16_bits_to_f32(dequant_bits(q[code], c1p));
         }
     }
@@ -108,7 +108,11 @@ simt_gemm(SimtGemm g, NF4Tables tb) {
 qlora_status launch_simt_gemm(const SimtGemm& g, cudaStream_t stream) {
     if (g.M <= 0 || g.N <= 0) return QLORA_OK;
     const dim3 grid((unsigned)((g.N + kTile - 1) / kTile), (unsigned)((g.M + kTile - 1) / kTile));
-    simt_gemm<<<grid, kThreads, 0, stream>>>(g, host_tables());
+    int codebook = QLORA_CODEBOOK_NF4;
+    for (int i = 0; i < g.nseg; ++i)
+        for (const SimtOperand* o : {&g.seg[i].a, &g.seg[i].b})
+            if (o->kind == SIMT_NF4 || o->kind == SIMT_NF4_T) codebook = o->codebook;
+    simt_gemm<<<grid, kThreads, 0, stream>>>(g, host_tables(codebook));
     QLORA_CHECK_LAUNCH();
     return QLORA_OK;
 }

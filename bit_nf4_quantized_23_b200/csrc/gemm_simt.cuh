@@ -19,7 +19,9 @@ struct SimtOperand {
     const uint8_t* c1_codes;    // NF4 kinds only
     const float* c2;
     const float* mu;
+    const float* c1f;           // NF4 kinds with double quantization off: fp32 block constants
     int64_t WK;                 // columns of W (NF4 kinds)
+    int32_t codebook;           // NF4 kinds: qlora_codebook
 };
 
 struct SimtSegment {
@@ -47,7 +49,8 @@ inline SimtOperand simt_dense(int32_t kind, const void* p, int64_t s_row, int64_
 inline SimtOperand simt_nf4(const qlora_nf4_weight* w, bool transposed) {
     SimtOperand o{};
     o.kind = transposed ? SIMT_NF4_T : SIMT_NF4;
-    o.ptr = w->codes; o.c1_codes = w->c1_codes; o.c2 = w->c2; o.mu = w->mu; o.WK = w->K;
+    o.ptr = w->codes; o.c1_codes = w->c1_codes; o.c2 = w->c2; o.mu = w->mu; o.c1f = w->c1; o.WK = w->K;
+    o.codebook = w->codebook;
     return o;
 }
 

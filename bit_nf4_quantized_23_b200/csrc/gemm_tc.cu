@@ -264,7 +264,7 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
         // dX: W row it*64 + (t & 63), K-block (n0 + 64*kc)/64 with kc = t >> 6.
         // The block constants are loaded kGemmPrefetch K-steps ahead (register queue).
         const int t = threadIdx.x - 64;
-        const float mu = *p.mu;
+        const float mu = p.c1f ? 0.f : *p.mu;
         const int64_t blocks_per_row = p.WK / 64;
         const uint32_t row = DX ? (uint32_t)(t & 63) : (uint32_t)t;
         const uint32_t kc = DX ? (uint32_t)(t >> 6) : 0u;
@@ -283,8 +283,12 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
             qcode[d] = 0;
             qc2[d] = 0.f;
             if (qblk[d] >= 0) {
-                qcode[d] = __ldg(p.c1_codes + qblk[d]);
-                qc2[d] = __ldg(p.c2 + (qblk[d] >> 8));
+                if (p.c1f) {   // single-level constants: the queue's c2 slot carries c1
+                    qc2[d] = __ldg(p.c1f + qblk[d]);
+                } else {
+                    qcode[d] = __ldg(p.c1_codes + qblk[d]);
+                    qc2[d] = __ldg(p.c2 + (qblk[d] >> 8));
+                }
             }
         }
         bool ok = true;
@@ -292,7 +296,7 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
             const int s = it % kStages;
             const uint32_t ph = (uint32_t)(it / kStages) & 1u;
             const int64_t blk = qblk[0];
-            const float c1p = blk >= 0 ? rebuild_c1(qcode[0], qc2[0], mu) : 0.f;
+            const float c1p = blk < 0 ? 0.f : (p.c1f ? qc2[0] : rebuild_c1(qcode[0], qc2[0], mu));
 #pragma unroll
             for (int d = 0; d + 1 < kGemmPrefetch; ++d) {
                 qblk[d] = qblk[d + 1];
@@ -304,8 +308,12 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
                 const int64_t b = ahead < ks0 ? unit_block(ahead) : -1;
                 qblk[kGemmPrefetch - 1] = b;
                 if (b >= 0) {
-                    qcode[kGemmPrefetch - 1] = __ldg(p.c1_codes + b);
-                    qc2[kGemmPrefetch - 1] = __ldg(p.c2 + (b >> 8));
+                    if (p.c1f) {
+                        qc2[kGemmPrefetch - 1] = __ldg(p.c1f + b);
+                    } else {
+                        qcode[kGemmPrefetch - 1] = __ldg(p.c1_codes + b);
+                        qc2[kGemmPrefetch - 1] = __ldg(p.c2 + (b >> 8));
+                    }
                 }
             }
             ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_full_a + 8 * s, ph, abort, p.err));
@@ -580,7 +588,7 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, const __grid_constant
         const int t = threadIdx.x - 64 - 128 * g;
         const int64_t nb1 = p.N * (p.K / 64);
         const int64_t kb = p.K / 64;
-        const float mu = *p.mu;
+        const float mu = p.c1f ? 0.f : *p.mu;
         // a unit cursor: tile, step and the first-level block index of row tile*128 + t at step 0
         struct Cursor { int64_t tile, rowblk; int step; };
         auto advance = [&](Cursor& c, int by) {
@@ -594,8 +602,12 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, const __grid_constant
             if (c.tile * 128 + t >= p.N) return;
             const int64_t blk = c.rowblk + c.step;
             if (blk >= nb1) { atomicOr(p.err, ERR_FLAG_BOUNDS); atomicMax(p.dbg, 0x20000000u); return; }
-            code = __ldg(p.c1_codes + blk);
-            c2 = __ldg(p.c2 + (blk >> 8));
+            if (p.c1f) {   // single-level constants: the queue's c2 slot carries c1
+                c2 = __ldg(p.c1f + blk);
+            } else {
+                code = __ldg(p.c1_codes + blk);
+                c2 = __ldg(p.c2 + (blk >> 8));
+            }
         };
         uint32_t qcode[kDecPrefetch];
         float qc2[kDecPrefetch];
@@ -636,7 +648,8 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, const __grid_constant
             const int seg = (int)(cur.tile - t0);
             while (epi_seg < seg && ok) { ok = epilogue(epi_seg); epi_seg += 2; }
             if (!ok) break;
-            const float c1p = __fadd_rn(__fmul_rn(e4tab[qcode[0]], qc2[0]), mu);   // c1' = fp32(fp32(v8 c2) + mu)
+            const float c1p = p.c1f ? qc2[0]                                  // c1' = c1, or
+                                    : __fadd_rn(__fmul_rn(e4tab[qcode[0]], qc2[0]), mu);   // fp32(fp32(v8 c2) + mu)
 #pragma unroll
             for (int d = 0; d + 1 < kDecPrefetch; ++d) {
                 qcode[d] = qcode[d + 1];
@@ -868,9 +881,9 @@ qlora_status launch_tc_decode(const DecodeArgs& a, cudaStream_t stream) {
     const int64_t tiles = (N + 127) / 128;
     p.units = tiles * p.ksteps;
     p.grid = decode_grid(p.units, sms);
-    p.c1_codes = w->c1_codes; p.c2 = w->c2; p.mu = w->mu;
+    p.c1_codes = w->c1_codes; p.c2 = w->c2; p.mu = w->mu; p.c1f = w->c1;
     p.partial = a.partial;
-    p.tb = host_tables();
+    p.tb = host_tables(w->codebook);
     p.err = device_error_word();
     if (!p.err) return QLORA_ERR_CUDA;
     p.dbg = p.err + 1;
@@ -919,11 +932,12 @@ qlora_status launch_tc_gemm_nf4(TcGemmArgs& a, bool dx, cudaStream_t stream) {
     a.p.ksteps0 = (int)(((dx ? N : K) + 63) / 64);
     a.p.ksteps1 = (int)(R2 / 64);
     a.p.c1_codes = w->c1_codes;
+    a.p.c1f = w->c1;
     a.p.c2 = w->c2;
     a.p.mu = w->mu;
     a.p.WN = N;
     a.p.WK = K;
-    a.p.tb = host_tables();
+    a.p.tb = host_tables(w->codebook);
     a.p.err = device_error_word();
     if (!a.p.err) return QLORA_ERR_CUDA;
     if (bm == 256) return dx ? launch_one<2, true>(a, stream) : launch_one<2, false>(a, stream);

@@ -15,6 +15,7 @@ struct TcGemmParams {
     const uint8_t* c1_codes;
     const float* c2;
     const float* mu;
+    const float* c1f;       // double quantization off: fp32 block constants (c1_codes, c2, mu unused)
     int64_t WN, WK;         // shape of W
     void* out;
     int64_t ldo;
@@ -46,6 +47,7 @@ struct DecodeParams {
     const uint8_t* c1_codes;
     const float* c2;
     const float* mu;
+    const float* c1f;       // double quantization off: fp32 block constants (c1_codes, c2, mu unused)
     float* partial;         // [tiles + grid][16][128] fp32 partial tiles, slot = tile + CTA
     uint32_t* err;
     uint32_t* dbg;          // second device word: where a self-check or a wait gave up

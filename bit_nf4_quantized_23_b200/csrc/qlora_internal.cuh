@@ -32,9 +32,9 @@ struct QuantBuckets {
     float2 e[kCodeBuckets];   // (.x = threshold, .y = base code as int bits)
 };
 
-// Host side: the library's tables, built once (codebook.cu).
-const NF4Tables& host_tables();
-const QuantBuckets& host_buckets();
+// Host side: the tables of a codebook (qlora_codebook), built once (codebook.cu).
+const NF4Tables& host_tables(int codebook = QLORA_CODEBOOK_NF4);
+const QuantBuckets& host_buckets(int codebook = QLORA_CODEBOOK_NF4);
 
 // Host side: count of kernels launched by this library (api.cu).
 void note_launches(int n);

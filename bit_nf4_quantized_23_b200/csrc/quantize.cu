@@ -269,7 +269,8 @@ qlora_status launch_quantize(const void* W, int64_t N, int64_t K, const qlora_nf
                              void* workspace, cudaStream_t stream) {
     const int64_t nb1 = N * K / 64;
     char* ws = static_cast<char*>(workspace);
-    float* c1 = reinterpret_cast<float*>(ws);
+    // with double quantization off the block constants are the output itself
+    float* c1 = out->c1 ? out->c1 : reinterpret_cast<float*>(ws);
     ws += align_up((size_t)nb1 * sizeof(float), 256);
     const int64_t n_chunks = (nb1 + kBlocksPerCta - 1) / kBlocksPerCta;
     int64_t p = n_chunks * (kQuantThreads / 32);                 // first tree level: one sum per 16 blocks
@@ -281,8 +282,9 @@ qlora_status launch_quantize(const void* W, int64_t N, int64_t K, const qlora_nf
     const int64_t grid = std::min<int64_t>(n_chunks, (int64_t)sms * kCtasPerSm);
     nf4_quantize_blocks<<<(unsigned)grid, kQuantThreads, 0, stream>>>(
         static_cast<const uint4*>(W), nb1, reinterpret_cast<uint4*>(out->codes), c1, level, n_chunks,
-        host_buckets());
+        host_buckets(out->codebook));
     QLORA_CHECK_LAUNCH();
+    if (out->c1) return QLORA_OK;                             // single-level quantization: done
     while (p > 1) {
         const int64_t np = (p + kTreeThreads - 1) / kTreeThreads;
         double* next = reinterpret_cast<double*>(ws);

@@ -73,9 +73,13 @@ extern "C" qlora_status qlora_quantize_nf4_dq_noalloc(const void* W, int64_t N, 
     if (blocksize != 64 || blocksize2 != 256) return QLORA_ERR_UNSUPPORTED;
     if (N < 1 || K < 1 || K % 64 != 0) return QLORA_ERR_SHAPE;
     if (N > kNoAllocMaxWeights / K) return QLORA_ERR_TOO_LARGE;
-    if (!W || !out || !out->codes || !out->c1_codes || !out->c2 || !out->mu) return QLORA_ERR_INVALID_ARG;
-    if (!aligned16(W) || !aligned16(out->codes) || !aligned16(out->c1_codes) || !aligned16(out->c2) ||
-        !aligned16(out->mu))
+    if (!W || !out || !out->codes) return QLORA_ERR_INVALID_ARG;
+    if (out->codebook != QLORA_CODEBOOK_NF4 && out->codebook != QLORA_CODEBOOK_UNIFORM4) return QLORA_ERR_INVALID_ARG;
+    if (out->reserved != 0) return QLORA_ERR_INVALID_ARG;
+    if (!out->c1 && (!out->c1_codes || !out->c2 || !out->mu)) return QLORA_ERR_INVALID_ARG;
+    if (!aligned16(W) || !aligned16(out->codes)) return QLORA_ERR_ALIGN;
+    if (out->c1 ? !aligned16(out->c1)
+                : (!aligned16(out->c1_codes) || !aligned16(out->c2) || !aligned16(out->mu)))
         return QLORA_ERR_ALIGN;
     if (out->N != N || out->K != K || out->blocksize != 64 || out->blocksize2 != 256) return QLORA_ERR_SHAPE;
     if (quantize_workspace_bytes(N * K / 64) > kNoAllocScratchBytes) return QLORA_ERR_TOO_LARGE;

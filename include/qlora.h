@@ -60,25 +60,41 @@ typedef enum {
 
 typedef enum { QLORA_DTYPE_BF16 = 0, QLORA_DTYPE_F32 = 1 } qlora_dtype;
 
+/* Code-value sets (the 16 values a 4-bit code indexes). */
+typedef enum {
+    QLORA_CODEBOOK_NF4 = 0,       /* NormalFloat: normal quantiles with an exact zero ([SD] section 3 part 1) */
+    QLORA_CODEBOOK_UNIFORM4 = 1   /* 16 evenly spaced values on [-1, 1] (the uniform 4-bit grid NF4 is
+                                     compared with, [SD] section 4 (2)); no exact zero */
+} qlora_codebook;
+
 /*
- * A quantized frozen weight: the four stored buffers of NF4 + Double
- * Quantization ([SD] section 3, parts 1 and 2).  All four pointers are device
- * memory owned by the caller; sizes come from qlora_nf4_sizes().
+ * A quantized frozen weight: the stored buffers of NF4 + Double Quantization
+ * ([SD] section 3, parts 1 and 2).  All pointers are device memory owned by
+ * the caller; sizes come from qlora_nf4_sizes().
  *
  *   codes    uint8 [N*K/2]  two 4-bit code indices per byte, element 2j of the
  *                           row-major flattening in the HIGH nibble of byte j,
  *                           element 2j+1 in the low nibble.  Index i stands for
- *                           the i-th NF4 value in ascending order (0 = -1,
- *                           7 = 0, 15 = +1).
+ *                           the i-th value of the codebook in ascending order
+ *                           (NF4: 0 = -1, 7 = 0, 15 = +1).
  *   c1_codes uint8 [nb1]    one FP8 E4M3 code per block of 64 weights
  *                           (nb1 = N*K/64): the block's absmax, centred by mu
  *                           and scaled by its group's c2.
  *   c2       fp32  [nb2]    absmax of the centred constants per group of 256
  *                           blocks (nb2 = ceil(nb1/256)).
  *   mu       fp32  [1]      mean of all block absmax values.
+ *   codebook qlora_codebook the value set the codes index (0 = NF4).
+ *   c1       fp32  [nb1]    NULL for double quantization (the default).  When
+ *                           set, double quantization is off: the fp32 block
+ *                           absmax values are stored here and c1_codes, c2,
+ *                           mu are neither written nor read (they may be NULL)
+ *                           -- the single-level variant that trades 0.37 bits
+ *                           per weight for one fewer lookup per block.
  *
- * The rebuilt block constant is c1' = fp32(fp32(e4m3(c1_code) * c2) + mu) and
- * the dequantized weight is bf16_rn(fp32(q[code] * c1')).
+ * With double quantization the rebuilt block constant is
+ * c1' = fp32(fp32(e4m3(c1_code) * c2) + mu); without it c1' = c1.  The
+ * dequantized weight is bf16_rn(fp32(q[code] * c1')).  A zero-initialised
+ * codebook and c1 give NF4 with double quantization.
  */
 typedef struct {
     uint8_t* codes;
@@ -89,6 +105,9 @@ typedef struct {
     int64_t  K;
     int32_t  blocksize;   /* must be 64 */
     int32_t  blocksize2;  /* must be 256 */
+    int32_t  codebook;    /* qlora_codebook */
+    int32_t  reserved;    /* must be 0 */
+    float*   c1;          /* NULL: double quantization; else fp32 block constants [N*K/64] */
 } qlora_nf4_weight;
 
 /* Human-readable name of a status code (static storage; never NULL). */
@@ -121,6 +140,14 @@ qlora_status qlora_nf4_sizes(int64_t N, int64_t K, int32_t blocksize, int32_t bl
 qlora_status qlora_nf4_codebook(float values[16], float thresholds[15]);
 
 /*
+ * The same for any codebook: QLORA_CODEBOOK_NF4 gives qlora_nf4_codebook's
+ * values; QLORA_CODEBOOK_UNIFORM4 gives -1 + 2i/15 (i = 0..15) computed in
+ * double and rounded to float, with thresholds by the same rule.
+ * Errors: QLORA_ERR_INVALID_ARG for an unknown codebook.  Host only.
+ */
+qlora_status qlora_codebook_values(int32_t codebook, float values[16], float thresholds[15]);
+
+/*
  * NF4 + Double Quantization of a frozen bf16 weight ([SD] section 3, parts 1-2).
  *   W          device bf16 [N,K], read only; must be finite.
  *   out        host struct whose four device buffers are written; out->N, K,
@@ -132,7 +159,9 @@ qlora_status qlora_nf4_codebook(float values[16], float thresholds[15]);
  * sum over a fixed pairwise tree, rounded to fp32); per group of 256 blocks
  * c2 = max|fp32(c1 - mu)|; c1_code = E4M3 round-to-nearest-even of
  * fp32((c1 - mu) / c2) (0 when c2 == 0).  Deterministic and bit-exact.
- * A non-finite weight sets the device NONFINITE flag.
+ * out->codebook selects the code values (the nearest-value rule is the same);
+ * with out->c1 set, the fp32 c1 values are written there and the second level
+ * is skipped.  A non-finite weight sets the device NONFINITE flag.
  */
 qlora_status qlora_quantize_nf4_dq(const void* W, int64_t N, int64_t K,
                                    int32_t blocksize, int32_t blocksize2,

@@ -55,6 +55,12 @@ R7  LoRA: Y = X W_hat^T + s (X A^T) B^T with s = alpha / r, A[r,K], B[N,r].
 R8  The GEMM references are exact fp64 on the bit-exact W_hat and the bf16
     inputs; U = X A^T and dU = s dY B are never rounded.
 R9  The INT8 example rounds half away from zero ("四舍五入").
+R10 Quantizer variants ([SD] section 4 (2) compares NF4 with uniform INT4 by
+    E||W - W_hat||^2): the uniform 4-bit grid is 16 evenly spaced values on
+    [-1, 1] (linspace, fp64 then fp32), coded with the same absmax blocks and
+    nearest-value rule; "double quantization off" keeps the fp32 block absmax
+    c1 and dequantizes W_hat = bf16_RN(fp32(q[code] * c1)).  The error study
+    measures sum (W_hat - W)^2 / sum W^2 in fp64.
 """
 from __future__ import annotations
 
@@ -226,20 +232,22 @@ def block_absmax(v: np.ndarray, block: int) -> np.ndarray:
 # First-level NF4 quantization ([SD] Section 3 (1); readings R2-R4)
 # ---------------------------------------------------------------------------
 
-def nearest_code(x: np.ndarray, q: np.ndarray, chunk: int = 1 << 20) -> np.ndarray:
-    """argmin_i |x - q_i| over the codebook, ties to the lower index (reading R3).
+def nearest_code(x: np.ndarray, q: np.ndarray) -> np.ndarray:
+    """argmin_i |x - q_i| over the ascending codebook, ties to the lower index (reading R3).
 
-    Differences are taken in fp64, where x - q_i is exact for fp32 x and q_i of
-    the magnitudes that can compete for the minimum.
+    For a sorted codebook the argmin is the number of neighbour midpoints
+    m_j = (q_j + q_{j+1}) / 2 that lie strictly below x (x equal to a midpoint
+    is a tie and stays with the lower code).  The midpoints of two fp32 values
+    of close magnitude are exact in fp64, and so is every fp32 x, so the count
+    is exact for every x, denormals included (fp64 differences |x - q_i| are
+    not: for a denormal x both distances to a pair +-q round to the same value).
     """
-    x = np.asarray(x, dtype=np.float32).ravel()
+    x = np.asarray(x, dtype=np.float32).ravel().astype(np.float64)
     qd = np.asarray(q, dtype=np.float64)
-    out = np.empty(x.size, dtype=np.uint8)
-    for s in range(0, x.size, chunk):
-        xd = x[s:s + chunk].astype(np.float64)
-        dist = np.abs(xd[:, None] - qd[None, :])
-        out[s:s + chunk] = np.argmin(dist, axis=1)      # first minimum -> lower index
-    return out
+    assert np.all(np.diff(qd) > 0), "codebook must be ascending"
+    mids = (qd[:-1] + qd[1:]) / 2.0
+    assert np.array_equal(2.0 * mids - qd[:-1], qd[1:]), "midpoint not exact in fp64"
+    return np.searchsorted(mids, x, side="left").astype(np.uint8)
 
 
 def normalize_blocks(w: np.ndarray, c1: np.ndarray, block: int = BLOCKSIZE) -> np.ndarray:
@@ -357,6 +365,24 @@ def dequantize(codes_packed: np.ndarray, c1_codes: np.ndarray, c2: np.ndarray, m
     c1e = np.repeat(c1p, BLOCKSIZE)[:N * K]
     prod = (q[idx] * c1e).astype(np.float32)
     return f32_to_bf16_bits(prod).reshape(N, K)
+
+
+def dequantize_single(codes_packed: np.ndarray, c1: np.ndarray, N: int, K: int,
+                      q: np.ndarray | None = None) -> np.ndarray:
+    """Double quantization off (reading R10): W_hat = bf16_RN(fp32(q[code] * c1)) with the
+    fp32 block absmax c1 kept as is; uint16 bf16 bits [N,K]."""
+    q = nf4_codebook() if q is None else q
+    idx = unpack_nibbles(codes_packed)[:N * K]
+    c1e = np.repeat(np.asarray(c1, dtype=np.float32), BLOCKSIZE)[:N * K]
+    prod = (q[idx] * c1e).astype(np.float32)
+    return f32_to_bf16_bits(prod).reshape(N, K)
+
+
+def relative_sq_error(W_bits: np.ndarray, What_bits: np.ndarray) -> float:
+    """sum (W_hat - W)^2 / sum W^2 in fp64 over bf16 bit patterns ([SD] section 4 (2))."""
+    w = bf16_bits_to_f32(W_bits).astype(np.float64)
+    e = bf16_bits_to_f32(What_bits).astype(np.float64) - w
+    return float((e * e).sum() / (w * w).sum())
 
 
 def dequantize_rows(qw: dict, rows: np.ndarray, q: np.ndarray | None = None) -> np.ndarray:

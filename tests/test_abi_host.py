@@ -61,6 +61,22 @@ def test_library_thresholds_give_the_nearest_code(L):
     assert np.array_equal(by_threshold, o.nearest_code(x, q))
 
 
+def test_library_uniform4_codebook_and_thresholds(L):
+    v = (ctypes.c_float * 16)()
+    t = (ctypes.c_float * 15)()
+    assert L.qlora_codebook_values(1, v, t) == 0
+    q = np.array(v, dtype=np.float32)
+    assert np.array_equal(q.view(np.uint32), o.uniform4_codebook().view(np.uint32))
+    thr = np.array(t, dtype=np.float32)
+    g = np.random.default_rng(22)
+    x = np.concatenate([g.uniform(-1, 1, 200000).astype(np.float32), q, thr,
+                        np.nextafter(thr, np.float32(2)), np.nextafter(thr, np.float32(-2))])
+    assert np.array_equal((x[:, None] > thr[None, :]).sum(axis=1), o.nearest_code(x, q))
+    assert L.qlora_codebook_values(0, v, t) == 0
+    assert np.array_equal(np.array(v, dtype=np.float32).view(np.uint32), o.nf4_codebook().view(np.uint32))
+    assert L.qlora_codebook_values(7, v, t) == 1          # unknown codebook: QLORA_ERR_INVALID_ARG
+
+
 def test_sizes_match_oracle(L):
     for N, K in ((256, 256), (4096, 11008), (3, 320), (1, 64)):
         a, b, c, d = (ctypes.c_size_t() for _ in range(4))

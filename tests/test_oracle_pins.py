@@ -89,6 +89,47 @@ def test_nf4_beats_uniform_int4_on_gaussian_weights():
     assert _blockwise_mse(w, Q) < 0.85 * _blockwise_mse(w, o.uniform4_codebook())
 
 
+def test_uniform4_grid_is_even_with_end_points():
+    # reading R10: 16 evenly spaced values on [-1, 1]
+    u = o.uniform4_codebook().astype(np.float64)
+    assert u[0] == -1.0 and u[-1] == 1.0 and u.size == 16
+    assert np.all(np.diff(u) > 0)
+    assert np.allclose(np.diff(u), 2.0 / 15.0, rtol=0, atol=2 ** -22)
+    assert np.allclose(u, -u[::-1], rtol=0, atol=2 ** -23)
+    assert not np.any(u == 0.0)                       # the uniform grid has no exact zero, NF4 does
+
+
+def test_error_study_nf4_beats_uniform_and_double_quantization_is_cheap():
+    # [SD] section 4 (2): E||W - W_hat||^2 of NF4 is below that of a uniform 4-bit grid on
+    # normal weights; section 3 part 2: double quantization saves 0.37 bits/param at a small cost.
+    # Whole pipeline (absmax blocks, nearest code, bf16 rounding), relative squared error in fp64.
+    errs = {}
+    for dist in ("normal", "t5_outliers"):
+        bits = si.bf16_bits(si.custom_linear(256, 1024, 1, 1, seed=3, sigma=0.02, dist=dist)[0])
+        for name, q in (("nf4", Q), ("uniform4", o.uniform4_codebook())):
+            qw = o.quantize_nf4_dq(bits, q=q)
+            dq = o.dequantize(qw["codes"], qw["c1_codes"], qw["c2"], qw["mu"], qw["N"], qw["K"], q=q)
+            single = o.dequantize_single(qw["codes"], qw["c1"], qw["N"], qw["K"], q=q)
+            errs[dist, name, "dq"] = o.relative_sq_error(bits, dq)
+            errs[dist, name, "single"] = o.relative_sq_error(bits, single)
+    assert errs["normal", "nf4", "single"] < 0.9 * errs["normal", "uniform4", "single"]
+    assert errs["t5_outliers", "nf4", "single"] < 0.6 * errs["t5_outliers", "uniform4", "single"]
+    for dist in ("normal", "t5_outliers"):
+        ratio = errs[dist, "nf4", "dq"] / errs[dist, "nf4", "single"]
+        assert 0.99 < ratio < 1.02, (dist, ratio)
+
+
+def test_relative_error_closed_forms_and_single_level_consistency():
+    bits = si.bf16_bits(si.custom_linear(64, 128, 1, 1, seed=5)[0])
+    assert o.relative_sq_error(bits, bits) == 0.0
+    assert o.relative_sq_error(bits, np.zeros_like(bits)) == 1.0
+    # with c1 set to the rebuilt c1' the single-level dequant is the double-quantized one
+    qw = o.quantize_nf4_dq(bits)
+    c1p = o.dq_constants(qw["c1_codes"], qw["c2"], qw["mu"])
+    assert np.array_equal(o.dequantize_single(qw["codes"], c1p, 64, 128),
+                          o.dequantize(qw["codes"], qw["c1_codes"], qw["c2"], qw["mu"], 64, 128))
+
+
 def test_planted_codebook_mistakes_are_caught():
     # A codebook with the pages' literal symmetric midpoints (clipped ends) has no zero.
     lit = [0.5 * (o.phi_inv_stdlib(max(i / 16, 1e-3)) + o.phi_inv_stdlib(min((i + 1) / 16, 1 - 1e-3)))
@@ -172,6 +213,16 @@ def test_nearest_code_matches_exact_rational_argmin():
     got = o.nearest_code(x, Q)
     want = np.array([o.exact_nearest_code(v, Q) for v in x])
     assert np.array_equal(got, want)
+
+
+def test_nearest_code_exact_at_denormals_for_a_grid_without_zero():
+    # the uniform grid has a code pair +-q around 0: a denormal x > 0 is nearer to +q
+    U = o.uniform4_codebook()
+    tiny = np.array([1e-45, -1e-45, 1e-38, -1e-38, 1e-30, -1e-30, 0.0, -0.0], dtype=np.float32)
+    g = np.random.default_rng(4)
+    x = np.concatenate([tiny, g.uniform(-1, 1, 2000).astype(np.float32), U])
+    want = np.array([o.exact_nearest_code(v, U) for v in x])
+    assert np.array_equal(o.nearest_code(x, U), want)
 
 
 def test_nearest_code_tie_goes_to_lower_index():
