@@ -404,6 +404,45 @@ def dequant_rate(device, peaks, wl):
             "bytes_per_weight": round(PACKED_BYTES_PER_WEIGHT + 2.0, 6)}
 
 
+def quantizer_variants(device, peaks, wl):
+    """Quantizer variants on the workload's first weight (and on a normal one of the same shape):
+    relative squared error sum (W_hat - W)^2 / sum W^2 of each codebook with and without double
+    quantization (from the library's dequantized weight), and the quantize rate of each variant."""
+    import torch
+    import bit_nf4_quantized_23_b200 as q4
+    import synthetic_inputs as si
+    N, K = wl.linears[0]
+    weights = {wl.dist: si.weight(wl, 0).to(device),
+               "normal": si.normal_bf16((N, K), wl.sigma, 0, wl.name, "W0n").to(device)}
+    out = {"weight": f"W[{N},{K}]", "metric": "sum (W_hat - W)^2 / sum W^2 (fp64)"}
+    for dist, W in weights.items():
+        w64 = W.double()
+        den = float((w64 * w64).sum())
+        for codebook in ("nf4", "uniform4"):
+            for dq in (True, False):
+                w = q4.qlora_quantize_nf4_dq(W, codebook=codebook, double_quant=dq)
+                Wh = q4.qlora_dequantize(w).double()
+                key = f"{dist}/{codebook}/{'dq' if dq else 'single'}"
+                out[key] = {"rel_sq_error": float(((Wh - w64) ** 2).sum()) / den}
+                if dist == "normal":
+                    for _ in range(2):
+                        q4.qlora_quantize_nf4_dq(W, out=w)
+                    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    a.record()
+                    for _ in range(10):
+                        q4.qlora_quantize_nf4_dq(W, out=w)
+                    b.record()
+                    b.synchronize()
+                    ms = a.elapsed_time(b) / 10
+                    nbytes = (2.0 + (0.5 + 1 / 64 + 4 / 16384 if dq else 0.5 + 4 / 64)) * N * K
+                    out[key]["quantize_GB/s"] = round(nbytes / (ms * 1e-3) / 1e9, 1)
+        nf = out[f"{dist}/nf4/single"]["rel_sq_error"]
+        out[f"{dist}/nf4_over_uniform4"] = round(nf / out[f"{dist}/uniform4/single"]["rel_sq_error"], 4)
+    del weights
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args):
     import torch
     import bit_nf4_quantized_23_b200 as q4
@@ -509,12 +548,13 @@ def run_ours(args):
                         "frac_of_hbm": round(quant_bytes / (q_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3),
                         "ms_per_step": round(q_ms, 4), "bytes_per_weight": round(2.0 + PACKED_BYTES_PER_WEIGHT, 6),
                         "source": "live CUDA events over the timed steps (7 calls per step)"}}
-    decode = None
+    decode = variants = None
     if rank == 0 and not args.no_decode:
         del lins
         torch.cuda.empty_cache()
         hbm["dequantize"] = dequant_rate(device, peaks, wl)
         decode = decode_sweep(device, peaks)
+        variants = quantizer_variants(device, peaks, wl)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -536,7 +576,8 @@ def run_ours(args):
                        "step": "quantize all 7 weights + fwd + bwd of all 7 linears"
                                + (" + NCCL all-reduce of dA/dB" if world > 1 else "")},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
-            "clocks": clk, "kernels": breakdown, "hbm_bound_ops": hbm, "decode_small_m": decode}
+            "clocks": clk, "kernels": breakdown, "hbm_bound_ops": hbm, "decode_small_m": decode,
+            "quantizer_variants": variants}
     print(json.dumps(line), flush=True)
     return 0
 

@@ -1,0 +1,145 @@
+"""GPU parity of the quantizer variants against the CPU oracle.
+
+Variants ([SD] section 4 (2) compares NF4 with a uniform 4-bit grid; section 3
+part 2 adds double quantization on top of single-level absmax constants):
+the uniform grid with and without double quantization, and NF4 without it
+(NF4 with it is covered by test_gpu_parity.py).  Bit-exact: codes, constants
+and the dequantized weight.  Within tolerance: the forward and backward of the
+linear layer through every GEMM path (tensor-core large-M, small-M stream-K,
+CUDA-core for N % 8 != 0).  The error study is recomputed from the GPU's
+dequantized weights and must equal the oracle's figure exactly.
+"""
+import numpy as np
+import pytest
+import torch
+
+import bit_nf4_quantized_23_b200 as q4
+import synthetic_inputs as si
+from oracle import nf4_oracle as o
+from parity import assert_close, to_numpy_bits
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+VARIANTS = [("uniform4", True), ("nf4", False), ("uniform4", False)]
+CODEBOOK = {"nf4": o.nf4_codebook(), "uniform4": o.uniform4_codebook()}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib_built():
+    from bit_nf4_quantized_23_b200.build import build
+    build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    q4.qlora_read_device_errors(clear=True)
+    yield
+    assert q4.qlora_read_device_errors(clear=True) == 0
+
+
+def oracle_variant(W_cpu, codebook, dq):
+    """Oracle buffers and W_hat bits of a variant."""
+    q = CODEBOOK[codebook]
+    qw = o.quantize_nf4_dq(si.bf16_bits(W_cpu), q=q)
+    if dq:
+        Wh = o.dequantize(qw["codes"], qw["c1_codes"], qw["c2"], qw["mu"], qw["N"], qw["K"], q=q)
+    else:
+        Wh = o.dequantize_single(qw["codes"], qw["c1"], qw["N"], qw["K"], q=q)
+    return qw, Wh
+
+
+def check_buffers(w, qw, dq):
+    assert np.array_equal(w.codes.cpu().numpy(), qw["codes"])
+    if dq:
+        assert w.c1 is None
+        assert np.array_equal(w.c1_codes.cpu().numpy(), qw["c1_codes"])
+        assert np.array_equal(w.c2.cpu().numpy().view(np.uint32), qw["c2"].view(np.uint32))
+        assert w.mu.cpu().numpy().view(np.uint32)[0] == np.float32(qw["mu"]).view(np.uint32)
+    else:
+        assert w.c1_codes is None and w.c2 is None and w.mu is None
+        assert np.array_equal(w.c1.cpu().numpy().view(np.uint32), qw["c1"].view(np.uint32))
+
+
+@pytest.mark.parametrize("codebook,dq", VARIANTS)
+@pytest.mark.parametrize("N,K", [(256, 256), (3, 320), (17, 1024), (520, 1088)])
+def test_variant_quantize_and_dequantize_bit_exact(codebook, dq, N, K):
+    W = si.custom_linear(N, K, 1, 1, seed=N + K, dist="t5_outliers")[0]
+    w = q4.qlora_quantize_nf4_dq(W.to(DEV), codebook=codebook, double_quant=dq)
+    qw, Wh_ref = oracle_variant(W, codebook, dq)
+    check_buffers(w, qw, dq)
+    assert np.array_equal(to_numpy_bits(q4.qlora_dequantize(w)), Wh_ref)
+
+
+def test_variant_quantize_every_finite_bf16_value():
+    # every finite bf16 pattern once, in blocks with large and tiny absmax, on both grids
+    bits = np.arange(0, 1 << 16, dtype=np.uint32).astype(np.uint16)
+    finite = bits[(bits & 0x7F80) != 0x7F80]
+    pad = (-finite.size) % 1024
+    allb = np.concatenate([finite, np.zeros(pad, np.uint16)]).reshape(-1, 1024)
+    W = torch.from_numpy(allb.view(np.int16)).view(torch.bfloat16)
+    for codebook, dq in VARIANTS:
+        w = q4.qlora_quantize_nf4_dq(W.to(DEV), codebook=codebook, double_quant=dq)
+        qw, Wh_ref = oracle_variant(W, codebook, dq)
+        check_buffers(w, qw, dq)
+        assert np.array_equal(to_numpy_bits(q4.qlora_dequantize(w)), Wh_ref)
+
+
+def run_variant_linear(codebook, dq, M, N, K, r, y_dtype=torch.bfloat16):
+    W, X, A, B, dY = si.custom_linear(N, K, M, r, seed=2 * M + N + K + r)
+    alpha = 2.0 * r
+    w = q4.qlora_quantize_nf4_dq(W.to(DEV), codebook=codebook, double_quant=dq)
+    Xd, Ad, Bd, dYd = (t.to(DEV) for t in (X, A, B, dY))
+    Y, U = q4.qlora_linear_fwd(w, Xd, Ad, Bd, r, alpha, y_dtype=y_dtype)
+    dX, dA, dB = q4.qlora_linear_bwd(w, Xd, dYd, Ad, Bd, r, alpha, U_saved=U, dx_dtype=y_dtype)
+    torch.cuda.synchronize()
+    _, Wh = oracle_variant(W, codebook, dq)
+    bX, bA, bB, bdY = (si.bf16_bits(t) for t in (X, A, B, dY))
+    Yr, Ur = o.linear_forward(bX, Wh, bA, bB, alpha, r)
+    g = o.linear_backward(bX, bdY, Wh, bA, bB, alpha, r)
+    assert_close(Y, Yr, "Y")
+    assert_close(U, Ur, "U")
+    assert_close(dX, g["dX"], "dX")
+    assert_close(dA, g["dA"], "dA")
+    assert_close(dB, g["dB"], "dB")
+
+
+@pytest.mark.parametrize("codebook,dq", VARIANTS)
+@pytest.mark.parametrize("M,N,K,r", [(5, 100, 128, 3), (16, 1000, 640, 16), (130, 96, 640, 64),
+                                     (300, 520, 1088, 96), (33, 130, 256, 8)])
+def test_variant_linear_fwd_bwd(codebook, dq, M, N, K, r):
+    run_variant_linear(codebook, dq, M, N, K, r)
+
+
+def test_variant_linear_fp32_outputs():
+    run_variant_linear("uniform4", False, 64, 256, 512, 16, y_dtype=torch.float32)
+
+
+def test_error_study_from_gpu_dequant_equals_oracle():
+    # relative squared error sum (W_hat - W)^2 / sum W^2 of each variant, from the GPU's W_hat
+    W = si.custom_linear(256, 1024, 1, 1, seed=3, sigma=0.02, dist="normal")[0]
+    bits = si.bf16_bits(W)
+    errs = {}
+    for codebook, dq in VARIANTS + [("nf4", True)]:
+        w = q4.qlora_quantize_nf4_dq(W.to(DEV), codebook=codebook, double_quant=dq)
+        gpu = o.relative_sq_error(bits, to_numpy_bits(q4.qlora_dequantize(w)))
+        ref = o.relative_sq_error(bits, oracle_variant(W, codebook, dq)[1])
+        assert gpu == ref
+        errs[codebook, dq] = gpu
+    assert errs["nf4", False] < 0.9 * errs["uniform4", False]
+
+
+def test_variant_argument_errors():
+    W = si.custom_linear(64, 128, 1, 1, seed=1)[0].to(DEV)
+    w = q4.NF4Weight.empty(64, 128, DEV, "nf4", double_quant=False)
+    ws = w.c_struct()
+    ws.codebook = 5
+    from bit_nf4_quantized_23_b200 import _lib
+    import ctypes
+    sizes = q4.qlora_nf4_sizes(64, 128)
+    scratch = torch.empty(sizes["workspace"], dtype=torch.uint8, device=DEV)
+    st = _lib.lib().qlora_quantize_nf4_dq(ctypes.c_void_p(W.data_ptr()), 64, 128, 64, 256, ctypes.byref(ws),
+                                         ctypes.c_void_p(scratch.data_ptr()), scratch.numel(), None)
+    assert st == 1                                    # QLORA_ERR_INVALID_ARG, nothing launched
+    ws.codebook = 0
+    ws.reserved = 3
+    st = _lib.lib().qlora_quantize_nf4_dq(ctypes.c_void_p(W.data_ptr()), 64, 128, 64, 256, ctypes.byref(ws),
+                                         ctypes.c_void_p(scratch.data_ptr()), scratch.numel(), None)
+    assert st == 1
