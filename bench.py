@@ -443,6 +443,41 @@ def quantizer_variants(device, peaks, wl):
     return out
 
 
+def merge_requantize(device, peaks, wl):
+    """Merge the adapters into the workload's first weight, requantize, and report the merge rate
+    and the error the requantization adds against the exact merged weight W + s B A (fp64)."""
+    import torch
+    import bit_nf4_quantized_23_b200 as q4
+    import synthetic_inputs as si
+    N, K = wl.linears[0]
+    W = si.weight(wl, 0).to(device)
+    A, B = (t.to(device) for t in si.lora(wl, 0))
+    w = q4.qlora_quantize_nf4_dq(W)
+    Wm = q4.qlora_merge_lora(w, A, B, wl.r, wl.alpha)
+    for _ in range(3):
+        q4.qlora_merge_lora(w, A, B, wl.r, wl.alpha, out=Wm)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(10):
+        q4.qlora_merge_lora(w, A, B, wl.r, wl.alpha, out=Wm)
+    b.record()
+    b.synchronize()
+    ms = a.elapsed_time(b) / 10
+    w2 = q4.qlora_quantize_nf4_dq(Wm)
+    s = wl.alpha / wl.r
+    exact = W.double() + s * (B.double() @ A.double())
+    rel = lambda X, ref: float(((X.double() - ref) ** 2).sum() / (ref ** 2).sum())
+    out = {"weight": f"W[{N},{K}]", "r": wl.r, "merge_us": round(ms * 1e3, 1),
+           "merge_GB/s": round((PACKED_BYTES_PER_WEIGHT + 2.0) * N * K / (ms * 1e-3) / 1e9, 1),
+           "quantize_error": rel(q4.qlora_dequantize(w), W.double()),
+           "merged_rounding_error": rel(Wm, exact),
+           "requantized_merged_error": rel(q4.qlora_dequantize(w2), exact),
+           "metric": "sum (X - ref)^2 / sum ref^2 (fp64); ref = W for the first, W + s B A after"}
+    del W, A, B, w, Wm, w2, exact
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args):
     import torch
     import bit_nf4_quantized_23_b200 as q4
@@ -548,13 +583,14 @@ def run_ours(args):
                         "frac_of_hbm": round(quant_bytes / (q_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3),
                         "ms_per_step": round(q_ms, 4), "bytes_per_weight": round(2.0 + PACKED_BYTES_PER_WEIGHT, 6),
                         "source": "live CUDA events over the timed steps (7 calls per step)"}}
-    decode = variants = None
+    decode = variants = merge = None
     if rank == 0 and not args.no_decode:
         del lins
         torch.cuda.empty_cache()
         hbm["dequantize"] = dequant_rate(device, peaks, wl)
         decode = decode_sweep(device, peaks)
         variants = quantizer_variants(device, peaks, wl)
+        merge = merge_requantize(device, peaks, wl)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -577,7 +613,7 @@ def run_ours(args):
                                + (" + NCCL all-reduce of dA/dB" if world > 1 else "")},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
             "clocks": clk, "kernels": breakdown, "hbm_bound_ops": hbm, "decode_small_m": decode,
-            "quantizer_variants": variants}
+            "quantizer_variants": variants, "merge_requantize": merge}
     print(json.dumps(line), flush=True)
     return 0
 

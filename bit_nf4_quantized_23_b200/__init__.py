@@ -21,7 +21,7 @@ __all__ = [
     "NF4Weight", "QloraError", "CODEBOOKS", "qlora_nf4_sizes", "qlora_nf4_codebook", "qlora_codebook_values",
     "qlora_quantize_nf4_dq",
     "qlora_quantize_nf4_dq_noalloc",
-    "qlora_dequantize", "qlora_linear_workspace_size", "qlora_linear_fwd", "qlora_linear_bwd",
+    "qlora_dequantize", "qlora_merge_lora", "qlora_linear_workspace_size", "qlora_linear_fwd", "qlora_linear_bwd",
     "qlora_read_device_errors", "qlora_launch_count", "qlora_timing_enable", "qlora_timing_read",
 ]
 
@@ -154,6 +154,21 @@ def qlora_dequantize(w: NF4Weight, out: torch.Tensor | None = None, stream=None)
     _need(out, torch.bfloat16, "out", (w.N, w.K))
     ws = w.c_struct()
     check(lib().qlora_dequantize(byref(ws), _ptr(out), _stream(stream)), "qlora_dequantize")
+    return out
+
+
+def qlora_merge_lora(w: NF4Weight, A: torch.Tensor, B: torch.Tensor, r: int, alpha: float,
+                     out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """W_merged = bf16(W_hat + (alpha / r) B A) for inference; requantize it with
+    qlora_quantize_nf4_dq to serve the merged model in 4 bits."""
+    _need(A, torch.bfloat16, "A", (r, w.K))
+    _need(B, torch.bfloat16, "B", (w.N, r))
+    if out is None:
+        out = torch.empty(w.N, w.K, dtype=torch.bfloat16, device=w.codes.device)
+    _need(out, torch.bfloat16, "out", (w.N, w.K))
+    ws = w.c_struct()
+    check(lib().qlora_merge_lora(byref(ws), _ptr(A), _ptr(B), r, float(alpha), _ptr(out), _stream(stream)),
+          "qlora_merge_lora")
     return out
 
 

@@ -25,6 +25,8 @@ qlora_status launch_split_hi_lo(const float* V, int64_t M, int r, int R, float s
 qlora_status launch_dup_cols(const void* B, int64_t N, int r, int R, void* B2, cudaStream_t s);
 qlora_status launch_dup_rows(const void* A, int r, int R, int64_t K, void* A2, cudaStream_t s);
 qlora_status launch_transpose_pad(const void* B, int64_t N, int r, int R, void* Bt, cudaStream_t s);
+qlora_status launch_merge(const qlora_nf4_weight* w, const void* A, const void* B, int32_t r, float scale,
+                          void* W_out, cudaStream_t stream);
 qlora_status launch_reduce_rows(const float* partial, int splits, int64_t rows, int r, int R, float scale_out,
                                 float* out, float scale_v2, void* V2, cudaStream_t s);
 qlora_status launch_reduce_transposed(const float* partial, int splits, int64_t rows, int r, int R, float* out,
@@ -206,6 +208,16 @@ qlora_status qlora_quantize_nf4_dq(const void* W, int64_t N, int64_t K, int32_t 
     if (!aligned16(workspace)) return QLORA_ERR_ALIGN;
     TimerScope t(QLORA_TIMER_QUANTIZE, static_cast<cudaStream_t>(stream));
     return launch_quantize(W, N, K, out, workspace, static_cast<cudaStream_t>(stream));
+}
+
+qlora_status qlora_merge_lora(const qlora_nf4_weight* w, const void* A, const void* B, int32_t r, float alpha,
+                              void* W_out, void* stream) {
+    QLORA_TRY(check_weight(w));
+    QLORA_TRY(check_lora(1, r, alpha));
+    QLORA_TRY(check_dev(A));
+    QLORA_TRY(check_dev(B));
+    QLORA_TRY(check_dev(W_out));
+    return launch_merge(w, A, B, r, alpha / (float)r, W_out, static_cast<cudaStream_t>(stream));
 }
 
 qlora_status qlora_dequantize(const qlora_nf4_weight* w, void* W_out, void* stream) {

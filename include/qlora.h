@@ -18,6 +18,9 @@
  *   [QR]  ainexis.cn, walkthrough of "QLoRA: Efficient Finetuning of Quantized
  *         LLMs", section 4.4: backpropagation passes through the frozen 4-bit
  *         weight into the adapters.
+ *   [Q103] agentalpha.top, "Q103: What is QLoRA, and how does it differ from
+ *         LoRA", follow-up 1: after fine-tuning, merge the LoRA weights and
+ *         dequantize for fast inference.
  *
  * Conventions for every entry point
  * ---------------------------------
@@ -234,6 +237,23 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const void* X, const vo
                               const float* U_saved, void* dX, int32_t dx_dtype,
                               float* dA, float* dB,
                               void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Merge trained adapters into the frozen weight for inference ([Q103]
+ * follow-up 1; [QP] section 5: merging and requantizing can add error): with
+ * s = alpha / r,
+ *   W_out[n,k] = bf16_rn(fp32(W_hat[n,k] + sum_j fp32(s * B[n,j]) * A[j,k])),
+ * the rank-r sum taken in ascending j with fp32 fused multiply-adds and W_hat
+ * the dequantized weight (any codebook, with or without double quantization).
+ * Requantize W_out with qlora_quantize_nf4_dq to serve the merged model in 4 bits.
+ *   w      quantized weight (read only);
+ *   A      device bf16 [r,K];  B  device bf16 [N,r];
+ *   W_out  device bf16 [N,K], written.
+ * Errors: QLORA_ERR_INVALID_ARG (null pointer, r outside 1..256, alpha not
+ * finite), QLORA_ERR_ALIGN, and the weight checks of qlora_dequantize.
+ */
+qlora_status qlora_merge_lora(const qlora_nf4_weight* w, const void* A, const void* B, int32_t r, float alpha,
+                              void* W_out, void* stream);
 
 /*
  * Device error flags raised since the last clear (bit 0: a bounded wait timed

@@ -442,6 +442,27 @@ def _f64(bits_or_array) -> np.ndarray:
     return a.astype(np.float64)
 
 
+def f64_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round fp64 values to bf16 directly (nearest, ties to even; no fp32 step, which could
+    round twice).  bf16 keeps 8 significant bits down to 2^-126 and a fixed step of 2^-133
+    below; values that round past the largest finite bf16 become infinity."""
+    x = np.asarray(x, dtype=np.float64)
+    _, e = np.frexp(x)                                   # |x| = m 2^e, 0.5 <= m < 1
+    step = np.ldexp(1.0, np.maximum(e, -125) - 8)        # spacing of bf16 values around x
+    r = np.rint(x / step) * step                         # exact scaling; rint ties to even
+    with np.errstate(over="ignore"):
+        r32 = r.astype(np.float32)                       # exact: <= 8 significant bits (or overflow)
+    return f32_to_bf16_bits(r32)
+
+
+def merge_lora(W_hat_bits, A_bits, B_bits, alpha: float, r: int) -> np.ndarray:
+    """Merged weight for inference ([Q103] follow-up 1; [QP] section 5):
+    W_merged = bf16_RN(W_hat + s B A), s = alpha / r, the rank-r product and the sum in fp64
+    (products of bf16 values are exact; one rounding at the end).  uint16 bf16 bits [N,K]."""
+    s = lora_scale(alpha, r)
+    return f64_to_bf16_bits(_f64(W_hat_bits) + s * (_f64(B_bits) @ _f64(A_bits)))
+
+
 def lora_scale(alpha: float, r: int) -> float:
     """s = alpha / r ([Q103] follow-up 3 names r and alpha)."""
     return float(alpha) / float(r)

@@ -143,3 +143,41 @@ def test_variant_argument_errors():
     st = _lib.lib().qlora_quantize_nf4_dq(ctypes.c_void_p(W.data_ptr()), 64, 128, 64, 256, ctypes.byref(ws),
                                          ctypes.c_void_p(scratch.data_ptr()), scratch.numel(), None)
     assert st == 1
+
+
+# ------------------------------------------------------------------ merge and requantize
+
+@pytest.mark.parametrize("codebook,dq", [("nf4", True), ("uniform4", False)])
+@pytest.mark.parametrize("N,K,r", [(256, 256, 8), (520, 1088, 96), (3, 320, 3), (130, 640, 256)])
+def test_merge_lora_matches_oracle_and_requantizes_exactly(codebook, dq, N, K, r):
+    # The GPU sums the rank-r term in fp32 and rounds once to bf16; the oracle sums in fp64.
+    # The two can differ by one bf16 step where the fp32 sum lands across a rounding
+    # boundary (rare); the requantization of the GPU's merged weight is bit-exact.
+    W, X, A, B, dY = si.custom_linear(N, K, 1, r, seed=N + K + r)
+    B = (B.float() * 30.0).to(torch.bfloat16)          # make the update visible next to W
+    alpha = 2.0 * r
+    w = q4.qlora_quantize_nf4_dq(W.to(DEV), codebook=codebook, double_quant=dq)
+    Wm = q4.qlora_merge_lora(w, A.to(DEV), B.to(DEV), r, alpha)
+    _, Wh = oracle_variant(W, codebook, dq)
+    ref = o.merge_lora(Wh, si.bf16_bits(A), si.bf16_bits(B), alpha, r)
+    got = to_numpy_bits(Wm)
+    # bound: one bf16 step of the result plus the fp32 accumulation error of r terms
+    # (r * 2^-23 * sum |s B A| covers r roundings or truncations); the second term only
+    # matters where the update cancels W_hat and the result is far below its terms
+    gv = o.bf16_bits_to_f32(got).astype(np.float64)
+    rv = o.bf16_bits_to_f32(ref).astype(np.float64)
+    sumabs = (alpha / r) * (np.abs(o._f64(si.bf16_bits(B))) @ np.abs(o._f64(si.bf16_bits(A))))
+    step = np.ldexp(1.0, np.maximum(np.frexp(rv)[1], -125) - 8)
+    assert np.all(np.abs(gv - rv) <= step + r * 2.0 ** -23 * sumabs), "beyond one step + accumulation bound"
+    assert np.count_nonzero(got != ref) <= max(2, got.size // 500)
+    # requantize the merged weight: bit-exact against the oracle on the same bits
+    w2 = q4.qlora_quantize_nf4_dq(Wm, codebook=codebook, double_quant=dq)
+    qw2 = o.quantize_nf4_dq(got, q=CODEBOOK[codebook])
+    check_buffers(w2, qw2, dq)
+
+
+def test_merge_with_zero_B_is_the_dequantized_weight():
+    W, X, A, B, dY = si.custom_linear(64, 512, 1, 16, seed=12)
+    w = q4.qlora_quantize_nf4_dq(W.to(DEV))
+    Wm = q4.qlora_merge_lora(w, A.to(DEV), torch.zeros_like(B).to(DEV), 16, 32.0)
+    assert torch.equal(Wm, q4.qlora_dequantize(w))

@@ -511,3 +511,50 @@ def test_row_and_column_samplers_match_full_quantize():
     Wh = o.dequantize(full["codes"], full["c1_codes"], full["c2"], full["mu"], 24, 512)
     cols = np.array([0, 1, 63, 64, 511])
     assert np.array_equal(o.dequantize_cols(full, cols), Wh[:, cols])
+
+
+# ---------------------------------------------------------------- merge and requantize
+
+def _nearest_bf16_exact(v: float) -> int:
+    """Brute force: the bf16 pattern nearest to v (exact rationals; ties to the even pattern)."""
+    from fractions import Fraction
+    fv = Fraction(v)
+    b0 = int(o.f32_to_bf16_bits(np.array([v], np.float32))[0])   # a candidate within one step
+    best = None
+    for b in (b0 - 1, b0, b0 + 1):
+        if b & 0x7F80 == 0x7F80:
+            continue
+        val = Fraction(float(o.bf16_bits_to_f32(np.array([b], np.uint16))[0]))
+        key = (abs(val - fv), b & 1)
+        if best is None or key < best[0]:
+            best = (key, b)
+    return best[1]
+
+
+def test_f64_to_bf16_rounds_once():
+    g = np.random.default_rng(8)
+    x = np.concatenate([g.normal(0, 0.02, 3000), g.normal(0, 1e-38, 200), [0.0, -0.0, 1.0, -3.5]])
+    # values just above a bf16 midpoint by less than half an fp32 ulp: fp32 first would land on the
+    # midpoint and round to even (down); the direct rounding must go up
+    mids = [1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8]
+    x = np.concatenate([x, [m + 2.0 ** -30 for m in mids], [m - 2.0 ** -30 for m in mids], mids])
+    got = o.f64_to_bf16_bits(x)
+    want = np.array([_nearest_bf16_exact(float(v)) for v in x], dtype=np.uint16)
+    assert np.array_equal(got, want)
+    assert o.f64_to_bf16_bits(np.array([1.0 + 2.0 ** -8 + 2.0 ** -30]))[0] == 0x3F81
+
+
+def test_merge_definition_and_degenerate_cases():
+    W, X, A, B, dY = si.custom_linear(7, 128, 1, 3, seed=9)
+    qw = o.quantize_nf4_dq(si.bf16_bits(W))
+    Wh = o.dequantize(qw["codes"], qw["c1_codes"], qw["c2"], qw["mu"], 7, 128)
+    bA, bB = si.bf16_bits(A), si.bf16_bits(B)
+    # B = 0: the merged weight is the dequantized weight, bit for bit
+    assert np.array_equal(o.merge_lora(Wh, bA, np.zeros_like(bB), 6.0, 3), Wh)
+    # brute-force loops over the definition
+    Whf, Af, Bf = o._f64(Wh), o._f64(bA), o._f64(bB)
+    brute = np.zeros((7, 128))
+    for n in range(7):
+        for k in range(128):
+            brute[n, k] = Whf[n, k] + 2.0 * sum(Bf[n, j] * Af[j, k] for j in range(3))
+    assert np.array_equal(o.merge_lora(Wh, bA, bB, 6.0, 3), o.f64_to_bf16_bits(brute))
