@@ -373,6 +373,32 @@ def decode_sweep(device, peaks):
                 "kernel_us": round(kms * 1e3, 2), "kernel_GB/s": round(wbytes / (kms * 1e-3) / 1e9, 1),
                 "kernel_frac_of_hbm": round(wbytes / (kms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3),
                 "kernel_frac_of_alu_roofline": round(wbytes / (kms * 1e-3) / 1e9 / alu_gbs, 3)}
+        if i == len(wl.linears) - 1:
+            # one base, many adapters: 16 tokens, each on its own adapter, same weight copies
+            M, n_ad = 16, 16
+            X = si.activations(wl, K, M).to(device)
+            A_all = torch.stack([si.lora(wl, i)[0]] * n_ad).to(device)
+            B_all = torch.stack([si.lora(wl, i)[1]] * n_ad).to(device)
+            idx = torch.arange(n_ad, dtype=torch.int32, device=device)
+            Y = torch.empty(M, N, dtype=torch.bfloat16, device=device)
+            lws = torch.empty(max(16, q4.qlora_linear_workspace_size(M, N, K, wl.r)), dtype=torch.uint8,
+                              device=device)
+            call = lambda j: q4.qlora_linear_fwd_multi(ws[j % copies], X, A_all, B_all, idx, wl.r, wl.alpha,
+                                                       out=Y, workspace=lws)
+            for j in range(3):
+                call(j)
+            reps = 8 * copies
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            for j in range(reps):
+                call(j)
+            b.record()
+            b.synchronize()
+            ms = a.elapsed_time(b) / reps
+            out[f"W[{N},{K}] M=16, 16 adapters"] = {
+                "call_us": round(ms * 1e3, 2), "call_GB/s": round(wbytes / (ms * 1e-3) / 1e9, 1),
+                "note": "qlora_linear_fwd_multi: every token on its own adapter over one base"}
         del ws
         torch.cuda.empty_cache()
     return out

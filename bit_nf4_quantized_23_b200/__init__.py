@@ -21,7 +21,7 @@ __all__ = [
     "NF4Weight", "QloraError", "CODEBOOKS", "qlora_nf4_sizes", "qlora_nf4_codebook", "qlora_codebook_values",
     "qlora_quantize_nf4_dq",
     "qlora_quantize_nf4_dq_noalloc",
-    "qlora_dequantize", "qlora_merge_lora", "qlora_linear_workspace_size", "qlora_linear_fwd", "qlora_linear_bwd",
+    "qlora_dequantize", "qlora_merge_lora", "qlora_linear_workspace_size", "qlora_linear_fwd", "qlora_linear_fwd_multi", "qlora_linear_bwd",
     "qlora_read_device_errors", "qlora_launch_count", "qlora_timing_enable", "qlora_timing_read",
 ]
 
@@ -207,6 +207,32 @@ def qlora_linear_fwd(w: NF4Weight, X: torch.Tensor, A: torch.Tensor, B: torch.Te
                                  _dtype_code(y_dtype), _ptr(U_out), _ptr(workspace), workspace.numel(),
                                  _stream(stream)), "qlora_linear_fwd")
     return out, U_out
+
+
+def qlora_linear_fwd_multi(w: NF4Weight, X: torch.Tensor, A_all: torch.Tensor, B_all: torch.Tensor,
+                           adapter_idx: torch.Tensor, r: int, alpha: float, y_dtype=torch.bfloat16,
+                           save_U: bool = False, out: torch.Tensor | None = None,
+                           workspace: torch.Tensor | None = None, stream=None):
+    """One base, many adapters (M <= 16 tokens): Y[m] = X[m] W_hat^T + (alpha/r) (X[m] A_a^T) B_a^T
+    with a = adapter_idx[m] (-1: base only).  A_all [n, r, K], B_all [n, N, r] bf16; adapter_idx
+    int32 [M] on the device.  Returns (Y, U or None)."""
+    M = X.shape[0]
+    n_ad = A_all.shape[0]
+    _need(X, torch.bfloat16, "X", (M, w.K))
+    _need(A_all, torch.bfloat16, "A_all", (n_ad, r, w.K))
+    _need(B_all, torch.bfloat16, "B_all", (n_ad, w.N, r))
+    _need(adapter_idx, torch.int32, "adapter_idx", (M,))
+    if out is None:
+        out = torch.empty(M, w.N, dtype=y_dtype, device=X.device)
+    _need(out, y_dtype, "Y", (M, w.N))
+    U = torch.empty(M, r, dtype=torch.float32, device=X.device) if save_U else None
+    workspace = _workspace(M, w.N, w.K, r, X.device, workspace)
+    ws = w.c_struct()
+    check(lib().qlora_linear_fwd_multi(byref(ws), _ptr(X), M, _ptr(A_all), _ptr(B_all), n_ad, _ptr(adapter_idx),
+                                       r, c_float(alpha), _ptr(out), _dtype_code(y_dtype), _ptr(U),
+                                       _ptr(workspace), workspace.numel(), _stream(stream)),
+          "qlora_linear_fwd_multi")
+    return out, U
 
 
 def qlora_linear_bwd(w: NF4Weight, X: torch.Tensor, dY: torch.Tensor, A: torch.Tensor, B: torch.Tensor,

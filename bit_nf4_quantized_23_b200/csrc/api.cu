@@ -281,6 +281,36 @@ qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const void* X, int64_t 
     return launch_tc_gemm_nf4(a, false, s);
 }
 
+qlora_status qlora_linear_fwd_multi(const qlora_nf4_weight* w, const void* X, int64_t M, const void* A_all,
+                                    const void* B_all, int32_t n_adapters, const int32_t* adapter_idx, int32_t r,
+                                    float alpha, void* Y, int32_t y_dtype, float* U_save, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+    QLORA_TRY(check_weight(w));
+    QLORA_TRY(check_lora(M, r, alpha));
+    if (M > kDecodeMaxM) return QLORA_ERR_SHAPE;
+    if (n_adapters < 1) return QLORA_ERR_INVALID_ARG;
+    QLORA_TRY(check_dev(X));
+    QLORA_TRY(check_dev(A_all));
+    QLORA_TRY(check_dev(B_all));
+    QLORA_TRY(check_dev(Y));
+    if (!adapter_idx) return QLORA_ERR_INVALID_ARG;
+    if (y_dtype != QLORA_DTYPE_BF16 && y_dtype != QLORA_DTYPE_F32) return QLORA_ERR_INVALID_ARG;
+    if (U_save && !aligned16(U_save)) return QLORA_ERR_ALIGN;
+    const LinearWs lw = linear_ws(M, w->N, w->K, r);
+    if (!workspace || workspace_bytes < lw.total) return QLORA_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return QLORA_ERR_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    char* ws = static_cast<char*>(workspace);
+    DecodeArgs d{};
+    d.w = w; d.X = X; d.A = A_all; d.B = B_all; d.r = r; d.scale = alpha / (float)r; d.M = M; d.out = Y;
+    d.out_f32 = (y_dtype == QLORA_DTYPE_F32);
+    d.U = U_save ? U_save : reinterpret_cast<float*>(ws + lw.u_off);
+    d.partial = reinterpret_cast<float*>(ws + lw.part_off);
+    d.aidx = adapter_idx; d.n_adapters = n_adapters;
+    TimerScope t(QLORA_TIMER_DECODE, s);
+    return launch_tc_decode(d, s);
+}
+
 qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const void* X, const void* dY, int64_t M,
                               const void* A, const void* B, int32_t r, float alpha,
                               const float* U_saved, void* dX, int32_t dx_dtype,

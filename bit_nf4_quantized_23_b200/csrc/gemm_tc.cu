@@ -696,13 +696,25 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, const __grid_constant
     if (threadIdx.x == 0) grid_dependency_wait();
 }
 
-// U[m, j] = sum_k X[m, k] A[j, k] in fp32 (one CTA per (j, m); fixed reduction order).
+// U[m, j] = sum_k X[m, k] A[j, k] in fp32 (one CTA per (j, m); fixed reduction order).  With
+// per-token adapters (aidx), token m uses A[aidx[m]] and a token without one (-1) gets U = 0.
 __global__ void __launch_bounds__(256)
-decode_lora_u(const uint4* __restrict__ X, const uint4* __restrict__ A, int64_t K8, int r, float* __restrict__ U) {
+decode_lora_u(const uint4* __restrict__ X, const uint4* __restrict__ A, int64_t K8, int r, float* __restrict__ U,
+              const int32_t* __restrict__ aidx, int n_adapters, uint32_t* err) {
     allow_dependents();                                       // the dequant GEMM does not read U
     const int j = blockIdx.x, m = blockIdx.y;
+    int64_t arow = j;
+    if (aidx) {
+        const int a = aidx[m];
+        if (a < 0 || a >= n_adapters) {                       // no adapter (or an index out of range)
+            if (a >= n_adapters && threadIdx.x == 0) atomicOr(err, ERR_FLAG_BOUNDS);
+            if (threadIdx.x == 0) U[(int64_t)m * r + j] = 0.f;
+            return;
+        }
+        arow = (int64_t)a * r + j;
+    }
     const uint4* xr = X + (int64_t)m * K8;
-    const uint4* ar = A + (int64_t)j * K8;
+    const uint4* ar = A + arow * K8;
     float acc = 0.f;
     for (int64_t c0 = threadIdx.x; c0 < K8; c0 += 4 * 256) {
         uint4 xv[4], av[4];
@@ -740,12 +752,18 @@ decode_lora_u(const uint4* __restrict__ X, const uint4* __restrict__ A, int64_t 
 // every group of loads is issued back to back (the kernel is latency-bound, not bandwidth-bound).
 __global__ void __launch_bounds__(128)
 decode_fixup(const float* __restrict__ partial, int64_t units, int64_t G, int S, int64_t M, int64_t N,
-             const float* __restrict__ U, const uint16_t* __restrict__ B, int r, float scale, void* out, int out_f32) {
+             const float* __restrict__ U, const uint16_t* __restrict__ B, int r, float scale, void* out, int out_f32,
+             const int32_t* __restrict__ aidx, int n_adapters) {
     extern __shared__ float us[];                             // us[j * 16 + m] = U[m, j]
+    __shared__ int32_t tok_adapter[16];
     grid_dependency_wait();                                   // partial tiles and U are complete
     for (int i = threadIdx.x; i < r * 16; i += 128) {
         const int j = i >> 4, m = i & 15;
         us[i] = m < M ? U[(int64_t)m * r + j] : 0.f;
+    }
+    if (threadIdx.x < 16) {
+        const int a = (aidx && threadIdx.x < M) ? aidx[threadIdx.x] : 0;
+        tok_adapter[threadIdx.x] = (a >= 0 && a < n_adapters) ? a : -1;
     }
     __syncthreads();
     const int64_t tile = blockIdx.x;
@@ -772,8 +790,26 @@ decode_fixup(const float* __restrict__ partial, int64_t units, int64_t G, int S,
     float lora[16];
 #pragma unroll
     for (int m = 0; m < 16; ++m) lora[m] = 0.f;
+    if (aidx) {
+        // per-token adapters: lora[m] = sum_j U[m, j] B[a(m)][n, j] (ascending j), 0 without one
+        for (int m = 0; m < M; ++m) {
+            const int a = tok_adapter[m];
+            if (a < 0) continue;
+            const uint16_t* br = B + ((int64_t)a * N + n) * r;
+            float d = 0.f;
+            for (int j0 = 0; j0 < r; j0 += 8) {
+                float bv[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) bv[q] = j0 + q < r ? bf16_bits_to_f32(br[j0 + q]) : 0.f;
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    if (j0 + q < r) d = __fmaf_rn(us[(j0 + q) * 16 + m], bv[q], d);
+            }
+            lora[m] = d;
+        }
+    }
     const uint16_t* brow = B + n * r;
-    for (int j0 = 0; j0 < r; j0 += 8) {
+    for (int j0 = 0; j0 < (aidx ? 0 : r); j0 += 8) {
         float bv[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) bv[q] = j0 + q < r ? bf16_bits_to_f32(brow[j0 + q]) : 0.f;
@@ -895,7 +931,7 @@ qlora_status launch_tc_decode(const DecodeArgs& a, cudaStream_t stream) {
         configured = true;
     }
     decode_lora_u<<<dim3((unsigned)a.r, (unsigned)a.M), 256, 0, stream>>>(
-        static_cast<const uint4*>(a.X), static_cast<const uint4*>(a.A), K / 8, a.r, a.U);
+        static_cast<const uint4*>(a.X), static_cast<const uint4*>(a.A), K / 8, a.r, a.U, a.aidx, a.n_adapters, p.err);
     QLORA_CHECK_LAUNCH();
     // the three kernels are chained with programmatic dependent launch (the dequant GEMM
     // overlaps the U kernel and the launch gaps; see grid_dependency_wait in each)
@@ -904,7 +940,8 @@ qlora_status launch_tc_decode(const DecodeArgs& a, cudaStream_t stream) {
     QLORA_CHECK_LAUNCH();
     (void)launch_dependent(decode_fixup, dim3((unsigned)tiles), dim3(128), (size_t)a.r * 16 * sizeof(float), stream,
                            (const float*)a.partial, p.units, p.grid, (int)p.ksteps, a.M, N, (const float*)a.U,
-                           static_cast<const uint16_t*>(a.B), a.r, a.scale, a.out, (int)a.out_f32);
+                           static_cast<const uint16_t*>(a.B), a.r, a.scale, a.out, (int)a.out_f32, a.aidx,
+                           (int)a.n_adapters);
     QLORA_CHECK_LAUNCH();
     return QLORA_OK;
 }

@@ -66,6 +66,8 @@ struct DecodeArgs {
     int32_t out_f32;
     float* U;               // [M, r] fp32, written (X A^T)
     float* partial;         // decode_partial_bytes(N, K)
+    const int32_t* aidx;    // multi-adapter: device [M] adapter of each token (-1: none); NULL: one adapter
+    int32_t n_adapters;     // multi-adapter: A is [n_adapters, r, K], B is [n_adapters, N, r]
 };
 
 constexpr int64_t kDecodeMaxM = 16;

@@ -18,6 +18,8 @@
  *   [QR]  ainexis.cn, walkthrough of "QLoRA: Efficient Finetuning of Quantized
  *         LLMs", section 4.4: backpropagation passes through the frozen 4-bit
  *         weight into the adapters.
+ *   [CH9] mdooai.com, "Ch.09 QLoRA 与量化：缩得更小再微调", section "3. 一个
+ *         底座，多个适配器": one shared compressed base, one thin adapter per task.
  *   [Q103] agentalpha.top, "Q103: What is QLoRA, and how does it differ from
  *         LoRA", follow-up 1: after fine-tuning, merge the LoRA weights and
  *         dequantize for fast inference.
@@ -221,6 +223,28 @@ qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const void* X, int64_t 
                               const void* A, const void* B, int32_t r, float alpha,
                               void* Y, int32_t y_dtype, float* U_save,
                               void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Forward for a batch of at most 16 tokens that each use their own adapter
+ * over one shared quantized base weight ([CH9] section "3. 一个底座，多个适配器":
+ * one shared compressed base, each task swaps only a thin LoRA adapter):
+ *     Y[m] = X[m] W_hat^T + s (X[m] A_a^T) B_a^T,  a = adapter_idx[m], s = alpha / r,
+ * and Y[m] = X[m] W_hat^T for a token with adapter_idx[m] == -1.
+ *   A_all       device bf16 [n_adapters, r, K]
+ *   B_all       device bf16 [n_adapters, N, r]
+ *   adapter_idx device int32 [M]; an index >= n_adapters is treated as -1 and
+ *               raises the device BOUNDS flag (bit 2 of qlora_read_device_errors).
+ *   U_save      optional device fp32 [M, r]: U[m] = X[m] A_a^T (0 without adapter).
+ *   workspace   at least qlora_linear_workspace_size(M, N, K, r) bytes.
+ * The base product uses the same small-M kernel as qlora_linear_fwd.
+ * Errors: QLORA_ERR_SHAPE for M > 16, QLORA_ERR_INVALID_ARG for n_adapters < 1
+ * or a null adapter_idx, and those of qlora_linear_fwd.
+ */
+qlora_status qlora_linear_fwd_multi(const qlora_nf4_weight* w, const void* X, int64_t M,
+                                    const void* A_all, const void* B_all, int32_t n_adapters,
+                                    const int32_t* adapter_idx, int32_t r, float alpha,
+                                    void* Y, int32_t y_dtype, float* U_save,
+                                    void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Backward of the QLoRA linear layer through the frozen dequantized weight

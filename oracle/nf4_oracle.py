@@ -477,6 +477,23 @@ def linear_forward(X, W_hat, A, B, alpha: float, r: int):
     return Y, U
 
 
+def linear_forward_multi(X, W_hat, A_all, B_all, adapter_idx, alpha: float, r: int):
+    """One base, many adapters ([CH9] section "3. 一个底座，多个适配器"): token m uses adapter
+    a = adapter_idx[m] (A_all[a] [r,K], B_all[a] [N,r]); a == -1 means the base alone.
+    Y[m] = X[m] W_hat^T + s (X[m] A_a^T) B_a^T in fp64.  Returns (Y, U), U[m] = X[m] A_a^T (0 for -1)."""
+    Xd, Wd = _f64(X), _f64(W_hat)
+    Ad, Bd = _f64(A_all), _f64(B_all)
+    s = lora_scale(alpha, r)
+    Y = Xd @ Wd.T
+    U = np.zeros((Xd.shape[0], r))
+    for m, a in enumerate(np.asarray(adapter_idx).ravel()):
+        if a < 0:
+            continue
+        U[m] = Xd[m] @ Ad[a].T
+        Y[m] += s * (U[m] @ Bd[a].T)
+    return Y, U
+
+
 def linear_backward(X, dY, W_hat, A, B, alpha: float, r: int):
     """Gradients of <dY, Y> through the frozen W_hat; no gradient for the codes.
 

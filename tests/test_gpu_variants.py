@@ -181,3 +181,40 @@ def test_merge_with_zero_B_is_the_dequantized_weight():
     w = q4.qlora_quantize_nf4_dq(W.to(DEV))
     Wm = q4.qlora_merge_lora(w, A.to(DEV), torch.zeros_like(B).to(DEV), 16, 32.0)
     assert torch.equal(Wm, q4.qlora_dequantize(w))
+
+
+# ------------------------------------------------------------------ one base, many adapters
+
+@pytest.mark.parametrize("M,N,K,r,n_ad", [(16, 1000, 640, 16, 16), (7, 2600, 64, 8, 3), (1, 300, 4096, 64, 2),
+                                          (16, 9000, 1024, 3, 5), (12, 264, 320, 96, 4)])
+def test_multi_adapter_forward(M, N, K, r, n_ad):
+    g = np.random.default_rng(M + N + K)
+    W, X, A, B, dY = si.custom_linear(N, K, M, r, seed=M + N + K + r)
+    A_all = torch.stack([si.custom_linear(N, K, M, r, seed=100 + a)[2] for a in range(n_ad)])
+    B_all = torch.stack([(si.custom_linear(N, K, M, r, seed=200 + a)[3].float() * (a + 1)).to(torch.bfloat16)
+                         for a in range(n_ad)])
+    idx = g.integers(-1, n_ad, size=M).astype(np.int32)
+    idx[0] = n_ad - 1                                   # at least one adapted token
+    alpha = 2.0 * r
+    w = q4.qlora_quantize_nf4_dq(W.to(DEV))
+    Y, U = q4.qlora_linear_fwd_multi(w, X.to(DEV), A_all.to(DEV), B_all.to(DEV), torch.from_numpy(idx).to(DEV),
+                                     r, alpha, save_U=True)
+    torch.cuda.synchronize()
+    _, Wh = oracle_variant(W, "nf4", True)
+    Yr, Ur = o.linear_forward_multi(si.bf16_bits(X), Wh, si.bf16_bits(A_all), si.bf16_bits(B_all), idx, alpha, r)
+    assert_close(Y, Yr, "Y multi")
+    assert_close(U, Ur, "U multi")
+
+
+def test_multi_adapter_out_of_range_index_sets_flag_and_uses_base():
+    W, X, A, B, dY = si.custom_linear(256, 256, 2, 8, seed=21)
+    w = q4.qlora_quantize_nf4_dq(W.to(DEV))
+    idx = torch.tensor([0, 7], dtype=torch.int32, device=DEV)       # 7 >= n_adapters = 1
+    q4.qlora_read_device_errors(clear=True)
+    Y, _ = q4.qlora_linear_fwd_multi(w, X.to(DEV), A[None].to(DEV), B[None].to(DEV), idx, 8, 16.0)
+    flags = q4.qlora_read_device_errors(clear=True)
+    assert flags & 4
+    _, Wh = oracle_variant(W, "nf4", True)
+    Yr, _ = o.linear_forward_multi(si.bf16_bits(X), Wh, si.bf16_bits(A)[None], si.bf16_bits(B)[None], [0, -1],
+                                   16.0, 8)
+    assert_close(Y, Yr, "Y with one token on the base")

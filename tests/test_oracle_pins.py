@@ -558,3 +558,25 @@ def test_merge_definition_and_degenerate_cases():
         for k in range(128):
             brute[n, k] = Whf[n, k] + 2.0 * sum(Bf[n, j] * Af[j, k] for j in range(3))
     assert np.array_equal(o.merge_lora(Wh, bA, bB, 6.0, 3), o.f64_to_bf16_bits(brute))
+
+
+# ---------------------------------------------------------------- one base, many adapters
+
+def test_multi_adapter_forward_reduces_to_single_and_base():
+    W, X, A, B, dY = si.custom_linear(24, 128, 5, 4, seed=13)
+    qw = o.quantize_nf4_dq(si.bf16_bits(W))
+    Wh = o.dequantize(qw["codes"], qw["c1_codes"], qw["c2"], qw["mu"], 24, 128)
+    bX, bA, bB = si.bf16_bits(X), si.bf16_bits(A), si.bf16_bits(B)
+    A2 = np.stack([np.zeros_like(bA), bA]).astype(np.uint16)
+    B2 = np.stack([np.zeros_like(bB), bB]).astype(np.uint16)
+    Y1, U1 = o.linear_forward(bX, Wh, bA, bB, 8.0, 4)
+    Ym, Um = o.linear_forward_multi(bX, Wh, A2, B2, [1] * 5, 8.0, 4)
+    assert np.array_equal(Ym, Y1) and np.array_equal(Um, U1)            # every token on one adapter
+    Yb, Ub = o.linear_forward_multi(bX, Wh, A2, B2, [-1] * 5, 8.0, 4)
+    assert np.array_equal(Yb, o._f64(bX) @ o._f64(Wh).T) and not Ub.any()  # no adapter: base only
+    # mixed: each row equals the single-adapter result of its own adapter (brute force per row)
+    idx = [1, -1, 0, 1, -1]
+    Ymix, _ = o.linear_forward_multi(bX, Wh, A2, B2, idx, 8.0, 4)
+    for m, a in enumerate(idx):
+        ref = o.linear_forward(bX[m:m + 1], Wh, A2[max(a, 0)], B2[max(a, 0)], 8.0 if a >= 0 else 0.0, 4)[0]
+        assert np.allclose(Ymix[m], ref[0], rtol=1e-12, atol=1e-12)
