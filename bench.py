@@ -504,6 +504,41 @@ def merge_requantize(device, peaks, wl):
     return out
 
 
+def compute_dtype_compare(device, peaks, wl):
+    """Forward + backward of the workload's largest linear computing in bf16 and in fp16
+    (same weight, same kernels with fp16 operands): TFLOP/s of each."""
+    import torch
+    import bit_nf4_quantized_23_b200 as q4
+    import synthetic_inputs as si
+    i = max(range(len(wl.linears)), key=lambda j: wl.linears[j][0] * wl.linears[j][1])
+    N, K = wl.linears[i]
+    M, r = wl.M, wl.r
+    W = si.weight(wl, i).to(device)
+    X, A, B, dY = (si.activations(wl, K, M).to(device), *[t.to(device) for t in si.lora(wl, i)],
+                   si.grad_output(wl, i, M).to(device))
+    flops = 4 * M * N * K + 6 * M * r * (N + K)
+    out = {"linear": f"M={M}, W[{N},{K}], r={r}", "flops_per_call": flops}
+    for name, dt in (("bf16", torch.bfloat16), ("fp16", torch.float16)):
+        w = q4.qlora_quantize_nf4_dq(W, compute_dtype=dt)
+        Xc, Ac, Bc, dYc = (t.to(dt) for t in (X, A, B, dY))
+        def call():
+            Y, U = q4.qlora_linear_fwd(w, Xc, Ac, Bc, r, wl.alpha)
+            q4.qlora_linear_bwd(w, Xc, dYc, Ac, Bc, r, wl.alpha, U_saved=U)
+        for _ in range(3):
+            call()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(5):
+            call()
+        b.record()
+        b.synchronize()
+        ms = a.elapsed_time(b) / 5
+        out[name] = {"ms": round(ms, 4), "TFLOP/s": round(flops / (ms * 1e-3) / 1e12, 1)}
+    del W, X, A, B, dY
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args):
     import torch
     import bit_nf4_quantized_23_b200 as q4
@@ -609,7 +644,7 @@ def run_ours(args):
                         "frac_of_hbm": round(quant_bytes / (q_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3),
                         "ms_per_step": round(q_ms, 4), "bytes_per_weight": round(2.0 + PACKED_BYTES_PER_WEIGHT, 6),
                         "source": "live CUDA events over the timed steps (7 calls per step)"}}
-    decode = variants = merge = None
+    decode = variants = merge = dtypes = None
     if rank == 0 and not args.no_decode:
         del lins
         torch.cuda.empty_cache()
@@ -617,6 +652,7 @@ def run_ours(args):
         decode = decode_sweep(device, peaks)
         variants = quantizer_variants(device, peaks, wl)
         merge = merge_requantize(device, peaks, wl)
+        dtypes = compute_dtype_compare(device, peaks, wl)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -639,7 +675,7 @@ def run_ours(args):
                                + (" + NCCL all-reduce of dA/dB" if world > 1 else "")},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
             "clocks": clk, "kernels": breakdown, "hbm_bound_ops": hbm, "decode_small_m": decode,
-            "quantizer_variants": variants, "merge_requantize": merge}
+            "quantizer_variants": variants, "merge_requantize": merge, "compute_dtype": dtypes}
     print(json.dumps(line), flush=True)
     return 0
 

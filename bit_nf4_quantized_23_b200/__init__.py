@@ -15,7 +15,8 @@ from dataclasses import dataclass
 
 import torch
 
-from ._lib import (QLORA_DTYPE_BF16, QLORA_DTYPE_F32, TIMER_KINDS, NF4WeightC, QloraError, check, lib)
+from ._lib import (QLORA_DTYPE_BF16, QLORA_DTYPE_F16, QLORA_DTYPE_F32, TIMER_KINDS, NF4WeightC, QloraError,
+                   check, lib)
 
 __all__ = [
     "NF4Weight", "QloraError", "CODEBOOKS", "qlora_nf4_sizes", "qlora_nf4_codebook", "qlora_codebook_values",
@@ -49,9 +50,11 @@ def _need(t: torch.Tensor, dtype, name: str, shape=None):
 def _dtype_code(dtype) -> int:
     if dtype == torch.bfloat16:
         return QLORA_DTYPE_BF16
+    if dtype == torch.float16:
+        return QLORA_DTYPE_F16
     if dtype == torch.float32:
         return QLORA_DTYPE_F32
-    raise TypeError("output dtype must be torch.bfloat16 or torch.float32")
+    raise TypeError("output dtype must be torch.bfloat16, torch.float16 or torch.float32")
 
 
 @dataclass
@@ -69,25 +72,29 @@ class NF4Weight:
     K: int
     codebook: str = "nf4"
     c1: torch.Tensor | None = None      # fp32 [N*K/64] when double quantization is off
+    compute_dtype: torch.dtype = torch.bfloat16   # or torch.float16: W_hat, activations, adapters
 
     def c_struct(self) -> NF4WeightC:
         p = lambda t: t.data_ptr() if t is not None else None
         return NF4WeightC(self.codes.data_ptr(), p(self.c1_codes), p(self.c2), p(self.mu), self.N, self.K,
-                          64, 256, CODEBOOKS[self.codebook], 0, p(self.c1))
+                          64, 256, CODEBOOKS[self.codebook], _dtype_code(self.compute_dtype), p(self.c1))
 
     @staticmethod
-    def empty(N: int, K: int, device="cuda", codebook: str = "nf4", double_quant: bool = True) -> "NF4Weight":
+    def empty(N: int, K: int, device="cuda", codebook: str = "nf4", double_quant: bool = True,
+              compute_dtype: torch.dtype = torch.bfloat16) -> "NF4Weight":
         if codebook not in CODEBOOKS:
             raise ValueError(f"codebook must be one of {sorted(CODEBOOKS)}")
+        if compute_dtype not in (torch.bfloat16, torch.float16):
+            raise ValueError("compute_dtype must be torch.bfloat16 or torch.float16")
         s = qlora_nf4_sizes(N, K)
         codes = torch.empty(s["codes"], dtype=torch.uint8, device=device)
         if not double_quant:
             return NF4Weight(codes, None, None, None, N, K, codebook,
-                             torch.empty(s["c1_codes"], dtype=torch.float32, device=device))
+                             torch.empty(s["c1_codes"], dtype=torch.float32, device=device), compute_dtype)
         return NF4Weight(codes,
                          torch.empty(s["c1_codes"], dtype=torch.uint8, device=device),
                          torch.empty(s["c2"] // 4, dtype=torch.float32, device=device),
-                         torch.empty(1, dtype=torch.float32, device=device), N, K, codebook)
+                         torch.empty(1, dtype=torch.float32, device=device), N, K, codebook, None, compute_dtype)
 
 
 CODEBOOKS = {"nf4": 0, "uniform4": 1}
@@ -118,16 +125,17 @@ def qlora_codebook_values(codebook: str = "nf4"):
 
 def qlora_quantize_nf4_dq(W: torch.Tensor, blocksize: int = 64, blocksize2: int = 256,
                           out: NF4Weight | None = None, workspace: torch.Tensor | None = None,
-                          stream=None, codebook: str = "nf4", double_quant: bool = True) -> NF4Weight:
-    """Quantize W (bf16 [N, K]); `codebook` and `double_quant` apply when `out` is None
-    (otherwise `out` carries them)."""
+                          stream=None, codebook: str = "nf4", double_quant: bool = True,
+                          compute_dtype: torch.dtype = torch.bfloat16) -> NF4Weight:
+    """Quantize W (bf16 [N, K]); `codebook`, `double_quant` and `compute_dtype` apply when `out`
+    is None (otherwise `out` carries them)."""
     _need(W, torch.bfloat16, "W")
     if W.dim() != 2:
         raise ValueError("W must be 2-D [N, K]")
     N, K = W.shape
     sizes = qlora_nf4_sizes(N, K, blocksize, blocksize2)
     if out is None:
-        out = NF4Weight.empty(N, K, W.device, codebook, double_quant)
+        out = NF4Weight.empty(N, K, W.device, codebook, double_quant, compute_dtype)
     if workspace is None:
         workspace = torch.empty(sizes["workspace"], dtype=torch.uint8, device=W.device)
     ws = out.c_struct()
@@ -150,8 +158,8 @@ def qlora_quantize_nf4_dq_noalloc(W: torch.Tensor, out: NF4Weight, stream=None) 
 
 def qlora_dequantize(w: NF4Weight, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     if out is None:
-        out = torch.empty(w.N, w.K, dtype=torch.bfloat16, device=w.codes.device)
-    _need(out, torch.bfloat16, "out", (w.N, w.K))
+        out = torch.empty(w.N, w.K, dtype=w.compute_dtype, device=w.codes.device)
+    _need(out, w.compute_dtype, "out", (w.N, w.K))
     ws = w.c_struct()
     check(lib().qlora_dequantize(byref(ws), _ptr(out), _stream(stream)), "qlora_dequantize")
     return out
@@ -161,11 +169,11 @@ def qlora_merge_lora(w: NF4Weight, A: torch.Tensor, B: torch.Tensor, r: int, alp
                      out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """W_merged = bf16(W_hat + (alpha / r) B A) for inference; requantize it with
     qlora_quantize_nf4_dq to serve the merged model in 4 bits."""
-    _need(A, torch.bfloat16, "A", (r, w.K))
-    _need(B, torch.bfloat16, "B", (w.N, r))
+    _need(A, w.compute_dtype, "A", (r, w.K))
+    _need(B, w.compute_dtype, "B", (w.N, r))
     if out is None:
-        out = torch.empty(w.N, w.K, dtype=torch.bfloat16, device=w.codes.device)
-    _need(out, torch.bfloat16, "out", (w.N, w.K))
+        out = torch.empty(w.N, w.K, dtype=w.compute_dtype, device=w.codes.device)
+    _need(out, w.compute_dtype, "out", (w.N, w.K))
     ws = w.c_struct()
     check(lib().qlora_merge_lora(byref(ws), _ptr(A), _ptr(B), r, float(alpha), _ptr(out), _stream(stream)),
           "qlora_merge_lora")
@@ -186,14 +194,16 @@ def _workspace(M, N, K, r, device, workspace):
 
 
 def qlora_linear_fwd(w: NF4Weight, X: torch.Tensor, A: torch.Tensor, B: torch.Tensor, r: int,
-                     alpha: float, y_dtype=torch.bfloat16, save_U: bool = True,
+                     alpha: float, y_dtype=None, save_U: bool = True,
                      out: torch.Tensor | None = None, U_out: torch.Tensor | None = None,
                      workspace: torch.Tensor | None = None, stream=None):
-    """Y = X W_hat^T + (alpha/r) (X A^T) B^T.  Returns (Y, U) with U fp32 [M,r] (or None)."""
+    """Y = X W_hat^T + (alpha/r) (X A^T) B^T.  Returns (Y, U) with U fp32 [M,r] (or None).
+    X, A, B are in the weight's compute dtype; Y is in it too unless y_dtype is torch.float32."""
     M = X.shape[0]
-    _need(X, torch.bfloat16, "X", (M, w.K))
-    _need(A, torch.bfloat16, "A", (r, w.K))
-    _need(B, torch.bfloat16, "B", (w.N, r))
+    y_dtype = w.compute_dtype if y_dtype is None else y_dtype
+    _need(X, w.compute_dtype, "X", (M, w.K))
+    _need(A, w.compute_dtype, "A", (r, w.K))
+    _need(B, w.compute_dtype, "B", (w.N, r))
     if out is None:
         out = torch.empty(M, w.N, dtype=y_dtype, device=X.device)
     _need(out, y_dtype, "Y", (M, w.N))
@@ -210,7 +220,7 @@ def qlora_linear_fwd(w: NF4Weight, X: torch.Tensor, A: torch.Tensor, B: torch.Te
 
 
 def qlora_linear_fwd_multi(w: NF4Weight, X: torch.Tensor, A_all: torch.Tensor, B_all: torch.Tensor,
-                           adapter_idx: torch.Tensor, r: int, alpha: float, y_dtype=torch.bfloat16,
+                           adapter_idx: torch.Tensor, r: int, alpha: float, y_dtype=None,
                            save_U: bool = False, out: torch.Tensor | None = None,
                            workspace: torch.Tensor | None = None, stream=None):
     """One base, many adapters (M <= 16 tokens): Y[m] = X[m] W_hat^T + (alpha/r) (X[m] A_a^T) B_a^T
@@ -218,9 +228,10 @@ def qlora_linear_fwd_multi(w: NF4Weight, X: torch.Tensor, A_all: torch.Tensor, B
     int32 [M] on the device.  Returns (Y, U or None)."""
     M = X.shape[0]
     n_ad = A_all.shape[0]
-    _need(X, torch.bfloat16, "X", (M, w.K))
-    _need(A_all, torch.bfloat16, "A_all", (n_ad, r, w.K))
-    _need(B_all, torch.bfloat16, "B_all", (n_ad, w.N, r))
+    y_dtype = w.compute_dtype if y_dtype is None else y_dtype
+    _need(X, w.compute_dtype, "X", (M, w.K))
+    _need(A_all, w.compute_dtype, "A_all", (n_ad, r, w.K))
+    _need(B_all, w.compute_dtype, "B_all", (n_ad, w.N, r))
     _need(adapter_idx, torch.int32, "adapter_idx", (M,))
     if out is None:
         out = torch.empty(M, w.N, dtype=y_dtype, device=X.device)
@@ -237,15 +248,16 @@ def qlora_linear_fwd_multi(w: NF4Weight, X: torch.Tensor, A_all: torch.Tensor, B
 
 def qlora_linear_bwd(w: NF4Weight, X: torch.Tensor, dY: torch.Tensor, A: torch.Tensor, B: torch.Tensor,
                      r: int, alpha: float, U_saved: torch.Tensor | None = None, need_dX: bool = True,
-                     dx_dtype=torch.bfloat16, dX: torch.Tensor | None = None,
+                     dx_dtype=None, dX: torch.Tensor | None = None,
                      dA: torch.Tensor | None = None, dB: torch.Tensor | None = None,
                      workspace: torch.Tensor | None = None, stream=None):
     """(dX, dA, dB) of <dY, Y> through the frozen W_hat.  dX is None when need_dX is False."""
     M = X.shape[0]
-    _need(X, torch.bfloat16, "X", (M, w.K))
-    _need(dY, torch.bfloat16, "dY", (M, w.N))
-    _need(A, torch.bfloat16, "A", (r, w.K))
-    _need(B, torch.bfloat16, "B", (w.N, r))
+    dx_dtype = w.compute_dtype if dx_dtype is None else dx_dtype
+    _need(X, w.compute_dtype, "X", (M, w.K))
+    _need(dY, w.compute_dtype, "dY", (M, w.N))
+    _need(A, w.compute_dtype, "A", (r, w.K))
+    _need(B, w.compute_dtype, "B", (w.N, r))
     if U_saved is not None:
         _need(U_saved, torch.float32, "U_saved", (M, r))
     if need_dX and dX is None:

@@ -20,6 +20,7 @@ STATUS_NAMES = {
 }
 QLORA_DTYPE_BF16 = 0
 QLORA_DTYPE_F32 = 1
+QLORA_DTYPE_F16 = 2
 
 # Every symbol include/qlora.h declares, with (restype, argtypes).
 _W = None  # placeholder, replaced by POINTER(NF4WeightC) below
@@ -29,7 +30,7 @@ class NF4WeightC(ctypes.Structure):
     """Mirror of qlora_nf4_weight."""
     _fields_ = [("codes", c_void_p), ("c1_codes", c_void_p), ("c2", c_void_p), ("mu", c_void_p),
                 ("N", c_int64), ("K", c_int64), ("blocksize", c_int32), ("blocksize2", c_int32),
-                ("codebook", c_int32), ("reserved", c_int32), ("c1", c_void_p)]
+                ("codebook", c_int32), ("compute_dtype", c_int32), ("c1", c_void_p)]
 
 
 _W = POINTER(NF4WeightC)

@@ -21,14 +21,15 @@ qlora_status launch_quantize(const void* W, int64_t N, int64_t K, const qlora_nf
                              void* workspace, cudaStream_t stream);
 qlora_status launch_dequantize(const qlora_nf4_weight* w, void* W_out, cudaStream_t stream);
 uint32_t* device_error_word();
-qlora_status launch_split_hi_lo(const float* V, int64_t M, int r, int R, float scale, void* V2, cudaStream_t s);
+qlora_status launch_split_hi_lo(const float* V, int64_t M, int r, int R, float scale, void* V2, bool f16,
+                                cudaStream_t s);
 qlora_status launch_dup_cols(const void* B, int64_t N, int r, int R, void* B2, cudaStream_t s);
 qlora_status launch_dup_rows(const void* A, int r, int R, int64_t K, void* A2, cudaStream_t s);
 qlora_status launch_transpose_pad(const void* B, int64_t N, int r, int R, void* Bt, cudaStream_t s);
 qlora_status launch_merge(const qlora_nf4_weight* w, const void* A, const void* B, int32_t r, float scale,
                           void* W_out, cudaStream_t stream);
 qlora_status launch_reduce_rows(const float* partial, int splits, int64_t rows, int r, int R, float scale_out,
-                                float* out, float scale_v2, void* V2, cudaStream_t s);
+                                float* out, float scale_v2, void* V2, bool f16, cudaStream_t s);
 qlora_status launch_reduce_transposed(const float* partial, int splits, int64_t rows, int r, int R, float* out,
                                       cudaStream_t s);
 
@@ -56,7 +57,7 @@ qlora_status check_weight(const qlora_nf4_weight* w) {
     QLORA_TRY(check_blocks(w->blocksize, w->blocksize2));
     QLORA_TRY(check_shape(w->N, w->K));
     if (w->codebook != QLORA_CODEBOOK_NF4 && w->codebook != QLORA_CODEBOOK_UNIFORM4) return QLORA_ERR_INVALID_ARG;
-    if (w->reserved != 0) return QLORA_ERR_INVALID_ARG;
+    if (w->compute_dtype != QLORA_DTYPE_BF16 && w->compute_dtype != QLORA_DTYPE_F16) return QLORA_ERR_INVALID_ARG;
     if (!w->codes) return QLORA_ERR_INVALID_ARG;
     if (!aligned16(w->codes)) return QLORA_ERR_ALIGN;
     if (w->c1) {   // double quantization off: fp32 block constants only
@@ -119,13 +120,19 @@ LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int32_t r) {
 
 // U = X A^T on the tensor cores, reduced into U (fp32, may be null) and U2 = hi/lo(s U).
 qlora_status lora_U(const void* X, const void* A2, int64_t M, int64_t K, int32_t r, int32_t R, float s_lora,
-                    float* U, void* U2, float* partial, cudaStream_t s) {
+                    float* U, void* U2, float* partial, bool f16, cudaStream_t s) {
     TimerScope t(QLORA_TIMER_LORA, s);
     LoraGemmArgs g{};
     g.mn_major = false; g.A = X; g.lda = K; g.B = A2; g.ldb = K; g.rows = M; g.red = K; g.R = R; g.partial = partial;
+    g.f16 = f16;
     QLORA_TRY(launch_lora_gemm(g, s));
     const int splits = lora_splits(M, (int)((K + 63) / 64));
-    return launch_reduce_rows(partial, splits, M, r, R, 1.f, U, s_lora, U2, s);
+    return launch_reduce_rows(partial, splits, M, r, R, 1.f, U, s_lora, U2, f16, s);
+}
+
+// Output dtypes a layer may write: fp32, or its 16-bit compute dtype.
+qlora_status check_out_dtype(int32_t dt, const qlora_nf4_weight* w) {
+    return (dt == QLORA_DTYPE_F32 || dt == w->compute_dtype) ? QLORA_OK : QLORA_ERR_INVALID_ARG;
 }
 
 }  // namespace
@@ -245,13 +252,14 @@ qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const void* X, int64_t 
     QLORA_TRY(check_dev(A));
     QLORA_TRY(check_dev(B));
     QLORA_TRY(check_dev(Y));
-    if (y_dtype != QLORA_DTYPE_BF16 && y_dtype != QLORA_DTYPE_F32) return QLORA_ERR_INVALID_ARG;
+    QLORA_TRY(check_out_dtype(y_dtype, w));
     if (U_save && !aligned16(U_save)) return QLORA_ERR_ALIGN;
     const LinearWs lw = linear_ws(M, w->N, w->K, r);
     if (!workspace || workspace_bytes < lw.total) return QLORA_ERR_WORKSPACE;
     if (!aligned16(workspace)) return QLORA_ERR_ALIGN;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int64_t N = w->N, K = w->K;
+    const bool f16 = w->compute_dtype == QLORA_DTYPE_F16;
     char* ws = static_cast<char*>(workspace);
     float* U = U_save ? U_save : reinterpret_cast<float*>(ws + lw.u_off);
     const float scale = alpha / (float)r;
@@ -273,7 +281,7 @@ qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const void* X, int64_t 
         QLORA_TRY(launch_dup_rows(A, r, R, K, A2, s));
         QLORA_TRY(launch_dup_cols(B, N, r, R, B2, s));
     }
-    QLORA_TRY(lora_U(X, A2, M, K, r, R, scale, U, U2, partial, s));
+    QLORA_TRY(lora_U(X, A2, M, K, r, R, scale, U, U2, partial, f16, s));
     TcGemmArgs a{};
     a.w = w; a.A0 = X; a.A1 = U2; a.B1 = B2; a.Rpad = R;
     a.p.M = M; a.p.Nout = N; a.p.out = Y; a.p.ldo = N; a.p.out_f32 = (y_dtype == QLORA_DTYPE_F32);
@@ -294,7 +302,7 @@ qlora_status qlora_linear_fwd_multi(const qlora_nf4_weight* w, const void* X, in
     QLORA_TRY(check_dev(B_all));
     QLORA_TRY(check_dev(Y));
     if (!adapter_idx) return QLORA_ERR_INVALID_ARG;
-    if (y_dtype != QLORA_DTYPE_BF16 && y_dtype != QLORA_DTYPE_F32) return QLORA_ERR_INVALID_ARG;
+    QLORA_TRY(check_out_dtype(y_dtype, w));
     if (U_save && !aligned16(U_save)) return QLORA_ERR_ALIGN;
     const LinearWs lw = linear_ws(M, w->N, w->K, r);
     if (!workspace || workspace_bytes < lw.total) return QLORA_ERR_WORKSPACE;
@@ -326,7 +334,7 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const void* X, const vo
     QLORA_TRY(check_dev(dB));
     if (dX) {
         QLORA_TRY(check_dev(dX));
-        if (dx_dtype != QLORA_DTYPE_BF16 && dx_dtype != QLORA_DTYPE_F32) return QLORA_ERR_INVALID_ARG;
+        QLORA_TRY(check_out_dtype(dx_dtype, w));
     }
     if (U_saved && !aligned16(U_saved)) return QLORA_ERR_ALIGN;
     const LinearWs lw = linear_ws(M, w->N, w->K, r);
@@ -337,6 +345,8 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const void* X, const vo
     char* ws = static_cast<char*>(workspace);
     const float scale = alpha / (float)r;
     const int32_t R = rank_pad(r);
+    const bool f16 = w->compute_dtype == QLORA_DTYPE_F16;
+    const int32_t act = f16 ? SIMT_F16 : SIMT_BF16;   // activation / adapter operand kind (CUDA-core path)
 
     if (N % 8 == 0) {
         // Tensor-core path (dY rows are 16-byte strided, so dY can be a TMA source).
@@ -350,17 +360,18 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const void* X, const vo
             TimerScope t(QLORA_TIMER_LORA, s);
             QLORA_TRY(launch_dup_rows(A, r, R, K, A2, s));
             QLORA_TRY(launch_transpose_pad(B, N, r, R, Bt, s));
-            if (U_saved) QLORA_TRY(launch_split_hi_lo(U_saved, M, r, R, scale, U2, s));
+            if (U_saved) QLORA_TRY(launch_split_hi_lo(U_saved, M, r, R, scale, U2, f16, s));
         }
-        if (!U_saved) QLORA_TRY(lora_U(X, A2, M, K, r, R, scale, nullptr, U2, partial, s));
+        if (!U_saved) QLORA_TRY(lora_U(X, A2, M, K, r, R, scale, nullptr, U2, partial, f16, s));
         {   // dU = s dY B  ->  dU (fp32) and its hi/lo split
             TimerScope t(QLORA_TIMER_LORA, s);
             LoraGemmArgs g{};
             g.mn_major = false; g.A = dY; g.lda = N; g.B = Bt; g.ldb = N; g.rows = M; g.red = N; g.R = R;
             g.partial = partial;
+            g.f16 = f16;
             QLORA_TRY(launch_lora_gemm(g, s));
             QLORA_TRY(launch_reduce_rows(partial, lora_splits(M, (int)((N + 63) / 64)), M, r, R, scale, dUf, scale,
-                                         dU2, s));
+                                         dU2, f16, s));
         }
         if (dX) {   // dX = dY W_hat + dU A
             TcGemmArgs a{};
@@ -374,6 +385,7 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const void* X, const vo
             LoraGemmArgs g{};
             g.mn_major = true; g.A = X; g.lda = K; g.B = dU2; g.ldb = 2 * R; g.rows = K; g.red = M; g.R = R;
             g.partial = partial;
+            g.f16 = f16;
             QLORA_TRY(launch_lora_gemm(g, s));
             QLORA_TRY(launch_reduce_transposed(partial, lora_splits(K, (int)((M + 63) / 64)), K, r, R, dA, s));
         }
@@ -382,9 +394,10 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const void* X, const vo
             LoraGemmArgs g{};
             g.mn_major = true; g.A = dY; g.lda = N; g.B = U2; g.ldb = 2 * R; g.rows = N; g.red = M; g.R = R;
             g.partial = partial;
+            g.f16 = f16;
             QLORA_TRY(launch_lora_gemm(g, s));
             QLORA_TRY(launch_reduce_rows(partial, lora_splits(N, (int)((M + 63) / 64)), N, r, R, 1.f, dB, 0.f,
-                                         nullptr, s));
+                                         nullptr, f16, s));
         }
         return QLORA_OK;
     }
@@ -395,8 +408,8 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const void* X, const vo
         float* Uw = reinterpret_cast<float*>(ws + lw.u_off);
         SimtGemm g{};
         g.nseg = 1;
-        g.seg[0].a = simt_dense(SIMT_BF16, X, K, 1);
-        g.seg[0].b = simt_dense(SIMT_BF16, A, K, 1);
+        g.seg[0].a = simt_dense(act, X, K, 1);
+        g.seg[0].b = simt_dense(act, A, K, 1);
         g.seg[0].K = K; g.seg[0].scale = 1.f;
         g.M = M; g.N = r; g.C = Uw; g.c_dtype = QLORA_DTYPE_F32; g.ldc = r;
         TimerScope t(QLORA_TIMER_LORA, s);
@@ -407,8 +420,8 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const void* X, const vo
     {   // dU = s dY B
         SimtGemm g{};
         g.nseg = 1;
-        g.seg[0].a = simt_dense(SIMT_BF16, dY, N, 1);
-        g.seg[0].b = simt_dense(SIMT_BF16, B, 1, r);
+        g.seg[0].a = simt_dense(act, dY, N, 1);
+        g.seg[0].b = simt_dense(act, B, 1, r);
         g.seg[0].K = N; g.seg[0].scale = scale;
         g.M = M; g.N = r; g.C = dU; g.c_dtype = QLORA_DTYPE_F32; g.ldc = r;
         TimerScope t(QLORA_TIMER_LORA, s);
@@ -417,11 +430,11 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const void* X, const vo
     if (dX) {   // dX = dY W_hat + dU A on the CUDA cores
         SimtGemm g{};
         g.nseg = 2;
-        g.seg[0].a = simt_dense(SIMT_BF16, dY, N, 1);
+        g.seg[0].a = simt_dense(act, dY, N, 1);
         g.seg[0].b = simt_nf4(w, true);
         g.seg[0].K = N; g.seg[0].scale = 1.f;
         g.seg[1].a = simt_dense(SIMT_F32, dU, r, 1);
-        g.seg[1].b = simt_dense(SIMT_BF16, A, 1, K);
+        g.seg[1].b = simt_dense(act, A, 1, K);
         g.seg[1].K = r; g.seg[1].scale = 1.f;
         g.M = M; g.N = K; g.C = dX; g.c_dtype = dx_dtype; g.ldc = K;
         TimerScope t(QLORA_TIMER_DX_MAIN, s);
@@ -431,7 +444,7 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const void* X, const vo
         SimtGemm g{};
         g.nseg = 1;
         g.seg[0].a = simt_dense(SIMT_F32, dU, 1, r);
-        g.seg[0].b = simt_dense(SIMT_BF16, X, 1, K);
+        g.seg[0].b = simt_dense(act, X, 1, K);
         g.seg[0].K = M; g.seg[0].scale = 1.f;
         g.M = r; g.N = K; g.C = dA; g.c_dtype = QLORA_DTYPE_F32; g.ldc = K;
         TimerScope t(QLORA_TIMER_LORA, s);
@@ -440,7 +453,7 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const void* X, const vo
     {   // dB = s dY^T U   ([N,r])
         SimtGemm g{};
         g.nseg = 1;
-        g.seg[0].a = simt_dense(SIMT_BF16, dY, 1, N);
+        g.seg[0].a = simt_dense(act, dY, 1, N);
         g.seg[0].b = simt_dense(SIMT_F32, U, 1, r);
         g.seg[0].K = M; g.seg[0].scale = scale;
         g.M = N; g.N = r; g.C = dB; g.c_dtype = QLORA_DTYPE_F32; g.ldc = r;

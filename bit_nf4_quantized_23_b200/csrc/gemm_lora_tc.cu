@@ -131,7 +131,7 @@ tc_lora_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
         }
     } else if (warp == 1) {
         // MMA issuer: the whole warp runs the loop, one elected lane issues the MMAs and commits
-        const uint32_t idesc = ptx::idesc_bf16_f32_ab(128, R, MN ? 1 : 0, MN ? 1 : 0);
+        const uint32_t idesc = ptx::idesc_set_f16(ptx::idesc_bf16_f32_ab(128, R, MN ? 1 : 0, MN ? 1 : 0), p.f16 != 0);
         bool ok = true;
         for (int i = 0; i < nk && ok; ++i) {
             const int s = i % kStages;
@@ -241,6 +241,7 @@ qlora_status launch_lora_gemm(const LoraGemmArgs& a, cudaStream_t stream) {
     const int splits = lora_splits(a.rows, p.ksteps_total);
     p.ksteps_per_split = (p.ksteps_total + splits - 1) / splits;
     p.partial = a.partial;
+    p.f16 = a.f16;
     p.tmem_cols = a.R <= 64 ? 64u : (a.R <= 128 ? 128u : 256u);
     p.err = device_error_word();
     if (!p.err) return QLORA_ERR_CUDA;

@@ -1,7 +1,7 @@
 // Plain CUDA-core GEMM with on-the-fly NF4 dequantization.
 //
 // C = sum over up to two segments s of  scale_s * sum_k A_s(m,k) * B_s(n,k),
-// accumulated in fp32.  Each operand is a strided bf16 or fp32 matrix, or the
+// accumulated in fp32.  Each operand is a strided bf16, fp16 or fp32 matrix, or the
 // dequantized frozen weight W_hat (as W_hat[n][k] or transposed, W_hat[k][n]),
 // expanded element by element with the same arithmetic as the dequantize
 // kernel.  This path is the correctness baseline of the library and the GEMM
@@ -23,6 +23,8 @@ __device__ __forceinline__ float load_operand(const SimtOperand& op, int64_t row
             return bf16_bits_to_f32(static_cast<const uint16_t*>(op.ptr)[row * op.s_row + k * op.s_k]);
         case SIMT_F32:
             return static_cast<const float*>(op.ptr)[row * op.s_row + k * op.s_k];
+        case SIMT_F16:
+            return f16_bits_to_f32(static_cast<const uint16_t*>(op.ptr)[row * op.s_row + k * op.s_k]);
         default: {
             const int64_t wr = (op.kind == SIMT_NF4) ? row : k;
             const int64_t wc = (op.kind == SIMT_NF4) ? k : row;
@@ -31,7 +33,7 @@ __device__ __forceinline__ float load_operand(const SimtOperand& op, int64_t row
             const uint32_t code = (flat & 1) ? (byte & 0xFu) : (byte >> 4);
             const int64_t blk = flat >> 6;
             const float c1p = op.c1f ? op.c1f[blk] : rebuild_c1(op.c1_codes[blk], op.c2[blk >> 8], *op.mu);
-            return bf16_bits_to_f32(dequant_bits(q[code], c1p));
+            return from16(dequant_bits(q[code], c1p, op.f16 != 0), op.f16 != 0);
         }
     }
 }
@@ -97,7 +99,7 @@ simt_gemm(SimtGemm g, NF4Tables tb) {
             if (g.c_dtype == QLORA_DTYPE_F32) {
                 static_cast<float*>(g.C)[off] = total[i][j];
             } else {
-                static_cast<uint16_t*>(g.C)[off] = (uint16_t)f32_to_bf16_bits_rn(total[i][j]);
+                static_cast<uint16_t*>(g.C)[off] = (uint16_t)to16_rn(total[i][j], g.c_dtype == QLORA_DTYPE_F16);
             }
         }
     }

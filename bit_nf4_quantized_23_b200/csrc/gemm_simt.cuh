@@ -9,7 +9,8 @@ enum SimtKind : int32_t {
     SIMT_BF16 = 0,   // element (row, k) = ((bf16*)ptr)[row*s_row + k*s_k]
     SIMT_F32 = 1,    // element (row, k) = ((float*)ptr)[row*s_row + k*s_k]
     SIMT_NF4 = 2,    // element (row, k) = W_hat[row][k]
-    SIMT_NF4_T = 3   // element (row, k) = W_hat[k][row]
+    SIMT_NF4_T = 3,  // element (row, k) = W_hat[k][row]
+    SIMT_F16 = 4     // element (row, k) = ((fp16*)ptr)[row*s_row + k*s_k]
 };
 
 struct SimtOperand {
@@ -22,6 +23,7 @@ struct SimtOperand {
     const float* c1f;           // NF4 kinds with double quantization off: fp32 block constants
     int64_t WK;                 // columns of W (NF4 kinds)
     int32_t codebook;           // NF4 kinds: qlora_codebook
+    int32_t f16;                // NF4 kinds: W_hat rounded to fp16 (compute dtype) instead of bf16
 };
 
 struct SimtSegment {
@@ -35,7 +37,7 @@ struct SimtGemm {
     int32_t nseg;
     int64_t M, N;
     void* C;                    // [M,N] row-major with leading dim ldc, or its transpose
-    int32_t c_dtype;            // QLORA_DTYPE_BF16 / QLORA_DTYPE_F32
+    int32_t c_dtype;            // QLORA_DTYPE_BF16 / QLORA_DTYPE_F32 / QLORA_DTYPE_F16
     int64_t ldc;
     int32_t transpose_c;        // 1: element (m,n) stored at C[n*ldc + m]
 };
@@ -51,6 +53,7 @@ inline SimtOperand simt_nf4(const qlora_nf4_weight* w, bool transposed) {
     o.kind = transposed ? SIMT_NF4_T : SIMT_NF4;
     o.ptr = w->codes; o.c1_codes = w->c1_codes; o.c2 = w->c2; o.mu = w->mu; o.c1f = w->c1; o.WK = w->K;
     o.codebook = w->codebook;
+    o.f16 = w->compute_dtype == QLORA_DTYPE_F16;
     return o;
 }
 

@@ -75,11 +75,11 @@ struct Lut {
     uint32_t L[4], H[4];   // low / high bytes of the 16 bf16 entries, 4 entries per register
 };
 
-__device__ __forceinline__ void build_lut(Lut& t, float c1p, const NF4Tables& tb) {
-    uint32_t P[8];
+__device__ __forceinline__ void build_lut(Lut& t, float c1p, const NF4Tables& tb, bool f16) {
+    uint32_t P[8];   // entries 2j, 2j+1 rounded to the compute dtype (bf16 or fp16), packed
 #pragma unroll
     for (int j = 0; j < 8; ++j)
-        P[j] = pack_bf16x2_rn(__fmul_rn(tb.q[2 * j], c1p), __fmul_rn(tb.q[2 * j + 1], c1p));
+        P[j] = pack16x2_rn(__fmul_rn(tb.q[2 * j], c1p), __fmul_rn(tb.q[2 * j + 1], c1p), f16);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         t.L[j] = prmt(P[2 * j], P[2 * j + 1], 0x6420);
@@ -225,7 +225,7 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
         // (the whole warp runs the loop; one elected lane issues the MMAs and their commits;
         // descriptors are built once and advanced by stage offsets: start address >> 4 in
         // the low 14 bits, every shared address is below 256 KiB, so no carry leaves them)
-        constexpr uint32_t idesc = ptx::idesc_bf16_f32(128, kBN, DX ? 1 : 0);
+        const uint32_t idesc = ptx::idesc_set_f16(ptx::idesc_bf16_f32(128, kBN, DX ? 1 : 0), p.f16 != 0);
         const uint64_t adesc0 = ptx::smem_desc_sw128(sA, 16, 1024);
         const uint64_t bdesc0 = DX ? ptx::smem_desc_sw128(sB, 8192, 1024) : ptx::smem_desc_sw128(sB, 16, 1024);
         bool ok = true;
@@ -339,7 +339,7 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
                     c1 = ld_shared_v4(src + (((2u * kc + 1u) ^ (row & 7u)) << 4));
                 }
                 Lut lut;
-                build_lut(lut, c1p, p.tb);
+                build_lut(lut, c1p, p.tb, p.f16 != 0);
                 expand_block_row(row_addr, row & 7u, c0, c1, lut);
             }
             ptx::fence_proxy_async_smem();
@@ -383,15 +383,16 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
 #pragma unroll
                             for (int i = 0; i < 4; ++i) {
                                 uint4 o;
-                                o.x = pack_bf16x2_rn(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]));
-                                o.y = pack_bf16x2_rn(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]));
-                                o.z = pack_bf16x2_rn(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]));
-                                o.w = pack_bf16x2_rn(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]));
+                                const bool h = p.f16 != 0;
+                                o.x = pack16x2_rn(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]), h);
+                                o.y = pack16x2_rn(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]), h);
+                                o.z = pack16x2_rn(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]), h);
+                                o.w = pack16x2_rn(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]), h);
                                 reinterpret_cast<uint4*>(dst)[i] = o;
                             }
                         } else {
                             for (int i = 0; i < 32 && nb + i < p.Nout; ++i)
-                                dst[i] = (uint16_t)f32_to_bf16_bits_rn(__uint_as_float(v[i]));
+                                dst[i] = (uint16_t)to16_rn(__uint_as_float(v[i]), p.f16 != 0);
                         }
                     }
                 }
@@ -538,7 +539,7 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, const __grid_constant
         // MMA issuer: the whole warp runs the loop, one elected lane issues.  Descriptors are
         // built once and advanced by stage offsets (start address >> 4 in the low 14 bits;
         // every shared address here is below 256 KiB, so no carry leaves them).
-        constexpr uint32_t idesc = ptx::idesc_bf16_f32_ab(128, 16, 0, 0);
+        const uint32_t idesc = ptx::idesc_set_f16(ptx::idesc_bf16_f32_ab(128, 16, 0, 0), p.f16 != 0);
         const uint64_t adesc0 = ptx::smem_desc_sw128(sA, 16, 1024);
         const uint64_t bdesc0 = ptx::smem_desc_sw128(sX, 16, 1024);
         bool ok = true;
@@ -671,7 +672,7 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, const __grid_constant
                 const uint4 x = ld_shared_v4(src);
                 const uint4 y = ld_shared_v4(src + 16u);
                 Lut lut;
-                build_lut(lut, c1p, p.tb);
+                build_lut(lut, c1p, p.tb, p.f16 != 0);
                 expand_block_row(row_addr, (uint32_t)t & 7u, x, y, lut);
             }
             ptx::fence_proxy_async_smem();
@@ -700,7 +701,7 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, const __grid_constant
 // per-token adapters (aidx), token m uses A[aidx[m]] and a token without one (-1) gets U = 0.
 __global__ void __launch_bounds__(256)
 decode_lora_u(const uint4* __restrict__ X, const uint4* __restrict__ A, int64_t K8, int r, float* __restrict__ U,
-              const int32_t* __restrict__ aidx, int n_adapters, uint32_t* err) {
+              const int32_t* __restrict__ aidx, int n_adapters, uint32_t* err, bool f16) {
     allow_dependents();                                       // the dequant GEMM does not read U
     const int j = blockIdx.x, m = blockIdx.y;
     int64_t arow = j;
@@ -730,8 +731,8 @@ decode_lora_u(const uint4* __restrict__ X, const uint4* __restrict__ A, int64_t 
             const uint32_t aw[4] = {av[q].x, av[q].y, av[q].z, av[q].w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                acc = __fmaf_rn(bf16_bits_to_f32(xw[e] & 0xFFFFu), bf16_bits_to_f32(aw[e] & 0xFFFFu), acc);
-                acc = __fmaf_rn(bf16_bits_to_f32(xw[e] >> 16), bf16_bits_to_f32(aw[e] >> 16), acc);
+                acc = __fmaf_rn(from16(xw[e] & 0xFFFFu, f16), from16(aw[e] & 0xFFFFu, f16), acc);
+                acc = __fmaf_rn(from16(xw[e] >> 16, f16), from16(aw[e] >> 16, f16), acc);
             }
         }
     }
@@ -753,7 +754,7 @@ decode_lora_u(const uint4* __restrict__ X, const uint4* __restrict__ A, int64_t 
 __global__ void __launch_bounds__(128)
 decode_fixup(const float* __restrict__ partial, int64_t units, int64_t G, int S, int64_t M, int64_t N,
              const float* __restrict__ U, const uint16_t* __restrict__ B, int r, float scale, void* out, int out_f32,
-             const int32_t* __restrict__ aidx, int n_adapters) {
+             const int32_t* __restrict__ aidx, int n_adapters, bool f16) {
     extern __shared__ float us[];                             // us[j * 16 + m] = U[m, j]
     __shared__ int32_t tok_adapter[16];
     grid_dependency_wait();                                   // partial tiles and U are complete
@@ -792,15 +793,16 @@ decode_fixup(const float* __restrict__ partial, int64_t units, int64_t G, int S,
     for (int m = 0; m < 16; ++m) lora[m] = 0.f;
     if (aidx) {
         // per-token adapters: lora[m] = sum_j U[m, j] B[a(m)][n, j] (ascending j), 0 without one
-        for (int m = 0; m < M; ++m) {
-            const int a = tok_adapter[m];
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+            const int a = m < M ? tok_adapter[m] : -1;
             if (a < 0) continue;
             const uint16_t* br = B + ((int64_t)a * N + n) * r;
             float d = 0.f;
             for (int j0 = 0; j0 < r; j0 += 8) {
                 float bv[8];
 #pragma unroll
-                for (int q = 0; q < 8; ++q) bv[q] = j0 + q < r ? bf16_bits_to_f32(br[j0 + q]) : 0.f;
+                for (int q = 0; q < 8; ++q) bv[q] = j0 + q < r ? from16(br[j0 + q], f16) : 0.f;
 #pragma unroll
                 for (int q = 0; q < 8; ++q)
                     if (j0 + q < r) d = __fmaf_rn(us[(j0 + q) * 16 + m], bv[q], d);
@@ -812,7 +814,7 @@ decode_fixup(const float* __restrict__ partial, int64_t units, int64_t G, int S,
     for (int j0 = 0; j0 < (aidx ? 0 : r); j0 += 8) {
         float bv[8];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) bv[q] = j0 + q < r ? bf16_bits_to_f32(brow[j0 + q]) : 0.f;
+        for (int q = 0; q < 8; ++q) bv[q] = j0 + q < r ? from16(brow[j0 + q], f16) : 0.f;
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
             if (j0 + q >= r) continue;
@@ -832,7 +834,7 @@ decode_fixup(const float* __restrict__ partial, int64_t units, int64_t G, int S,
         if (m < M) {
             const float y = __fmaf_rn(scale, lora[m], acc[m]);
             if (out_f32) static_cast<float*>(out)[m * N + n] = y;
-            else static_cast<uint16_t*>(out)[m * N + n] = (uint16_t)f32_to_bf16_bits_rn(y);
+            else static_cast<uint16_t*>(out)[m * N + n] = (uint16_t)to16_rn(y, f16);
         }
     }
 }
@@ -918,6 +920,7 @@ qlora_status launch_tc_decode(const DecodeArgs& a, cudaStream_t stream) {
     p.units = tiles * p.ksteps;
     p.grid = decode_grid(p.units, sms);
     p.c1_codes = w->c1_codes; p.c2 = w->c2; p.mu = w->mu; p.c1f = w->c1;
+    p.f16 = w->compute_dtype == QLORA_DTYPE_F16;
     p.partial = a.partial;
     p.tb = host_tables(w->codebook);
     p.err = device_error_word();
@@ -931,7 +934,8 @@ qlora_status launch_tc_decode(const DecodeArgs& a, cudaStream_t stream) {
         configured = true;
     }
     decode_lora_u<<<dim3((unsigned)a.r, (unsigned)a.M), 256, 0, stream>>>(
-        static_cast<const uint4*>(a.X), static_cast<const uint4*>(a.A), K / 8, a.r, a.U, a.aidx, a.n_adapters, p.err);
+        static_cast<const uint4*>(a.X), static_cast<const uint4*>(a.A), K / 8, a.r, a.U, a.aidx, a.n_adapters, p.err,
+        p.f16 != 0);
     QLORA_CHECK_LAUNCH();
     // the three kernels are chained with programmatic dependent launch (the dequant GEMM
     // overlaps the U kernel and the launch gaps; see grid_dependency_wait in each)
@@ -941,7 +945,7 @@ qlora_status launch_tc_decode(const DecodeArgs& a, cudaStream_t stream) {
     (void)launch_dependent(decode_fixup, dim3((unsigned)tiles), dim3(128), (size_t)a.r * 16 * sizeof(float), stream,
                            (const float*)a.partial, p.units, p.grid, (int)p.ksteps, a.M, N, (const float*)a.U,
                            static_cast<const uint16_t*>(a.B), a.r, a.scale, a.out, (int)a.out_f32, a.aidx,
-                           (int)a.n_adapters);
+                           (int)a.n_adapters, p.f16 != 0);
     QLORA_CHECK_LAUNCH();
     return QLORA_OK;
 }
@@ -970,6 +974,7 @@ qlora_status launch_tc_gemm_nf4(TcGemmArgs& a, bool dx, cudaStream_t stream) {
     a.p.ksteps1 = (int)(R2 / 64);
     a.p.c1_codes = w->c1_codes;
     a.p.c1f = w->c1;
+    a.p.f16 = w->compute_dtype == QLORA_DTYPE_F16;
     a.p.c2 = w->c2;
     a.p.mu = w->mu;
     a.p.WN = N;

@@ -16,6 +16,7 @@ struct TcGemmParams {
     const float* c2;
     const float* mu;
     const float* c1f;       // double quantization off: fp32 block constants (c1_codes, c2, mu unused)
+    int32_t f16;            // compute dtype fp16 (W_hat, activations and 16-bit outputs) instead of bf16
     int64_t WN, WK;         // shape of W
     void* out;
     int64_t ldo;
@@ -48,6 +49,7 @@ struct DecodeParams {
     const float* c2;
     const float* mu;
     const float* c1f;       // double quantization off: fp32 block constants (c1_codes, c2, mu unused)
+    int32_t f16;            // compute dtype fp16 (W_hat, activations and 16-bit outputs) instead of bf16
     float* partial;         // [tiles + grid][16][128] fp32 partial tiles, slot = tile + CTA
     uint32_t* err;
     uint32_t* dbg;          // second device word: where a self-check or a wait gave up
@@ -83,6 +85,7 @@ struct LoraGemmParams {
     int32_t ksteps_per_split;
     uint32_t tmem_cols;
     uint32_t stages, b_stage;   // pipeline depth and bytes of one B stage (set by the launcher)
+    int32_t f16;                // operands in fp16 instead of bf16
     float* partial;
     uint32_t* err;
 };
@@ -96,6 +99,7 @@ struct LoraGemmArgs {
     int64_t rows, red;
     int32_t R;
     float* partial;
+    int32_t f16;       // operands in fp16 instead of bf16
 };
 
 qlora_status launch_lora_gemm(const LoraGemmArgs& a, cudaStream_t stream);

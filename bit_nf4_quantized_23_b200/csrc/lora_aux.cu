@@ -4,8 +4,10 @@
 // ("QLoRA 的原理是什么？4-bit 量化权重真的参与训练吗？", section 7: the LoRA path
 // is added to the output) are accumulated by the tensor cores as extra
 // reduction steps.  U and dU are fp32 and must not lose precision, so each is
-// split into two bf16 parts hi = bf16(v), lo = bf16(v - hi) (together within
-// 2^-17 relative of v), and the other operand is duplicated:
+// split into two parts of the 16-bit compute type, hi = t(v), lo = t(v - hi)
+// (bf16: together within 2^-17 relative of v; fp16: 2^-23 while lo stays a
+// normal fp16, i.e. |v| between ~2^-3 and 65504), and the other operand is
+// duplicated:
 //     s U B^T = [hi | lo] [B | B]^T,      dU A = [hi | lo] [A ; A].
 // Every half is zero-padded from r to R (a multiple of 64) columns or rows.
 // The reduce kernels finish the split-reduction LoRA GEMMs of gemm_lora_tc.cu.
@@ -18,14 +20,14 @@ constexpr int kThreads = 256;
 
 // V2[m, j] = hi(scale * V[m, j]), V2[m, R + j] = lo(scale * V[m, j]); zero for r <= j < R.
 __global__ void split_hi_lo(const float* __restrict__ V, int64_t M, int r, int R, float scale,
-                            uint16_t* __restrict__ V2) {
+                            uint16_t* __restrict__ V2, bool f16) {
     const int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
     if (i >= M * R) return;
     const int64_t m = i / R;
     const int j = (int)(i - m * R);
     const float v = j < r ? __fmul_rn(scale, V[m * r + j]) : 0.f;
-    const uint32_t hi = f32_to_bf16_bits_rn(v);
-    const uint32_t lo = f32_to_bf16_bits_rn(__fsub_rn(v, bf16_bits_to_f32(hi)));
+    const uint32_t hi = to16_rn(v, f16);
+    const uint32_t lo = to16_rn(__fsub_rn(v, from16(hi, f16)), f16);
     V2[m * 2 * R + j] = (uint16_t)hi;
     V2[m * 2 * R + R + j] = (uint16_t)lo;
 }
@@ -102,7 +104,8 @@ __device__ __forceinline__ float sum_splits(const float* __restrict__ partial, i
 // out[row, j] = scale_out * S (j < r, when out is given) and the bf16 hi/lo split
 // of scale_v2 * S into V2[row, j] and V2[row, R + j] (zero for r <= j < R).
 __global__ void reduce_rows(const float* __restrict__ partial, int splits, int64_t rows, int r, int R,
-                            float scale_out, float* __restrict__ out, float scale_v2, uint16_t* __restrict__ V2) {
+                            float scale_out, float* __restrict__ out, float scale_v2, uint16_t* __restrict__ V2,
+                            bool f16) {
     const int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
     if (i >= rows * R) return;
     const int64_t row = i / R;
@@ -111,8 +114,8 @@ __global__ void reduce_rows(const float* __restrict__ partial, int splits, int64
     if (out && j < r) out[row * r + j] = __fmul_rn(scale_out, S);
     if (V2) {
         const float v = j < r ? __fmul_rn(scale_v2, S) : 0.f;
-        const uint32_t hi = f32_to_bf16_bits_rn(v);
-        const uint32_t lo = f32_to_bf16_bits_rn(__fsub_rn(v, bf16_bits_to_f32(hi)));
+        const uint32_t hi = to16_rn(v, f16);
+        const uint32_t lo = to16_rn(__fsub_rn(v, from16(hi, f16)), f16);
         V2[row * 2 * R + j] = (uint16_t)hi;
         V2[row * 2 * R + R + j] = (uint16_t)lo;
     }
@@ -144,9 +147,9 @@ inline unsigned blocks(int64_t n) { return (unsigned)((n + kThreads - 1) / kThre
 
 }  // namespace
 
-qlora_status launch_split_hi_lo(const float* V, int64_t M, int r, int R, float scale, void* V2,
+qlora_status launch_split_hi_lo(const float* V, int64_t M, int r, int R, float scale, void* V2, bool f16,
                                 cudaStream_t s) {
-    split_hi_lo<<<blocks(M * R), kThreads, 0, s>>>(V, M, r, R, scale, static_cast<uint16_t*>(V2));
+    split_hi_lo<<<blocks(M * R), kThreads, 0, s>>>(V, M, r, R, scale, static_cast<uint16_t*>(V2), f16);
     QLORA_CHECK_LAUNCH();
     return QLORA_OK;
 }
@@ -170,9 +173,9 @@ qlora_status launch_transpose_pad(const void* B, int64_t N, int r, int R, void* 
 }
 
 qlora_status launch_reduce_rows(const float* partial, int splits, int64_t rows, int r, int R, float scale_out,
-                                float* out, float scale_v2, void* V2, cudaStream_t s) {
+                                float* out, float scale_v2, void* V2, bool f16, cudaStream_t s) {
     reduce_rows<<<blocks(rows * R), kThreads, 0, s>>>(partial, splits, rows, r, R, scale_out, out, scale_v2,
-                                                       static_cast<uint16_t*>(V2));
+                                                       static_cast<uint16_t*>(V2), f16);
     QLORA_CHECK_LAUNCH();
     return QLORA_OK;
 }

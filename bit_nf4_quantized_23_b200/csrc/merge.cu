@@ -5,7 +5,8 @@
 // follow-up 1: merge the LoRA weights after fine-tuning; "QLoRA 的原理是什么？
 // 4-bit 量化权重真的参与训练吗？", section 5: merging and requantizing can add
 // error again): W_merged = W_hat + (alpha / r) B A, here rounded once to
-// bf16:  W_merged[n,k] = bf16_rn(fp32(W_hat[n,k] + sum_j (s B[n,j]) A[j,k])),
+// the 16-bit compute type (bf16 or fp16):
+//        W_merged[n,k] = bf16_rn(fp32(W_hat[n,k] + sum_j (s B[n,j]) A[j,k])),
 // the rank-r sum accumulated in fp32 in ascending j.  Requantizing is the
 // ordinary NF4 + double-quantization pass over W_merged.
 //
@@ -38,7 +39,7 @@ __global__ void __launch_bounds__(kMergeThreads)
 merge_lora(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ c1_codes, const float* __restrict__ c2,
            const float* __restrict__ mu_p, const float* __restrict__ c1f, int64_t N, int64_t K,
            const uint16_t* __restrict__ A, const uint16_t* __restrict__ B, int r, float s,
-           uint16_t* __restrict__ out, NF4Tables tb) {
+           uint16_t* __restrict__ out, NF4Tables tb, bool f16) {
     __shared__ float Bs[kTile][kRChunk + 1];         // s * B[n0 + i, j0 + j]
     __shared__ __align__(16) float As[kRChunk][kTile];   // A[j0 + j, k0 + c]
     __shared__ float q[16];
@@ -52,9 +53,9 @@ merge_lora(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ c1_cod
         for (int e = threadIdx.x; e < kTile * kRChunk; e += kMergeThreads) {
             const int i = e / kRChunk, j = e % kRChunk;
             const int64_t n = n0 + i;
-            Bs[i][j] = (n < N && j0 + j < r) ? __fmul_rn(s, bf16_bits_to_f32(B[n * r + j0 + j])) : 0.f;
+            Bs[i][j] = (n < N && j0 + j < r) ? __fmul_rn(s, from16(B[n * r + j0 + j], f16)) : 0.f;
             const int jj = e / kTile, c = e % kTile;
-            As[jj][c] = (j0 + jj < r) ? bf16_bits_to_f32(A[(int64_t)(j0 + jj) * K + k0 + c]) : 0.f;
+            As[jj][c] = (j0 + jj < r) ? from16(A[(int64_t)(j0 + jj) * K + k0 + c], f16) : 0.f;
         }
         __syncthreads();
         const int jn = min(kRChunk, r - j0);
@@ -83,8 +84,8 @@ merge_lora(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ c1_cod
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
             const uint32_t code = (two >> (12 - 4 * v)) & 0xFu;          // element order: high nibble first
-            const float wh = bf16_bits_to_f32(dequant_bits(q[code], c1p));
-            o[v] = f32_to_bf16_bits_rn(__fadd_rn(wh, acc[u][v]));
+            const float wh = from16(dequant_bits(q[code], c1p, f16), f16);
+            o[v] = to16_rn(__fadd_rn(wh, acc[u][v]), f16);
         }
         reinterpret_cast<uint2*>(out + flat)[0] = make_uint2(o[0] | o[1] << 16, o[2] | o[3] << 16);
     }
@@ -107,7 +108,7 @@ __global__ void __launch_bounds__(kMgThreads, 3)
 merge_lora_tc(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmA,
               const uint8_t* __restrict__ codes, const uint8_t* __restrict__ c1_codes, const float* __restrict__ c2,
               const float* __restrict__ mu_p, const float* __restrict__ c1f, int64_t N, int64_t K, int steps,
-              float s, uint16_t* __restrict__ out, uint32_t* err, NF4Tables tb) {
+              float s, uint16_t* __restrict__ out, uint32_t* err, NF4Tables tb, bool f16) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t base = (ptx::smem_addr(smem_raw) + 1023u) & ~1023u;
     uint8_t* gbase = smem_raw + (base - ptx::smem_addr(smem_raw));
@@ -152,7 +153,7 @@ merge_lora_tc(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ C
         if (ok) {
             ptx::tc_fence_after();
             if (ptx::elect_one_sync()) {
-                constexpr uint32_t idesc = ptx::idesc_bf16_f32_ab(128, kMgN, 0, 1);
+                const uint32_t idesc = ptx::idesc_set_f16(ptx::idesc_bf16_f32_ab(128, kMgN, 0, 1), f16);
                 for (int j = 0; j < steps; ++j)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
@@ -193,11 +194,11 @@ merge_lora_tc(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ C
 #pragma unroll
             for (int b = 0; b < 16; ++b) {
                 const uint32_t byte = (wds[b >> 2] >> (8 * (b & 3))) & 0xFFu;
-                const float w0 = bf16_bits_to_f32(dequant_bits(q[byte >> 4], c1p));     // element 2b
-                const float w1 = bf16_bits_to_f32(dequant_bits(q[byte & 0xFu], c1p));   // element 2b + 1
+                const float w0 = from16(dequant_bits(q[byte >> 4], c1p, f16), f16);     // element 2b
+                const float w1 = from16(dequant_bits(q[byte & 0xFu], c1p, f16), f16);   // element 2b + 1
                 const float y0 = __fadd_rn(w0, __fmul_rn(s, __uint_as_float(v[2 * b])));
                 const float y1 = __fadd_rn(w1, __fmul_rn(s, __uint_as_float(v[2 * b + 1])));
-                o[b] = f32_to_bf16_bits_rn(y0) | f32_to_bf16_bits_rn(y1) << 16;
+                o[b] = pack16x2_rn(y0, y1, f16);
             }
             uint4* dst = reinterpret_cast<uint4*>(out + flat + c * 32);
 #pragma unroll
@@ -240,14 +241,15 @@ qlora_status launch_merge(const qlora_nf4_weight* w, const void* A, const void* 
         const int steps = (r + 63) / 64;
         merge_lora_tc<<<grid, kMgThreads, mg_alloc(steps), stream>>>(
             tmB, tmA, w->codes, w->c1_codes, w->c2, w->mu, w->c1, N, K, steps, scale,
-            static_cast<uint16_t*>(W_out), err, host_tables(w->codebook));
+            static_cast<uint16_t*>(W_out), err, host_tables(w->codebook), w->compute_dtype == QLORA_DTYPE_F16);
         QLORA_CHECK_LAUNCH();
         return QLORA_OK;
     }
     const dim3 grid((unsigned)(K / kTile), (unsigned)((N + kTile - 1) / kTile));
     merge_lora<<<grid, kMergeThreads, 0, stream>>>(
         w->codes, w->c1_codes, w->c2, w->mu, w->c1, N, K, static_cast<const uint16_t*>(A),
-        static_cast<const uint16_t*>(B), r, scale, static_cast<uint16_t*>(W_out), host_tables(w->codebook));
+        static_cast<const uint16_t*>(B), r, scale, static_cast<uint16_t*>(W_out), host_tables(w->codebook),
+        w->compute_dtype == QLORA_DTYPE_F16);
     QLORA_CHECK_LAUNCH();
     return QLORA_OK;
 }

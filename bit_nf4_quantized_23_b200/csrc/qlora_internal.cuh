@@ -6,6 +6,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_fp8.h>
 #include <stdint.h>
 
@@ -72,6 +73,24 @@ __device__ __forceinline__ uint32_t pack_bf16x2_rn(float a, float b) {
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// The 16-bit compute types: bf16 (the default) or IEEE fp16, chosen per weight
+// (a warp-uniform flag in the kernels).  Round to nearest even in both.
+__device__ __forceinline__ uint32_t f32_to_f16_bits_rn(float x) {
+    return (uint32_t)__half_as_ushort(__float2half_rn(x));
+}
+__device__ __forceinline__ float f16_bits_to_f32(uint32_t b) {
+    return __half2float(__ushort_as_half((unsigned short)b));
+}
+__device__ __forceinline__ uint32_t pack_f16x2_rn(float a, float b) {
+    __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ uint32_t to16_rn(float x, bool f16) { return f16 ? f32_to_f16_bits_rn(x) : f32_to_bf16_bits_rn(x); }
+__device__ __forceinline__ float from16(uint32_t b, bool f16) { return f16 ? f16_bits_to_f32(b) : bf16_bits_to_f32(b); }
+__device__ __forceinline__ uint32_t pack16x2_rn(float a, float b, bool f16) {
+    return f16 ? pack_f16x2_rn(a, b) : pack_bf16x2_rn(a, b);
+}
+
 // Exact value of an FP8 E4M3 (finite-only) code: sign, 4-bit exponent with
 // bias 7, 3-bit mantissa; exponent field 0 holds the subnormals m * 2^-9.
 __device__ __forceinline__ float e4m3_to_f32(uint32_t c) {
@@ -93,9 +112,9 @@ __device__ __forceinline__ float rebuild_c1(uint32_t c1_code, float c2, float mu
     return __fadd_rn(__fmul_rn(e4m3_to_f32(c1_code), c2), mu);
 }
 
-// The dequantized weight value in bf16 bits: bf16_rn(fp32(q * c1')).
-__device__ __forceinline__ uint32_t dequant_bits(float q, float c1p) {
-    return f32_to_bf16_bits_rn(__fmul_rn(q, c1p));
+// The dequantized weight value in bf16 bits: bf16_rn(fp32(q * c1')), or fp16 bits.
+__device__ __forceinline__ uint32_t dequant_bits(float q, float c1p, bool f16 = false) {
+    return to16_rn(__fmul_rn(q, c1p), f16);
 }
 
 }  // namespace qlora

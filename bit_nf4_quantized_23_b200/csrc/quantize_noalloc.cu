@@ -75,7 +75,7 @@ extern "C" qlora_status qlora_quantize_nf4_dq_noalloc(const void* W, int64_t N, 
     if (N > kNoAllocMaxWeights / K) return QLORA_ERR_TOO_LARGE;
     if (!W || !out || !out->codes) return QLORA_ERR_INVALID_ARG;
     if (out->codebook != QLORA_CODEBOOK_NF4 && out->codebook != QLORA_CODEBOOK_UNIFORM4) return QLORA_ERR_INVALID_ARG;
-    if (out->reserved != 0) return QLORA_ERR_INVALID_ARG;
+    if (out->compute_dtype != QLORA_DTYPE_BF16 && out->compute_dtype != QLORA_DTYPE_F16) return QLORA_ERR_INVALID_ARG;
     if (!out->c1 && (!out->c1_codes || !out->c2 || !out->mu)) return QLORA_ERR_INVALID_ARG;
     if (!aligned16(W) || !aligned16(out->codes)) return QLORA_ERR_ALIGN;
     if (out->c1 ? !aligned16(out->c1)

@@ -228,6 +228,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32_ab(int M, int N, int a_mn,
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// The same descriptor with fp16 A and B (format code 0 in both fields) when f16 is set.
+__host__ __device__ constexpr uint32_t idesc_set_f16(uint32_t idesc, bool f16) {
+    return f16 ? (idesc & ~((7u << 7) | (7u << 10))) : idesc;
+}
+
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int b_mn) {
     return idesc_bf16_f32_ab(M, N, 0, b_mn);
 }

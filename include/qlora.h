@@ -63,7 +63,7 @@ typedef enum {
     QLORA_ERR_TOO_LARGE = 9      /* tensor larger than qlora_quantize_nf4_dq_noalloc's static scratch */
 } qlora_status;
 
-typedef enum { QLORA_DTYPE_BF16 = 0, QLORA_DTYPE_F32 = 1 } qlora_dtype;
+typedef enum { QLORA_DTYPE_BF16 = 0, QLORA_DTYPE_F32 = 1, QLORA_DTYPE_F16 = 2 } qlora_dtype;
 
 /* Code-value sets (the 16 values a 4-bit code indexes). */
 typedef enum {
@@ -96,10 +96,18 @@ typedef enum {
  *                           -- the single-level variant that trades 0.37 bits
  *                           per weight for one fewer lookup per block.
  *
+ *   compute_dtype          the 16-bit type the layer computes in ([QP] section 4:
+ *                          bf16 is the usual compute type, fp16 where bf16 is not
+ *                          well supported).  The dequantized weight is rounded to
+ *                          it, and X, A, B, dY (and 16-bit Y, dX, W_out) of the
+ *                          linear, decode and merge entry points are in it.  The
+ *                          weight to quantize is always bf16.
+ *
  * With double quantization the rebuilt block constant is
  * c1' = fp32(fp32(e4m3(c1_code) * c2) + mu); without it c1' = c1.  The
- * dequantized weight is bf16_rn(fp32(q[code] * c1')).  A zero-initialised
- * codebook and c1 give NF4 with double quantization.
+ * dequantized weight is round_nearest_even(fp32(q[code] * c1')) in the compute
+ * dtype.  A zero-initialised codebook, compute_dtype and c1 give NF4 with
+ * double quantization computing in bf16.
  */
 typedef struct {
     uint8_t* codes;
@@ -111,7 +119,7 @@ typedef struct {
     int32_t  blocksize;   /* must be 64 */
     int32_t  blocksize2;  /* must be 256 */
     int32_t  codebook;    /* qlora_codebook */
-    int32_t  reserved;    /* must be 0 */
+    int32_t  compute_dtype; /* QLORA_DTYPE_BF16 (0) or QLORA_DTYPE_F16: see below */
     float*   c1;          /* NULL: double quantization; else fp32 block constants [N*K/64] */
 } qlora_nf4_weight;
 

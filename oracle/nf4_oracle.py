@@ -61,6 +61,9 @@ R10 Quantizer variants ([SD] section 4 (2) compares NF4 with uniform INT4 by
     nearest-value rule; "double quantization off" keeps the fp32 block absmax
     c1 and dequantizes W_hat = bf16_RN(fp32(q[code] * c1)).  The error study
     measures sum (W_hat - W)^2 / sum W^2 in fp64.
+R11 fp16 compute dtype ([QP] section 4: bf16 is the usual compute type, fp16
+    where bf16 is poorly supported): W_hat = fp16_RN(fp32(q[code] * c1')),
+    activations and adapters in fp16, the same fp32 accumulation.
 """
 from __future__ import annotations
 
@@ -357,25 +360,26 @@ def quantize_nf4_dq(W_bits: np.ndarray, blocksize: int = BLOCKSIZE, blocksize2: 
 
 
 def dequantize(codes_packed: np.ndarray, c1_codes: np.ndarray, c2: np.ndarray, mu,
-               N: int, K: int, q: np.ndarray | None = None) -> np.ndarray:
-    """W_hat = bf16_RN(fp32(q[code] * c1')) as uint16 bf16 bits [N,K] (reading R6)."""
+               N: int, K: int, q: np.ndarray | None = None, f16: bool = False) -> np.ndarray:
+    """W_hat = bf16_RN(fp32(q[code] * c1')) as uint16 bf16 bits [N,K] (reading R6); with f16,
+    rounded to fp16 instead (the fp16 compute dtype)."""
     q = nf4_codebook() if q is None else q
     idx = unpack_nibbles(codes_packed)[:N * K]
     c1p = dq_constants(c1_codes, c2, mu)
     c1e = np.repeat(c1p, BLOCKSIZE)[:N * K]
     prod = (q[idx] * c1e).astype(np.float32)
-    return f32_to_bf16_bits(prod).reshape(N, K)
+    return (f32_to_f16_bits(prod) if f16 else f32_to_bf16_bits(prod)).reshape(N, K)
 
 
 def dequantize_single(codes_packed: np.ndarray, c1: np.ndarray, N: int, K: int,
-                      q: np.ndarray | None = None) -> np.ndarray:
+                      q: np.ndarray | None = None, f16: bool = False) -> np.ndarray:
     """Double quantization off (reading R10): W_hat = bf16_RN(fp32(q[code] * c1)) with the
     fp32 block absmax c1 kept as is; uint16 bf16 bits [N,K]."""
     q = nf4_codebook() if q is None else q
     idx = unpack_nibbles(codes_packed)[:N * K]
     c1e = np.repeat(np.asarray(c1, dtype=np.float32), BLOCKSIZE)[:N * K]
     prod = (q[idx] * c1e).astype(np.float32)
-    return f32_to_bf16_bits(prod).reshape(N, K)
+    return (f32_to_f16_bits(prod) if f16 else f32_to_bf16_bits(prod)).reshape(N, K)
 
 
 def relative_sq_error(W_bits: np.ndarray, What_bits: np.ndarray) -> float:
@@ -442,6 +446,29 @@ def _f64(bits_or_array) -> np.ndarray:
     return a.astype(np.float64)
 
 
+def f32_to_f16_bits(x: np.ndarray) -> np.ndarray:
+    """Round fp32 values to IEEE fp16 (nearest, ties to even: NumPy's float16 conversion);
+    uint16 bits.  The fp16 compute dtype ([QP] section 4: fp16 where bf16 is not well supported)."""
+    with np.errstate(over="ignore"):
+        return np.asarray(x, dtype=np.float32).astype(np.float16).view(np.uint16)
+
+
+def f16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    """fp16 bit patterns -> exact fp32 values."""
+    return np.asarray(bits, dtype=np.uint16).view(np.float16).astype(np.float32)
+
+
+def f64_to_f16_bits(x: np.ndarray) -> np.ndarray:
+    """Round fp64 values to fp16 directly (nearest, ties to even): 11 significant bits down to
+    2^-14, a fixed step of 2^-24 below, infinity past 65504 (after rounding)."""
+    x = np.asarray(x, dtype=np.float64)
+    _, e = np.frexp(x)
+    step = np.ldexp(1.0, np.maximum(e, -13) - 11)
+    r = np.rint(x / step) * step
+    with np.errstate(over="ignore"):
+        return r.astype(np.float16).view(np.uint16)
+
+
 def f64_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     """Round fp64 values to bf16 directly (nearest, ties to even; no fp32 step, which could
     round twice).  bf16 keeps 8 significant bits down to 2^-126 and a fixed step of 2^-133
@@ -455,12 +482,14 @@ def f64_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     return f32_to_bf16_bits(r32)
 
 
-def merge_lora(W_hat_bits, A_bits, B_bits, alpha: float, r: int) -> np.ndarray:
+def merge_lora(W_hat, A, B, alpha: float, r: int, f16: bool = False) -> np.ndarray:
     """Merged weight for inference ([Q103] follow-up 1; [QP] section 5):
-    W_merged = bf16_RN(W_hat + s B A), s = alpha / r, the rank-r product and the sum in fp64
-    (products of bf16 values are exact; one rounding at the end).  uint16 bf16 bits [N,K]."""
+    W_merged = RN16(W_hat + s B A), s = alpha / r, the rank-r product and the sum in fp64
+    (products of 16-bit values are exact; one rounding at the end to bf16, or fp16 when f16).
+    Inputs: bf16 bits (uint16) or float arrays.  Returns uint16 bits [N,K]."""
     s = lora_scale(alpha, r)
-    return f64_to_bf16_bits(_f64(W_hat_bits) + s * (_f64(B_bits) @ _f64(A_bits)))
+    merged = _f64(W_hat) + s * (_f64(B) @ _f64(A))
+    return f64_to_f16_bits(merged) if f16 else f64_to_bf16_bits(merged)
 
 
 def lora_scale(alpha: float, r: int) -> float:

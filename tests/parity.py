@@ -3,8 +3,9 @@
 Tolerance (GEMM outputs and gradients): relative Frobenius error <= 1e-3 and
 per-element |err| <= 1e-2 * max|ref|.  A bf16 output is compared with the fp64
 reference rounded to bf16 (the rounding of the output alone is ~1.6e-3 relative,
-so the unrounded reference cannot be met by any bf16 result); fp32 outputs are
-compared with the unrounded fp64 reference.
+so the unrounded reference cannot be met by any bf16 result), an fp16 output
+with the reference rounded to fp16; fp32 outputs are compared with the
+unrounded fp64 reference.
 """
 import numpy as np
 import torch
@@ -38,6 +39,8 @@ def assert_close(got_tensor: torch.Tensor, ref64: np.ndarray, name: str):
     got = gpu_values(got_tensor)
     if got_tensor.dtype == torch.bfloat16:
         ref = o.bf16_bits_to_f32(o.f32_to_bf16_bits(np.asarray(ref64).astype(np.float32))).astype(np.float64)
+    elif got_tensor.dtype == torch.float16:
+        ref = o.f16_bits_to_f32(o.f64_to_f16_bits(np.asarray(ref64))).astype(np.float64)
     else:
         ref = np.asarray(ref64, np.float64)
     assert got.shape == ref.shape, (name, got.shape, ref.shape)

@@ -139,7 +139,7 @@ def test_variant_argument_errors():
                                          ctypes.c_void_p(scratch.data_ptr()), scratch.numel(), None)
     assert st == 1                                    # QLORA_ERR_INVALID_ARG, nothing launched
     ws.codebook = 0
-    ws.reserved = 3
+    ws.compute_dtype = 3
     st = _lib.lib().qlora_quantize_nf4_dq(ctypes.c_void_p(W.data_ptr()), 64, 128, 64, 256, ctypes.byref(ws),
                                          ctypes.c_void_p(scratch.data_ptr()), scratch.numel(), None)
     assert st == 1
@@ -218,3 +218,81 @@ def test_multi_adapter_out_of_range_index_sets_flag_and_uses_base():
     Yr, _ = o.linear_forward_multi(si.bf16_bits(X), Wh, si.bf16_bits(A)[None], si.bf16_bits(B)[None], [0, -1],
                                    16.0, 8)
     assert_close(Y, Yr, "Y with one token on the base")
+
+
+# ------------------------------------------------------------------ fp16 compute dtype
+
+F16 = torch.float16
+
+
+def _f64_of(t: torch.Tensor) -> np.ndarray:
+    return t.detach().double().cpu().numpy()
+
+
+@pytest.mark.parametrize("codebook,dq", [("nf4", True), ("uniform4", False)])
+@pytest.mark.parametrize("N,K", [(256, 256), (3, 320), (520, 1088)])
+def test_fp16_dequantize_bit_exact(codebook, dq, N, K):
+    W = si.custom_linear(N, K, 1, 1, seed=N + K + 5, dist="t5_outliers")[0]
+    w = q4.qlora_quantize_nf4_dq(W.to(DEV), codebook=codebook, double_quant=dq, compute_dtype=F16)
+    q = CODEBOOK[codebook]
+    qw = o.quantize_nf4_dq(si.bf16_bits(W), q=q)
+    check_buffers(w, qw, dq)
+    ref = (o.dequantize(qw["codes"], qw["c1_codes"], qw["c2"], qw["mu"], N, K, q=q, f16=True) if dq
+           else o.dequantize_single(qw["codes"], qw["c1"], N, K, q=q, f16=True))
+    Wh = q4.qlora_dequantize(w)
+    assert Wh.dtype == F16
+    assert np.array_equal(to_numpy_bits(Wh), ref)
+
+
+@pytest.mark.parametrize("M,N,K,r", [(5, 100, 128, 3), (16, 1000, 640, 16), (130, 96, 640, 64),
+                                     (300, 520, 1088, 96), (33, 130, 256, 8)])
+def test_fp16_linear_fwd_bwd(M, N, K, r):
+    W, X, A, B, dY = si.custom_linear(N, K, M, r, seed=3 * M + N + K + r)
+    Xh, Ah, Bh, dYh = (t.float().half() for t in (X, A, B, dY))      # exact: bf16 values in fp16 range
+    alpha = 2.0 * r
+    w = q4.qlora_quantize_nf4_dq(W.to(DEV), compute_dtype=F16)
+    Xd, Ad, Bd, dYd = (t.to(DEV) for t in (Xh, Ah, Bh, dYh))
+    Y, U = q4.qlora_linear_fwd(w, Xd, Ad, Bd, r, alpha)
+    dX, dA, dB = q4.qlora_linear_bwd(w, Xd, dYd, Ad, Bd, r, alpha, U_saved=U)
+    torch.cuda.synchronize()
+    assert Y.dtype == F16 and dX.dtype == F16
+    qw = o.quantize_nf4_dq(si.bf16_bits(W))
+    Wh = o.f16_bits_to_f32(o.dequantize(qw["codes"], qw["c1_codes"], qw["c2"], qw["mu"], N, K,
+                                        f16=True)).astype(np.float64)
+    Xf, Af, Bf, dYf = (_f64_of(t) for t in (Xh, Ah, Bh, dYh))
+    Yr, Ur = o.linear_forward(Xf, Wh, Af, Bf, alpha, r)
+    g = o.linear_backward(Xf, dYf, Wh, Af, Bf, alpha, r)
+    assert_close(Y, Yr, "Y fp16")
+    assert_close(U, Ur, "U fp16")
+    assert_close(dX, g["dX"], "dX fp16")
+    assert_close(dA, g["dA"], "dA fp16")
+    assert_close(dB, g["dB"], "dB fp16")
+
+
+def test_fp16_multi_adapter_and_merge():
+    N, K, M, r, n_ad = 1000, 640, 16, 16, 4
+    W, X, A, B, dY = si.custom_linear(N, K, M, r, seed=77)
+    w = q4.qlora_quantize_nf4_dq(W.to(DEV), compute_dtype=F16)
+    qw = o.quantize_nf4_dq(si.bf16_bits(W))
+    Whb = o.dequantize(qw["codes"], qw["c1_codes"], qw["c2"], qw["mu"], N, K, f16=True)
+    Wh = o.f16_bits_to_f32(Whb).astype(np.float64)
+    A_all = torch.stack([si.custom_linear(N, K, M, r, seed=300 + a)[2] for a in range(n_ad)]).float().half()
+    B_all = torch.stack([si.custom_linear(N, K, M, r, seed=400 + a)[3] for a in range(n_ad)]).float().half()
+    idx = np.array([0, 1, 2, 3, -1, 0, 1, 2, 3, -1, 3, 2, 1, 0, 0, 1], dtype=np.int32)
+    Xh = X.float().half()
+    Y, U = q4.qlora_linear_fwd_multi(w, Xh.to(DEV), A_all.to(DEV), B_all.to(DEV), torch.from_numpy(idx).to(DEV),
+                                     r, 2.0 * r, save_U=True)
+    Yr, Ur = o.linear_forward_multi(_f64_of(Xh), Wh, _f64_of(A_all), _f64_of(B_all), idx, 2.0 * r, r)
+    assert Y.dtype == F16
+    assert_close(Y, Yr, "Y fp16 multi")
+    assert_close(U, Ur, "U fp16 multi")
+    # merge in fp16: within one fp16 step plus the fp32 accumulation bound of the fp64 merge
+    Ah, Bh = A.float().half(), (B.float() * 30.0).half()
+    Wm = q4.qlora_merge_lora(w, Ah.to(DEV), Bh.to(DEV), r, 2.0 * r)
+    assert Wm.dtype == F16
+    ref = o.merge_lora(Wh, _f64_of(Ah), _f64_of(Bh), 2.0 * r, r, f16=True)
+    gv = o.f16_bits_to_f32(to_numpy_bits(Wm)).astype(np.float64)
+    rv = o.f16_bits_to_f32(ref).astype(np.float64)
+    sumabs = 2.0 * (np.abs(_f64_of(Bh)) @ np.abs(_f64_of(Ah)))
+    step = np.ldexp(1.0, np.maximum(np.frexp(rv)[1], -13) - 11)
+    assert np.all(np.abs(gv - rv) <= step + r * 2.0 ** -23 * sumabs)

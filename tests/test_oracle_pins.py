@@ -580,3 +580,32 @@ def test_multi_adapter_forward_reduces_to_single_and_base():
     for m, a in enumerate(idx):
         ref = o.linear_forward(bX[m:m + 1], Wh, A2[max(a, 0)], B2[max(a, 0)], 8.0 if a >= 0 else 0.0, 4)[0]
         assert np.allclose(Ymix[m], ref[0], rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- fp16 compute dtype
+
+def test_fp16_rounding_matches_torch_and_rounds_once_from_fp64():
+    g = np.random.default_rng(31)
+    x = np.concatenate([g.normal(0, 1, 4000), g.normal(0, 1e-5, 500), [65504.0, 65519.0, 65520.0, -0.0, 6e-8]])
+    x32 = x.astype(np.float32)
+    assert np.array_equal(o.f32_to_f16_bits(x32),
+                          torch.from_numpy(x32).to(torch.float16).view(torch.int16).numpy().view(np.uint16))
+    assert np.array_equal(o.f16_bits_to_f32(o.f32_to_f16_bits(x32)),
+                          torch.from_numpy(x32).to(torch.float16).float().numpy())
+    # direct fp64 rounding: just above an fp16 midpoint by less than half an fp32 ulp goes up
+    m = 1.0 + 2.0 ** -11
+    assert o.f64_to_f16_bits(np.array([m + 2.0 ** -40]))[0] == 0x3C01
+    assert o.f64_to_f16_bits(np.array([m]))[0] == 0x3C00                  # tie: to even
+    y = g.normal(0, 0.3, 3000)
+    assert np.array_equal(o.f64_to_f16_bits(y.astype(np.float32).astype(np.float64)),
+                          o.f32_to_f16_bits(y.astype(np.float32)))        # fp32-exact inputs: same
+
+
+def test_fp16_dequantize_is_the_fp16_rounding_of_the_same_products():
+    bits = si.bf16_bits(si.custom_linear(16, 256, 1, 1, seed=17)[0])
+    qw = o.quantize_nf4_dq(bits)
+    h = o.dequantize(qw["codes"], qw["c1_codes"], qw["c2"], qw["mu"], 16, 256, f16=True)
+    b = o.dequantize(qw["codes"], qw["c1_codes"], qw["c2"], qw["mu"], 16, 256)
+    hv, bv = o.f16_bits_to_f32(h).astype(np.float64), o.bf16_bits_to_f32(b).astype(np.float64)
+    assert np.all(np.abs(hv - bv) <= np.abs(bv) * 2.0 ** -8)            # both round the same fp32 product
+    assert np.all(np.sign(hv) == np.sign(bv))
