@@ -54,6 +54,8 @@ __host__ __device__ inline LoraLayout lora_layout(uint32_t stages, uint32_t b_st
 template <bool MN>
 __global__ void __launch_bounds__(kThreads, 2)
 tc_lora_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, LoraGemmParams p) {
+    grid_dependency_wait();                                   // operands written by the previous kernel
+    allow_dependents();
     extern __shared__ uint8_t smem_raw[];
     const uint32_t base = (ptx::smem_addr(smem_raw) + 1023u) & ~1023u;
     uint8_t* gbase = smem_raw + (base - ptx::smem_addr(smem_raw));
@@ -217,7 +219,7 @@ qlora_status launch_lora(const CUtensorMap& tmA, const CUtensorMap& tmB, LoraGem
     p.b_stage = b_stage;
     const LoraLayout lay = lora_layout(stages, b_stage);
     const dim3 grid((unsigned)((p.rows + 127) / 128), (unsigned)splits);
-    kern<<<grid, kThreads, lay.alloc, stream>>>(tmA, tmB, p);
+    (void)launch_dependent(kern, grid, dim3(kThreads), lay.alloc, stream, tmA, tmB, p);
     QLORA_CHECK_LAUNCH();
     return QLORA_OK;
 }

@@ -141,6 +141,8 @@ template <int NUM_ACC, bool DX>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmCodes,
             const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1, TcGemmParams p) {
+    grid_dependency_wait();                                   // operands written by the previous kernel
+    allow_dependents();
     using L = Layout<NUM_ACC>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t base = (ptx::smem_addr(smem_raw) + 1023u) & ~1023u;
@@ -884,7 +886,8 @@ static qlora_status launch_one(const TcGemmArgs& a, cudaStream_t stream) {
         configured = true;
     }
     const dim3 grid((unsigned)((a.p.Nout + kBN - 1) / kBN), (unsigned)((a.p.M + L::kBM - 1) / L::kBM));
-    kern<<<grid, kGemmThreads, L::kAlloc, stream>>>(a.tmA0, a.tmCodes, a.tmA1, a.tmB1, a.p);
+    (void)launch_dependent(kern, grid, dim3(kGemmThreads), L::kAlloc, stream, a.tmA0, a.tmCodes, a.tmA1, a.tmB1,
+                           a.p);
     QLORA_CHECK_LAUNCH();
     return QLORA_OK;
 }

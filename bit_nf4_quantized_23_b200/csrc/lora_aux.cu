@@ -21,6 +21,8 @@ constexpr int kThreads = 256;
 // V2[m, j] = hi(scale * V[m, j]), V2[m, R + j] = lo(scale * V[m, j]); zero for r <= j < R.
 __global__ void split_hi_lo(const float* __restrict__ V, int64_t M, int r, int R, float scale,
                             uint16_t* __restrict__ V2, bool f16) {
+    grid_dependency_wait();                                   // inputs of the previous kernel
+    allow_dependents();
     const int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
     if (i >= M * R) return;
     const int64_t m = i / R;
@@ -34,6 +36,8 @@ __global__ void split_hi_lo(const float* __restrict__ V, int64_t M, int r, int R
 
 // B2[n, j] = B2[n, R + j] = B[n, j]; zero for r <= j < R.
 __global__ void dup_cols(const uint16_t* __restrict__ B, int64_t N, int r, int R, uint16_t* __restrict__ B2) {
+    grid_dependency_wait();                                   // inputs of the previous kernel
+    allow_dependents();
     const int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
     if (i >= N * R) return;
     const int64_t n = i / R;
@@ -45,6 +49,8 @@ __global__ void dup_cols(const uint16_t* __restrict__ B, int64_t N, int r, int R
 
 // The same with 8 columns (16 bytes) per thread, for r % 8 == 0 (B rows are then 16-byte aligned).
 __global__ void dup_cols8(const uint4* __restrict__ B, int64_t N, int r8, int R8, uint4* __restrict__ B2) {
+    grid_dependency_wait();                                   // inputs of the previous kernel
+    allow_dependents();
     const int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
     if (i >= N * R8) return;
     const int64_t n = i / R8;
@@ -56,6 +62,8 @@ __global__ void dup_cols8(const uint4* __restrict__ B, int64_t N, int r8, int R8
 
 // A2[j, k] = A2[R + j, k] = A[j, k]; zero rows for r <= j < R.  Moves 8 bf16 per thread.
 __global__ void dup_rows(const uint4* __restrict__ A, int r, int R, int64_t K8, uint4* __restrict__ A2) {
+    grid_dependency_wait();                                   // inputs of the previous kernel
+    allow_dependents();
     const int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
     if (i >= (int64_t)R * K8) return;
     const int64_t j = i / K8;
@@ -69,6 +77,8 @@ __global__ void dup_rows(const uint4* __restrict__ A, int r, int R, int64_t K8, 
 // through shared memory so that reads (along j) and writes (along n) are both coalesced.
 __global__ void __launch_bounds__(256)
 transpose_pad(const uint16_t* __restrict__ B, int64_t N, int r, int R, uint16_t* __restrict__ Bt) {
+    grid_dependency_wait();                                   // inputs of the previous kernel
+    allow_dependents();
     __shared__ uint16_t tile[32][64 + 2];
     const int64_t n0 = (int64_t)blockIdx.x * 64;
     const int j0 = blockIdx.y * 32;
@@ -106,6 +116,8 @@ __device__ __forceinline__ float sum_splits(const float* __restrict__ partial, i
 __global__ void reduce_rows(const float* __restrict__ partial, int splits, int64_t rows, int r, int R,
                             float scale_out, float* __restrict__ out, float scale_v2, uint16_t* __restrict__ V2,
                             bool f16) {
+    grid_dependency_wait();                                   // inputs of the previous kernel
+    allow_dependents();
     const int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
     if (i >= rows * R) return;
     const int64_t row = i / R;
@@ -127,6 +139,8 @@ __global__ void reduce_rows(const float* __restrict__ partial, int splits, int64
 constexpr int kTrRows = 32;
 __global__ void __launch_bounds__(256)
 reduce_transposed(const float* __restrict__ partial, int splits, int64_t rows, int r, int R, float* __restrict__ out) {
+    grid_dependency_wait();                                   // inputs of the previous kernel
+    allow_dependents();
     __shared__ float tile[64][kTrRows + 1];
     const int64_t row0 = (int64_t)blockIdx.x * kTrRows;
     const int j0 = blockIdx.y * 64;
@@ -149,33 +163,35 @@ inline unsigned blocks(int64_t n) { return (unsigned)((n + kThreads - 1) / kThre
 
 qlora_status launch_split_hi_lo(const float* V, int64_t M, int r, int R, float scale, void* V2, bool f16,
                                 cudaStream_t s) {
-    split_hi_lo<<<blocks(M * R), kThreads, 0, s>>>(V, M, r, R, scale, static_cast<uint16_t*>(V2), f16);
+    (void)launch_dependent(split_hi_lo, dim3(blocks(M * R)), dim3(kThreads), 0, s, V, M, r, R, scale,
+                           static_cast<uint16_t*>(V2), f16);
     QLORA_CHECK_LAUNCH();
     return QLORA_OK;
 }
 
 qlora_status launch_dup_cols(const void* B, int64_t N, int r, int R, void* B2, cudaStream_t s) {
     if (r % 8 == 0 && (reinterpret_cast<uintptr_t>(B) & 15u) == 0)
-        dup_cols8<<<blocks(N * (R / 8)), kThreads, 0, s>>>(static_cast<const uint4*>(B), N, r / 8, R / 8,
-                                                          static_cast<uint4*>(B2));
+        (void)launch_dependent(dup_cols8, dim3(blocks(N * (R / 8))), dim3(kThreads), 0, s,
+                               static_cast<const uint4*>(B), N, r / 8, R / 8, static_cast<uint4*>(B2));
     else
-        dup_cols<<<blocks(N * R), kThreads, 0, s>>>(static_cast<const uint16_t*>(B), N, r, R,
-                                                    static_cast<uint16_t*>(B2));
+        (void)launch_dependent(dup_cols, dim3(blocks(N * R)), dim3(kThreads), 0, s,
+                               static_cast<const uint16_t*>(B), N, r, R, static_cast<uint16_t*>(B2));
     QLORA_CHECK_LAUNCH();
     return QLORA_OK;
 }
 
 qlora_status launch_transpose_pad(const void* B, int64_t N, int r, int R, void* Bt, cudaStream_t s) {
     const dim3 grid((unsigned)((N + 63) / 64), (unsigned)((R + 31) / 32));
-    transpose_pad<<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(B), N, r, R, static_cast<uint16_t*>(Bt));
+    (void)launch_dependent(transpose_pad, grid, dim3(256), 0, s, static_cast<const uint16_t*>(B), N, r, R,
+                           static_cast<uint16_t*>(Bt));
     QLORA_CHECK_LAUNCH();
     return QLORA_OK;
 }
 
 qlora_status launch_reduce_rows(const float* partial, int splits, int64_t rows, int r, int R, float scale_out,
                                 float* out, float scale_v2, void* V2, bool f16, cudaStream_t s) {
-    reduce_rows<<<blocks(rows * R), kThreads, 0, s>>>(partial, splits, rows, r, R, scale_out, out, scale_v2,
-                                                       static_cast<uint16_t*>(V2), f16);
+    (void)launch_dependent(reduce_rows, dim3(blocks(rows * R)), dim3(kThreads), 0, s, partial, splits, rows, r, R,
+                           scale_out, out, scale_v2, static_cast<uint16_t*>(V2), f16);
     QLORA_CHECK_LAUNCH();
     return QLORA_OK;
 }
@@ -183,15 +199,15 @@ qlora_status launch_reduce_rows(const float* partial, int splits, int64_t rows, 
 qlora_status launch_reduce_transposed(const float* partial, int splits, int64_t rows, int r, int R, float* out,
                                       cudaStream_t s) {
     const dim3 grid((unsigned)((rows + kTrRows - 1) / kTrRows), (unsigned)((R + 63) / 64));
-    reduce_transposed<<<grid, 256, 0, s>>>(partial, splits, rows, r, R, out);
+    (void)launch_dependent(reduce_transposed, grid, dim3(256), 0, s, partial, splits, rows, r, R, out);
     QLORA_CHECK_LAUNCH();
     return QLORA_OK;
 }
 
 qlora_status launch_dup_rows(const void* A, int r, int R, int64_t K, void* A2, cudaStream_t s) {
     const int64_t K8 = K / 8;
-    dup_rows<<<blocks((int64_t)R * K8), kThreads, 0, s>>>(static_cast<const uint4*>(A), r, R, K8,
-                                                          static_cast<uint4*>(A2));
+    (void)launch_dependent(dup_rows, dim3(blocks((int64_t)R * K8)), dim3(kThreads), 0, s,
+                           static_cast<const uint4*>(A), r, R, K8, static_cast<uint4*>(A2));
     QLORA_CHECK_LAUNCH();
     return QLORA_OK;
 }
