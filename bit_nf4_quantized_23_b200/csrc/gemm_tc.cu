@@ -53,7 +53,8 @@ struct Layout {
     static constexpr uint32_t kA = 0;
     static constexpr uint32_t kB = kA + kStages * kAStageBytes;
     static constexpr uint32_t kCodes = kB + kStages * kBStageBytes;
-    static constexpr uint32_t kBars = kCodes + kStages * kCodesStageBytes;   // 8-byte aligned
+    static constexpr uint32_t kE4 = kCodes + kStages * kCodesStageBytes;     // E4M3 values [256] fp32
+    static constexpr uint32_t kBars = kE4 + 256 * 4;                         // 8-byte aligned
     // barriers: full_a[S], full_b[S], empty[S], acc_full; then tmem slot and abort flag
     static constexpr uint32_t kTmemSlot = kBars + (3 * kStages + 1) * 8;
     static constexpr uint32_t kAbort = kTmemSlot + 4;
@@ -159,6 +160,8 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
     const int64_t n0 = (int64_t)blockIdx.x * kBN;        // output column tile
     const int64_t m0 = (int64_t)blockIdx.y * L::kBM;     // output row tile
     const int ks0 = p.ksteps0, ktotal = p.ksteps0 + p.ksteps1;
+    float* e4tab = reinterpret_cast<float*>(gbase + L::kE4);
+    if (threadIdx.x < 256) e4tab[threadIdx.x] = e4m3_to_f32(threadIdx.x);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -298,7 +301,8 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
             const int s = it % kStages;
             const uint32_t ph = (uint32_t)(it / kStages) & 1u;
             const int64_t blk = qblk[0];
-            const float c1p = blk < 0 ? 0.f : (p.c1f ? qc2[0] : rebuild_c1(qcode[0], qc2[0], mu));
+            // c1' = fp32(fp32(v8 c2) + mu) with v8 from the shared E4M3 table, or the stored c1
+            const float c1p = blk < 0 ? 0.f : (p.c1f ? qc2[0] : __fadd_rn(__fmul_rn(e4tab[qcode[0]], qc2[0]), mu));
 #pragma unroll
             for (int d = 0; d + 1 < kGemmPrefetch; ++d) {
                 qblk[d] = qblk[d + 1];
@@ -327,13 +331,11 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
                 const uint32_t c_base = sCodes + s * kCodesStageBytes;
                 uint4 c0, c1;
                 if (!DX) {
-                    // codes tile: 256 rows x 32 bytes, unswizzled; stagger the two halves to avoid bank conflicts
+                    // codes tile: 256 rows x 32 bytes, unswizzled (2-way bank conflicts on an idle pipe
+                    // cost less than staggering the halves)
                     const uint32_t src = c_base + row * 32u;
-                    const uint32_t first = (row >> 2) & 1u;
-                    const uint4 x = ld_shared_v4(src + first * 16u);
-                    const uint4 y = ld_shared_v4(src + (first ^ 1u) * 16u);
-                    c0 = first ? y : x;
-                    c1 = first ? x : y;
+                    c0 = ld_shared_v4(src);
+                    c1 = ld_shared_v4(src + 16u);
                 } else {
                     // codes tile: 64 rows x 128 bytes, 128-byte swizzled; this unit's 32 bytes are chunks 2kc, 2kc+1
                     const uint32_t src = c_base + row * 128u;
