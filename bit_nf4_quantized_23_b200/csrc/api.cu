@@ -24,7 +24,6 @@ uint32_t* device_error_word();
 qlora_status launch_split_hi_lo(const float* V, int64_t M, int r, int R, float scale, void* V2, bool f16,
                                 cudaStream_t s);
 qlora_status launch_dup_cols(const void* B, int64_t N, int r, int R, void* B2, cudaStream_t s);
-qlora_status launch_dup_rows(const void* A, int r, int R, int64_t K, void* A2, cudaStream_t s);
 qlora_status launch_transpose_pad(const void* B, int64_t N, int r, int R, void* Bt, cudaStream_t s);
 qlora_status launch_merge(const qlora_nf4_weight* w, const void* A, const void* B, int32_t r, float scale,
                           void* W_out, cudaStream_t stream);
@@ -89,12 +88,11 @@ inline int32_t rank_pad(int32_t r) { return (r + 63) / 64 * 64; }
 //   dU  fp32 [M,r]
 //   U2  bf16 [M,2R]       hi/lo split of s*U
 //   dU2 bf16 [M,2R]       hi/lo split of dU
-//   B2  bf16 [N,2R]       [B | B]
-//   A2  bf16 [2R,K]       [A ; A]
+//   B2  bf16 [N,2R]       [B | B] (only when r % 8 != 0; otherwise the GEMM reads B itself)
 //   Bt  bf16 [R,N]        B^T, zero-padded
 //   partial fp32          split-reduction partial sums of the LoRA GEMMs
 struct LinearWs {
-    size_t u_off, du_off, u2_off, du2_off, b2_off, a2_off, bt_off, part_off, total;
+    size_t u_off, du_off, u2_off, du2_off, b2_off, bt_off, part_off, total;
 };
 
 LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int32_t r) {
@@ -106,7 +104,6 @@ LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int32_t r) {
     l.u2_off = o;  o += align_up((size_t)M * 2 * R * 2, 256);
     l.du2_off = o; o += align_up((size_t)M * 2 * R * 2, 256);
     l.b2_off = o;  o += align_up((size_t)N * 2 * R * 2, 256);
-    l.a2_off = o;  o += align_up(2 * R * (size_t)K * 2, 256);
     l.bt_off = o;  o += align_up(R * (size_t)N * 2, 256);
     size_t part = lora_partial_bytes(M, K, (int)R);
     part = std::max(part, lora_partial_bytes(M, N, (int)R));
@@ -119,11 +116,13 @@ LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int32_t r) {
 }
 
 // U = X A^T on the tensor cores, reduced into U (fp32, may be null) and U2 = hi/lo(s U).
-qlora_status lora_U(const void* X, const void* A2, int64_t M, int64_t K, int32_t r, int32_t R, float s_lora,
+// A [r, K] is read directly (ranks r .. R-1 read as zero).
+qlora_status lora_U(const void* X, const void* A, int64_t M, int64_t K, int32_t r, int32_t R, float s_lora,
                     float* U, void* U2, float* partial, bool f16, cudaStream_t s) {
     TimerScope t(QLORA_TIMER_LORA, s);
     LoraGemmArgs g{};
-    g.mn_major = false; g.A = X; g.lda = K; g.B = A2; g.ldb = K; g.rows = M; g.red = K; g.R = R; g.partial = partial;
+    g.mn_major = false; g.A = X; g.lda = K; g.B = A; g.ldb = K; g.rows = M; g.red = K; g.R = R; g.partial = partial;
+    g.b_rows = r;
     g.f16 = f16;
     QLORA_TRY(launch_lora_gemm(g, s));
     const int splits = lora_splits(M, (int)((K + 63) / 64));
@@ -266,7 +265,6 @@ qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const void* X, int64_t 
     const int32_t R = rank_pad(r);
     void* U2 = ws + lw.u2_off;
     void* B2 = ws + lw.b2_off;
-    void* A2 = ws + lw.a2_off;
     float* partial = reinterpret_cast<float*>(ws + lw.part_off);
     if (M <= kDecodeMaxM) {
         // decode: U = X A^T and the LoRA term are computed in fp32 around the dequant GEMM
@@ -276,14 +274,16 @@ qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const void* X, int64_t 
         TimerScope t(QLORA_TIMER_DECODE, s);
         return launch_tc_decode(d, s);
     }
-    {
+    const bool b_direct = (r % 8 == 0);   // B rows are 16-byte multiples: the GEMM reads B itself
+    if (!b_direct) {
         TimerScope t(QLORA_TIMER_LORA, s);
-        QLORA_TRY(launch_dup_rows(A, r, R, K, A2, s));
         QLORA_TRY(launch_dup_cols(B, N, r, R, B2, s));
     }
-    QLORA_TRY(lora_U(X, A2, M, K, r, R, scale, U, U2, partial, f16, s));
+    QLORA_TRY(lora_U(X, A, M, K, r, R, scale, U, U2, partial, f16, s));
     TcGemmArgs a{};
-    a.w = w; a.A0 = X; a.A1 = U2; a.B1 = B2; a.Rpad = R;
+    a.w = w; a.A0 = X; a.A1 = U2; a.Rpad = R;
+    a.B1 = b_direct ? B : B2;
+    a.b1_r = b_direct ? r : 0;
     a.p.M = M; a.p.Nout = N; a.p.out = Y; a.p.ldo = N; a.p.out_f32 = (y_dtype == QLORA_DTYPE_F32);
     TimerScope t(QLORA_TIMER_FWD_MAIN, s);
     return launch_tc_gemm_nf4(a, false, s);
@@ -352,17 +352,15 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const void* X, const vo
         // Tensor-core path (dY rows are 16-byte strided, so dY can be a TMA source).
         void* U2 = ws + lw.u2_off;
         void* dU2 = ws + lw.du2_off;
-        void* A2 = ws + lw.a2_off;
         void* Bt = ws + lw.bt_off;
         float* dUf = reinterpret_cast<float*>(ws + lw.du_off);
         float* partial = reinterpret_cast<float*>(ws + lw.part_off);
         {
             TimerScope t(QLORA_TIMER_LORA, s);
-            QLORA_TRY(launch_dup_rows(A, r, R, K, A2, s));
             QLORA_TRY(launch_transpose_pad(B, N, r, R, Bt, s));
             if (U_saved) QLORA_TRY(launch_split_hi_lo(U_saved, M, r, R, scale, U2, f16, s));
         }
-        if (!U_saved) QLORA_TRY(lora_U(X, A2, M, K, r, R, scale, nullptr, U2, partial, f16, s));
+        if (!U_saved) QLORA_TRY(lora_U(X, A, M, K, r, R, scale, nullptr, U2, partial, f16, s));
         {   // dU = s dY B  ->  dU (fp32) and its hi/lo split
             TimerScope t(QLORA_TIMER_LORA, s);
             LoraGemmArgs g{};
@@ -375,7 +373,7 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const void* X, const vo
         }
         if (dX) {   // dX = dY W_hat + dU A
             TcGemmArgs a{};
-            a.w = w; a.A0 = dY; a.A1 = dU2; a.B1 = A2; a.Rpad = R;
+            a.w = w; a.A0 = dY; a.A1 = dU2; a.B1 = A; a.b1_r = r; a.Rpad = R;   // A [r, K] read directly
             a.p.M = M; a.p.Nout = K; a.p.out = dX; a.p.ldo = K; a.p.out_f32 = (dx_dtype == QLORA_DTYPE_F32);
             TimerScope t(QLORA_TIMER_DX_MAIN, s);
             QLORA_TRY(launch_tc_gemm_nf4(a, true, s));

@@ -251,7 +251,8 @@ qlora_status launch_lora_gemm(const LoraGemmArgs& a, cudaStream_t stream) {
     if (!a.mn_major) {
         // A [rows, red] and B [R, red], reduction contiguous
         if (!make_tmap_2d(&tmA, true, a.A, a.red, a.rows, a.lda * 2, 64, 128, true)) return QLORA_ERR_CUDA;
-        if (!make_tmap_2d(&tmB, true, a.B, a.red, a.R, a.ldb * 2, 64, (uint32_t)a.R, true)) return QLORA_ERR_CUDA;
+        const uint64_t b_rows = a.b_rows > 0 ? (uint64_t)a.b_rows : (uint64_t)a.R;   // rows past it read as zero
+        if (!make_tmap_2d(&tmB, true, a.B, a.red, b_rows, a.ldb * 2, 64, (uint32_t)a.R, true)) return QLORA_ERR_CUDA;
         return launch_lora<false>(tmA, tmB, p, splits, stream);
     }
     // S [red, rows] with rows contiguous, V2 [red, 2R] (hi | lo)

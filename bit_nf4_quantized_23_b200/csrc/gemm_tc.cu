@@ -10,7 +10,9 @@
 // where U2 = [hi | lo] bf16 split of s*U (and dU2 of dU), B2 = [B | B] and
 // A2 = [A ; A], each half zero-padded from r to R columns/rows, so that the
 // low-rank term is computed by the tensor cores at ~fp32 accuracy as R extra
-// reduction steps accumulated into the same fp32 TMEM accumulator.
+// reduction steps accumulated into the same fp32 TMEM accumulator.  B2 and A2
+// are not materialised when the tensor maps can read B and A themselves (the
+// hi and lo steps load the same tile; ranks past r read as zero).
 //
 // CTA tile: BM = 128*NUM_ACC rows of the output (tokens) x BN = 256 columns;
 // one or two 128-row fp32 accumulators (256 TMEM columns each).  K-steps of 64
@@ -207,14 +209,15 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
                     else ptx::tma_load_2d(sCodes + s * kCodesStageBytes, &tmCodes, (int32_t)(n0 / 2), it * 64, fa);
                 } else {
                     const int j = it - ks0;
+                    const int jb = p.b1_wrap ? j % p.b1_wrap : j;   // hi and lo steps share the B1 tile
                     ptx::mbar_arrive_expect_tx(fa, L::kAStageBytes + kBStageBytes);
                     ptx::tma_load_2d(a_dst, &tmA1, j * 64, (int32_t)m0, fa);
                     if (!DX) {
-                        ptx::tma_load_2d(b_dst, &tmB1, j * 64, (int32_t)n0, fa);
+                        ptx::tma_load_2d(b_dst, &tmB1, jb * 64, (int32_t)n0, fa);
                     } else {
 #pragma unroll
                         for (int c = 0; c < 4; ++c)
-                            ptx::tma_load_2d(b_dst + c * 8192, &tmB1, (int32_t)(n0 + c * 64), j * 64, fa);
+                            ptx::tma_load_2d(b_dst + c * 8192, &tmB1, (int32_t)(n0 + c * 64), jb * 64, fa);
                     }
                 }
             }
@@ -970,7 +973,15 @@ qlora_status launch_tc_gemm_nf4(TcGemmArgs& a, bool dx, cudaStream_t stream) {
     // segment 1: LoRA operands, [M, 2R] and [N, 2R] (forward) or [2R, K] (dX)
     const int64_t R2 = 2 * (int64_t)a.Rpad;
     if (!make_tmap_2d(&a.tmA1, true, a.A1, R2, a.p.M, R2 * 2, 64, bm, true)) return QLORA_ERR_CUDA;
-    if (!dx) {
+    if (a.b1_r > 0) {   // B [N, r] or A [r, K] directly
+        const uint64_t r = (uint64_t)a.b1_r;
+        if (!dx) {
+            if (!make_tmap_2d(&a.tmB1, true, a.B1, r, N, r * 2, 64, 256, true)) return QLORA_ERR_CUDA;
+        } else {
+            if (!make_tmap_2d(&a.tmB1, true, a.B1, K, r, K * 2, 64, 64, true)) return QLORA_ERR_CUDA;
+        }
+        a.p.b1_wrap = (int32_t)(R2 / 128);
+    } else if (!dx) {
         if (!make_tmap_2d(&a.tmB1, true, a.B1, R2, N, R2 * 2, 64, 256, true)) return QLORA_ERR_CUDA;
     } else {
         if (!make_tmap_2d(&a.tmB1, true, a.B1, K, R2, K * 2, 64, 64, true)) return QLORA_ERR_CUDA;

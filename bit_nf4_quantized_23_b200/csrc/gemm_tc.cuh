@@ -21,6 +21,7 @@ struct TcGemmParams {
     void* out;
     int64_t ldo;
     int32_t out_f32;
+    int32_t b1_wrap;        // 0, or R/64 when B1 is the undoubled B / A: LoRA step j reads its step j % b1_wrap
     uint32_t* err;
     NF4Tables tb;
 };
@@ -29,8 +30,11 @@ struct TcGemmArgs {
     const qlora_nf4_weight* w;
     const void* A0;         // X [M,K] (forward) or dY [M,N] (dX), bf16
     const void* A1;         // U2 or dU2 [M, 2*Rpad], bf16
-    const void* B1;         // B2 [N, 2*Rpad] (forward) or A2 [2*Rpad, K] (dX), bf16
-    int32_t Rpad;           // LoRA rank padded to a multiple of 32
+    const void* B1;         // B2 [N, 2*Rpad] (forward) or A2 [2*Rpad, K] (dX), bf16; or, with b1_r > 0,
+                            // B [N, b1_r] / A [b1_r, K] themselves (the hi and lo steps read the same tile,
+                            // ranks past b1_r read as zero; B needs b1_r % 8 == 0)
+    int32_t b1_r;
+    int32_t Rpad;           // LoRA rank padded to a multiple of 64
     TcGemmParams p;
     CUtensorMap tmA0, tmCodes, tmA1, tmB1;
 };
@@ -98,6 +102,7 @@ struct LoraGemmArgs {
     int64_t ldb;
     int64_t rows, red;
     int32_t R;
+    int64_t b_rows;    // K-major B: rows present in memory (B rows past it, up to R, read as zero); 0: R
     float* partial;
     int32_t f16;       // operands in fp16 instead of bf16
 };

@@ -7,8 +7,11 @@
 // split into two parts of the 16-bit compute type, hi = t(v), lo = t(v - hi)
 // (bf16: together within 2^-17 relative of v; fp16: 2^-23 while lo stays a
 // normal fp16, i.e. |v| between ~2^-3 and 65504), and the other operand is
-// duplicated:
+// read twice:
 //     s U B^T = [hi | lo] [B | B]^T,      dU A = [hi | lo] [A ; A].
+// The GEMMs read A and B themselves for the two halves (their tensor maps
+// zero-fill ranks r .. R-1); only B with r % 8 != 0 (rows not 16-byte
+// multiples) is copied into [B | B] here.
 // Every half is zero-padded from r to R (a multiple of 64) columns or rows.
 // The reduce kernels finish the split-reduction LoRA GEMMs of gemm_lora_tc.cu.
 #include "qlora_internal.cuh"
@@ -58,19 +61,6 @@ __global__ void dup_cols8(const uint4* __restrict__ B, int64_t N, int r8, int R8
     const uint4 v = c < r8 ? B[n * r8 + c] : make_uint4(0, 0, 0, 0);
     B2[n * 2 * R8 + c] = v;
     B2[n * 2 * R8 + R8 + c] = v;
-}
-
-// A2[j, k] = A2[R + j, k] = A[j, k]; zero rows for r <= j < R.  Moves 8 bf16 per thread.
-__global__ void dup_rows(const uint4* __restrict__ A, int r, int R, int64_t K8, uint4* __restrict__ A2) {
-    grid_dependency_wait();                                   // inputs of the previous kernel
-    allow_dependents();
-    const int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-    if (i >= (int64_t)R * K8) return;
-    const int64_t j = i / K8;
-    const int64_t k = i - j * K8;
-    const uint4 v = j < r ? A[j * K8 + k] : make_uint4(0, 0, 0, 0);
-    A2[j * K8 + k] = v;
-    A2[(R + j) * K8 + k] = v;
 }
 
 // Bt[j, n] = B[n, j] for j < r, zero rows for r <= j < R.  A CTA moves a [64 n x 32 j] block
@@ -204,12 +194,5 @@ qlora_status launch_reduce_transposed(const float* partial, int splits, int64_t 
     return QLORA_OK;
 }
 
-qlora_status launch_dup_rows(const void* A, int r, int R, int64_t K, void* A2, cudaStream_t s) {
-    const int64_t K8 = K / 8;
-    (void)launch_dependent(dup_rows, dim3(blocks((int64_t)R * K8)), dim3(kThreads), 0, s,
-                           static_cast<const uint4*>(A), r, R, K8, static_cast<uint4*>(A2));
-    QLORA_CHECK_LAUNCH();
-    return QLORA_OK;
-}
 
 }  // namespace qlora
