@@ -86,16 +86,19 @@ transpose_pad(const uint16_t* __restrict__ B, int64_t N, int r, int R, uint16_t*
 }
 
 // Sum of the split partials partial[s][row][j] in the fixed order s = 0, 1, ...; the loads of
-// four splits are issued together (the kernels are latency-bound, not bandwidth-bound).
+// eight splits are issued together (the kernels are latency-bound, not bandwidth-bound).
 __device__ __forceinline__ float sum_splits(const float* __restrict__ partial, int splits, int64_t rows, int R,
                                             int64_t row, int j) {
     const int64_t stride = rows * R;
     const float* p = partial + row * R + j;
     float acc = 0.f;
     int s = 0;
-    for (; s + 4 <= splits; s += 4) {
-        const float a = p[(s + 0) * stride], b = p[(s + 1) * stride], c = p[(s + 2) * stride], d = p[(s + 3) * stride];
-        acc = __fadd_rn(__fadd_rn(__fadd_rn(__fadd_rn(acc, a), b), c), d);
+    for (; s + 8 <= splits; s += 8) {
+        float v[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) v[q] = p[(s + q) * stride];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc = __fadd_rn(acc, v[q]);
     }
     for (; s < splits; ++s) acc = __fadd_rn(acc, p[s * stride]);
     return acc;
@@ -124,9 +127,10 @@ __global__ void reduce_rows(const float* __restrict__ partial, int splits, int64
 }
 
 // out[j, row] = S for j < r (the transposed [r, rows] result, e.g. dA from dA^T partials).
-// A CTA sums a [32 rows x 64 j] block (reads along j, coalesced) into shared memory and writes
-// it transposed (writes along rows, coalesced).
-constexpr int kTrRows = 32;
+// A CTA sums a [16 rows x 64 j] block (reads along j, coalesced; each thread 4 elements with
+// all their split loads issued before any add) into shared memory and writes it transposed
+// (writes along rows, coalesced).
+constexpr int kTrRows = 16;
 __global__ void __launch_bounds__(256)
 reduce_transposed(const float* __restrict__ partial, int splits, int64_t rows, int r, int R, float* __restrict__ out) {
     grid_dependency_wait();                                   // inputs of the previous kernel
@@ -134,10 +138,34 @@ reduce_transposed(const float* __restrict__ partial, int splits, int64_t rows, i
     __shared__ float tile[64][kTrRows + 1];
     const int64_t row0 = (int64_t)blockIdx.x * kTrRows;
     const int j0 = blockIdx.y * 64;
-    for (int e = threadIdx.x; e < kTrRows * 64; e += 256) {
-        const int rr = e >> 6, jj = e & 63;
-        const int64_t row = row0 + rr;
-        tile[jj][rr] = (row < rows && j0 + jj < R) ? sum_splits(partial, splits, rows, R, row, j0 + jj) : 0.f;
+    const int64_t stride = rows * R;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    int64_t src[4];
+    bool ok[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {                             // element e = tid + 256 u: row e / 64, j e % 64
+        const int e = threadIdx.x + 256 * u;
+        const int64_t row = row0 + (e >> 6);
+        ok[u] = row < rows && j0 + (e & 63) < R;
+        src[u] = row * R + j0 + (e & 63);
+    }
+    for (int s = 0; s < splits; s += 2) {
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            v[2 * u] = ok[u] ? partial[s * stride + src[u]] : 0.f;
+            v[2 * u + 1] = (ok[u] && s + 1 < splits) ? partial[(s + 1) * stride + src[u]] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            acc[u] = __fadd_rn(acc[u], v[2 * u]);
+            if (s + 1 < splits) acc[u] = __fadd_rn(acc[u], v[2 * u + 1]);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int e = threadIdx.x + 256 * u;
+        tile[e & 63][e >> 6] = acc[u];
     }
     __syncthreads();
     for (int e = threadIdx.x; e < kTrRows * 64; e += 256) {
