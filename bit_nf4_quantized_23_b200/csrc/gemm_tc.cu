@@ -140,6 +140,19 @@ __device__ __forceinline__ void zero_row(uint32_t row_addr) {
     for (int c = 0; c < 8; ++c) st_shared_v4(row_addr + (c << 4), make_uint4(0, 0, 0, 0));
 }
 
+// Output tile of CTA t: row tiles run fastest within groups of kRasterGroup of them, so the
+// CTAs resident at one time share a W strip (read from HBM once, then from L2) and keep the
+// group's activation panel resident in L2 across the column tiles.
+constexpr int64_t kRasterGroup = 16;
+__device__ __forceinline__ void raster_tile(int64_t t, int64_t mtiles, int64_t ntiles, int64_t& mt, int64_t& nt) {
+    const int64_t per_group = kRasterGroup * ntiles;
+    const int64_t first = (t / per_group) * kRasterGroup;
+    const int64_t gm = min(mtiles - first, kRasterGroup);
+    const int64_t local = t % per_group;
+    mt = first + local % gm;
+    nt = local / gm;
+}
+
 template <int NUM_ACC, bool DX>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmCodes,
@@ -159,8 +172,10 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
     volatile int* abort = reinterpret_cast<volatile int*>(gbase + L::kAbort);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t n0 = (int64_t)blockIdx.x * kBN;        // output column tile
-    const int64_t m0 = (int64_t)blockIdx.y * L::kBM;     // output row tile
+    int64_t mt, nt;
+    raster_tile(blockIdx.x, (p.M + L::kBM - 1) / L::kBM, (p.Nout + kBN - 1) / kBN, mt, nt);
+    const int64_t n0 = nt * kBN;                          // output column tile
+    const int64_t m0 = mt * L::kBM;                       // output row tile
     const int ks0 = p.ksteps0, ktotal = p.ksteps0 + p.ksteps1;
     float* e4tab = reinterpret_cast<float*>(gbase + L::kE4);
     if (threadIdx.x < 256) e4tab[threadIdx.x] = e4m3_to_f32(threadIdx.x);
@@ -890,7 +905,9 @@ static qlora_status launch_one(const TcGemmArgs& a, cudaStream_t stream) {
             return QLORA_ERR_CUDA;
         configured = true;
     }
-    const dim3 grid((unsigned)((a.p.Nout + kBN - 1) / kBN), (unsigned)((a.p.M + L::kBM - 1) / L::kBM));
+    const int64_t tiles = ((a.p.Nout + kBN - 1) / kBN) * ((a.p.M + L::kBM - 1) / L::kBM);
+    if (tiles > INT32_MAX) return QLORA_ERR_SHAPE;
+    const dim3 grid((unsigned)tiles);
     (void)launch_dependent(kern, grid, dim3(kGemmThreads), L::kAlloc, stream, a.tmA0, a.tmCodes, a.tmA1, a.tmB1,
                            a.p);
     QLORA_CHECK_LAUNCH();
