@@ -64,6 +64,14 @@ R10 Quantizer variants ([SD] section 4 (2) compares NF4 with uniform INT4 by
 R11 fp16 compute dtype ([QP] section 4: bf16 is the usual compute type, fp16
     where bf16 is poorly supported): W_hat = fp16_RN(fp32(q[code] * c1')),
     activations and adapters in fp16, the same fp32 accumulation.
+R14 Blockwise INT8 ([CH9] section "2. INT8 量化" fixes the steps but not the
+    precision or the block): blocks of 64, 128 or 256 consecutive elements of
+    a bf16 tensor, fp32 arithmetic with round-to-nearest-even:
+    alpha = fp32(127 / amax), code = round half away from zero (R9) of
+    fp32(x * alpha), dequantized x_hat = fp32(code / alpha).  Degenerate
+    blocks: amax = 0 gives alpha = 0, zero codes and x_hat = 0; amax below
+    127 / FLT_MAX makes alpha = +inf, a zero element still codes to 0 and
+    every other element to +-127 (clamp), and x_hat = code / inf = +-0.
 """
 from __future__ import annotations
 
@@ -82,6 +90,10 @@ class OracleShapeError(ValueError):
 
 
 class OracleUnsupported(ValueError):
+    pass
+
+
+class OracleNonFiniteError(ValueError):
     pass
 
 
@@ -619,3 +631,35 @@ def absmax_int8(x):
     scaled = x * alpha
     code = np.sign(scaled) * np.floor(np.abs(scaled) + 0.5)
     return alpha, code.astype(np.int64), code / alpha
+
+
+def quantize_int8_blocks(bits, blocksize: int = 64):
+    """Blockwise absmax INT8 of a bf16 tensor (bits, uint16), [CH9] section
+    "2. INT8 量化" steps 1-3 in fp32 (reading R14).  Returns (codes int8 [n],
+    alpha fp32 [n / blocksize])."""
+    if blocksize not in (64, 128, 256):
+        raise OracleShapeError("blocksize must be 64, 128 or 256")
+    x = bf16_bits_to_f32(np.asarray(bits, dtype=np.uint16).ravel())
+    if x.size < 1 or x.size % blocksize:
+        raise OracleShapeError("n must be a positive multiple of blocksize")
+    if not np.all(np.isfinite(x)):
+        raise OracleNonFiniteError("tensor holds Inf or NaN")
+    xb = x.reshape(-1, blocksize)
+    amax = np.max(np.abs(xb), axis=1)                                  # step 1, exact
+    with np.errstate(divide="ignore", over="ignore", invalid="ignore"):
+        alpha = np.where(amax > 0, np.float32(127.0) / amax, np.float32(0.0)).astype(np.float32)   # step 2
+        s = (xb * alpha[:, None]).astype(np.float32)                   # step 3: x * alpha in fp32
+    s = np.where(xb == 0, np.float32(0.0), s)
+    s = np.clip(s.astype(np.float64), -127.0, 127.0)
+    code = np.sign(s) * np.floor(np.abs(s) + 0.5)                      # half away from zero, exact in fp64
+    return code.astype(np.int8).ravel(), alpha
+
+
+def dequantize_int8_blocks(codes, alpha, blocksize: int = 64):
+    """[CH9] section "2. INT8 量化" step 4 (reading R14): x_hat = fp32(code / alpha),
+    0 where alpha = 0.  Returns fp32 [n]."""
+    c = np.asarray(codes, dtype=np.int8).astype(np.float32).reshape(-1, blocksize)
+    a = np.asarray(alpha, dtype=np.float32)
+    with np.errstate(divide="ignore", over="ignore", invalid="ignore"):
+        xh = np.where(a[:, None] == 0, np.float32(0.0), c / a[:, None]).astype(np.float32)
+    return xh.ravel()

@@ -410,6 +410,94 @@ def test_int8_worked_example():
     assert abs(codes[0] / alpha - g["dequant_of_28_approx"]) <= g["dequant_tolerance"]
 
 
+def _int8_block(vals, blocksize=64):
+    x = np.zeros(blocksize, np.float32)
+    x[:len(vals)] = vals
+    return o.f32_to_bf16_bits(x)
+
+
+def test_int8_blocks_worked_example():
+    # the page's vector (1.2, -0.5, 5.4) as one block of 64 (the rest zeros), in bf16
+    g = read_golden("int8_absmax_example.txt")
+    codes, alpha = o.quantize_int8_blocks(_int8_block(g["input"]), 64)
+    # (5.4 is 5.40625 in bf16, so alpha is 23.49 here: the page's "rounds to 24" holds for the
+    # exact 5.4 only and is pinned by test_int8_worked_example)
+    assert abs(float(alpha[0]) - g["alpha_approx"]) <= g["alpha_tolerance"]
+    assert codes[0] == g["code_of_1.2"] and codes[2] == g["peak_code"] and codes[1] == -12
+    assert np.all(codes[3:] == 0)
+    xh = o.dequantize_int8_blocks(codes, alpha, 64)
+    assert abs(float(xh[0]) - g["dequant_of_28_approx"]) <= g["dequant_tolerance"]
+
+
+def test_int8_blocks_round_half_away():
+    # amax = 127 makes alpha exactly 1, so x * alpha = x: exact halves must round away from zero
+    codes, alpha = o.quantize_int8_blocks(_int8_block([127.0, 2.5, -2.5, 0.5, -0.5, 1.5, -1.5, 126.5]), 64)
+    assert float(alpha[0]) == 1.0
+    assert list(codes[:8]) == [127, 3, -3, 1, -1, 2, -2, 127]
+    assert np.array_equal(o.dequantize_int8_blocks(codes, alpha, 64)[:8], codes[:8].astype(np.float32))
+
+
+def test_int8_blocks_agree_with_the_fp64_example_rule():
+    # per block, the fp32 rule gives the fp64 single-block rule's codes except where the
+    # fp64 product sits within 1e-4 of a half-integer (fp32 rounding may then flip it by one)
+    rng = np.random.default_rng(5)
+    for bs in (64, 128, 256):
+        x = (rng.standard_t(5, size=bs * 6) * 0.02).astype(np.float32)
+        bits = o.f32_to_bf16_bits(x)
+        codes, alpha = o.quantize_int8_blocks(bits, bs)
+        xb = o.bf16_bits_to_f32(bits).reshape(-1, bs)
+        for b in range(xb.shape[0]):
+            a64, c64, _ = o.absmax_int8(xb[b])
+            assert abs(float(alpha[b]) - a64) <= 2 ** -23 * a64
+            s64 = xb[b].astype(np.float64) * a64
+            near_tie = np.abs(np.abs(s64) - np.floor(np.abs(s64)) - 0.5) < 1e-4
+            blk = codes[b * bs:(b + 1) * bs].astype(np.int64)
+            assert np.all((blk == c64) | (near_tie & (np.abs(blk - c64) <= 1)))
+
+
+def test_int8_blocks_invariants_and_error_bound():
+    rng = np.random.default_rng(6)
+    x = (rng.standard_normal(64 * 40) * 0.02).astype(np.float32)
+    x[::97] *= 10.0                                         # outliers
+    bits = o.f32_to_bf16_bits(x)
+    codes, alpha = o.quantize_int8_blocks(bits, 64)
+    xb = o.bf16_bits_to_f32(bits).reshape(-1, 64).astype(np.float64)
+    cb = codes.reshape(-1, 64).astype(np.int64)
+    assert np.all(np.abs(cb) <= 127)
+    peak = np.argmax(np.abs(xb), axis=1)
+    assert np.all(np.abs(cb[np.arange(len(peak)), peak]) == 127)           # the peak maps to 127
+    assert np.all((cb == 0) | (np.sign(cb) == np.sign(xb)))                # sign kept
+    xh = o.dequantize_int8_blocks(codes, alpha, 64).reshape(-1, 64).astype(np.float64)
+    a = alpha.astype(np.float64)[:, None]
+    # half a step from rounding, the fp32 product's and quotient's roundings on top
+    bound = (0.5 + 127 * 2.0 ** -23) / a + 2.0 ** -23 * np.abs(xh)
+    assert np.all(np.abs(xh - xb) <= bound)
+
+
+def test_int8_blocks_degenerate():
+    tiny = float(o.bf16_bits_to_f32(np.array([0x0001], np.uint16))[0])   # smallest bf16 subnormal
+    bits = np.concatenate([_int8_block([]), _int8_block([tiny, -tiny, 0.0]), _int8_block([3.0, -1.5])])
+    codes, alpha = o.quantize_int8_blocks(bits, 64)
+    assert alpha[0] == 0 and np.all(codes[:64] == 0)                       # zero block
+    assert np.isinf(alpha[1]) and list(codes[64:67]) == [127, -127, 0]     # 127 / amax overflows
+    assert np.all(codes[67:128] == 0)
+    assert list(codes[128:130]) == [127, -64]                              # -1.5 * 127/3 = -63.5 -> -64
+    xh = o.dequantize_int8_blocks(codes, alpha, 64)
+    assert np.all(xh[:128] == 0)
+    assert np.signbit(xh[65]) and not np.signbit(xh[64])                   # -127 / inf = -0
+
+
+def test_int8_blocks_reject():
+    with pytest.raises(o.OracleShapeError):
+        o.quantize_int8_blocks(_int8_block([1.0], 64), 32)
+    with pytest.raises(o.OracleShapeError):
+        o.quantize_int8_blocks(_int8_block([1.0], 64)[:60], 64)
+    bad = _int8_block([1.0])
+    bad[5] = 0x7F80                                                        # +Inf
+    with pytest.raises(o.OracleNonFiniteError):
+        o.quantize_int8_blocks(bad, 64)
+
+
 # ---------------------------------------------------------------- the linear layer
 
 def _small_linear(M=3, N=5, K=64, r=2, seed=11):
