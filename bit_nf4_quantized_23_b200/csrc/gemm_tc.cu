@@ -140,6 +140,22 @@ __device__ __forceinline__ void zero_row(uint32_t row_addr) {
     for (int c = 0; c < 8; ++c) st_shared_v4(row_addr + (c << 4), make_uint4(0, 0, 0, 0));
 }
 
+// The same row in a non-swizzled K-major image (rows 16 bytes apart, chunk c of
+// every row LBO bytes after chunk 0): the eight stores take immediate offsets from
+// one address, and a warp's 32 rows fill 512 contiguous bytes per chunk.
+template <uint32_t LBO>
+__device__ __forceinline__ void expand_block_row_kn(uint32_t row_addr, uint4 c0, uint4 c1, const Lut& t) {
+    const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+    for (int c = 0; c < 8; ++c) st_shared_v4(row_addr + c * LBO, expand8(w[c], t));
+}
+
+template <uint32_t LBO>
+__device__ __forceinline__ void zero_row_kn(uint32_t row_addr) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) st_shared_v4(row_addr + c * LBO, make_uint4(0, 0, 0, 0));
+}
+
 // Output tile of CTA t: row tiles run fastest within groups of kRasterGroup of them, so the
 // CTAs resident at one time share a W strip (read from HBM once, then from L2) and keep the
 // group's activation panel resident in L2 across the column tiles.
@@ -251,6 +267,7 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
         const uint32_t idesc = ptx::idesc_set_f16(ptx::idesc_bf16_f32(128, kBN, DX ? 1 : 0), p.f16 != 0);
         const uint64_t adesc0 = ptx::smem_desc_sw128(sA, 16, 1024);
         const uint64_t bdesc0 = DX ? ptx::smem_desc_sw128(sB, 8192, 1024) : ptx::smem_desc_sw128(sB, 16, 1024);
+        const uint64_t bdesc0_kn = ptx::smem_desc_kmajor_none(sB, kBN * 16, 128);   // forward W_hat steps
         bool ok = true;
         int s = 0;
         uint32_t ph = 0;
@@ -262,10 +279,12 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
             ptx::tc_fence_after();
             if (ptx::elect_one_sync()) {
                 const uint64_t ad = adesc0 + ((uint32_t)s * (L::kAStageBytes >> 4));
-                const uint64_t bd = bdesc0 + ((uint32_t)s * (kBStageBytes >> 4));
+                const bool kn = !DX && it < ks0;
+                const uint64_t bd = (kn ? bdesc0_kn : bdesc0) + ((uint32_t)s * (kBStageBytes >> 4));
+                const uint32_t kstep = DX ? (2048 >> 4) : kn ? ((2 * kBN * 16) >> 4) : (32 >> 4);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t bdesc = bd + (DX ? kk * (2048 >> 4) : kk * (32 >> 4));
+                    const uint64_t bdesc = bd + kk * kstep;
 #pragma unroll
                     for (int h = 0; h < NUM_ACC; ++h)
                         ptx::mma_bf16_ss(tmem + h * 256, ad + h * (16384 >> 4) + kk * (32 >> 4), bdesc, idesc,
@@ -291,7 +310,9 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
         const int64_t blocks_per_row = p.WK / 64;
         const uint32_t row = DX ? (uint32_t)(t & 63) : (uint32_t)t;
         const uint32_t kc = DX ? (uint32_t)(t >> 6) : 0u;
-        const uint32_t img = DX ? kc * 8192u + row * 128u : row * 128u;
+        // forward: non-swizzled K-major image (row t at 16 t, chunk c at 4096 c);
+        // dX: 128-byte-swizzled 64-row images, one per K-block, read as an MN-major operand
+        const uint32_t img = DX ? kc * 8192u + row * 128u : row * 16u;
         auto unit_block = [&](int it) -> int64_t {
             const int64_t n = DX ? (int64_t)it * 64 + row : n0 + row;
             const int64_t k = DX ? n0 + (int64_t)kc * 64 : (int64_t)it * 64;
@@ -344,7 +365,8 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
             if (!ok) break;
             const uint32_t row_addr = sB + s * kBStageBytes + img;
             if (blk < 0) {
-                zero_row(row_addr);
+                if (DX) zero_row(row_addr);
+                else zero_row_kn<kBN * 16>(row_addr);
             } else {
                 const uint32_t c_base = sCodes + s * kCodesStageBytes;
                 uint4 c0, c1;
@@ -362,7 +384,8 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
                 }
                 Lut lut;
                 build_lut(lut, c1p, p.tb, p.f16 != 0);
-                expand_block_row(row_addr, row & 7u, c0, c1, lut);
+                if (DX) expand_block_row(row_addr, row & 7u, c0, c1, lut);
+                else expand_block_row_kn<kBN * 16>(row_addr, c0, c1, lut);
             }
             ptx::fence_proxy_async_smem();
             __syncwarp();
@@ -562,7 +585,7 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, const __grid_constant
         // built once and advanced by stage offsets (start address >> 4 in the low 14 bits;
         // every shared address here is below 256 KiB, so no carry leaves them).
         const uint32_t idesc = ptx::idesc_set_f16(ptx::idesc_bf16_f32_ab(128, 16, 0, 0), p.f16 != 0);
-        const uint64_t adesc0 = ptx::smem_desc_sw128(sA, 16, 1024);
+        const uint64_t adesc0 = ptx::smem_desc_kmajor_none(sA, 128 * 16, 128);   // W_hat rows, non-swizzled
         const uint64_t bdesc0 = ptx::smem_desc_sw128(sX, 16, 1024);
         bool ok = true;
         int step = step0, seg = 0;
@@ -585,10 +608,11 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, const __grid_constant
                 const uint64_t ad = adesc0 + ((uint32_t)s * (kDecAStage >> 4));
                 const uint64_t bd = bdesc0 + ((uint32_t)cs * (kDecXStage >> 4));
                 const uint32_t d = tmem + 16u * (uint32_t)a;
+                constexpr uint32_t ak = (2 * 128 * 16) >> 4;       // one K step of 16: two core-matrix columns
                 ptx::mma_bf16_ss(d, ad, bd, idesc, fresh ? 0u : 1u);
-                ptx::mma_bf16_ss(d, ad + 2, bd + 2, idesc, 1u);
-                ptx::mma_bf16_ss(d, ad + 4, bd + 4, idesc, 1u);
-                ptx::mma_bf16_ss(d, ad + 6, bd + 6, idesc, 1u);
+                ptx::mma_bf16_ss(d, ad + ak, bd + 2, idesc, 1u);
+                ptx::mma_bf16_ss(d, ad + 2 * ak, bd + 4, idesc, 1u);
+                ptx::mma_bf16_ss(d, ad + 3 * ak, bd + 6, idesc, 1u);
                 ptx::mma_commit(bar_aempty + 8 * s);
                 ptx::mma_commit(bar_cempty + 8 * cs);
                 if (last) ptx::mma_commit(bar_accfull + 8 * a);   // segment ends: hand the accumulator over
@@ -686,16 +710,16 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, const __grid_constant
             if (!w_ok) atomicMax(p.dbg, 0x50000000u | (uint32_t)i);
             ok = __all_sync(0xffffffffu, w_ok);
             if (!ok) break;
-            const uint32_t row_addr = sA + s * kDecAStage + (uint32_t)t * 128u;
+            const uint32_t row_addr = sA + s * kDecAStage + (uint32_t)t * 16u;   // non-swizzled K-major
             if (cur.tile * 128 + t >= p.N) {
-                zero_row(row_addr);
+                zero_row_kn<128 * 16>(row_addr);
             } else {
                 const uint32_t src = sCodes + cs * kDecCodesStage + (uint32_t)t * 32u;
                 const uint4 x = ld_shared_v4(src);
                 const uint4 y = ld_shared_v4(src + 16u);
                 Lut lut;
                 build_lut(lut, c1p, p.tb, p.f16 != 0);
-                expand_block_row(row_addr, (uint32_t)t & 7u, x, y, lut);
+                expand_block_row_kn<128 * 16>(row_addr, x, y, lut);
             }
             ptx::fence_proxy_async_smem();
             __syncwarp();

@@ -221,6 +221,14 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
            ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
+// The same descriptor for the non-swizzled ("interleaved") K-major layout: 8-row
+// core matrices of 16-byte rows (rows 16 bytes apart), sbo between 8-row groups,
+// lbo between the two K-adjacent core matrices of a 16-element K step.
+__device__ __forceinline__ uint64_t smem_desc_kmajor_none(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+
 // Instruction descriptor of kind::f16 with bf16 A and B, fp32 D, shape M x N;
 // A and B each K-major (0) or MN-major (1).
 __host__ __device__ constexpr uint32_t idesc_bf16_f32_ab(int M, int N, int a_mn, int b_mn) {
