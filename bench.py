@@ -464,6 +464,28 @@ def quantizer_variants(device, peaks, wl):
                     out[key]["quantize_GB/s"] = round(nbytes / (ms * 1e-3) / 1e9, 1)
         nf = out[f"{dist}/nf4/single"]["rel_sq_error"]
         out[f"{dist}/nf4_over_uniform4"] = round(nf / out[f"{dist}/uniform4/single"]["rel_sq_error"], 4)
+        # the 8-bit absmax comparison quantizer (blocks of 64, one fp32 scale each)
+        codes, alpha = q4.qlora_quantize_int8_absmax(W, 64)
+        Wh = q4.qlora_dequantize_int8_absmax(codes, alpha, 64).double()
+        key = f"{dist}/int8_absmax/b64"
+        out[key] = {"rel_sq_error": float(((Wh - w64) ** 2).sum()) / den}
+        if dist == "normal":
+            nbytes = (2.0 + 1.0 + 4 / 64) * N * K
+            Wb = torch.empty_like(W)
+            for name, fn in (("quantize", lambda: q4.qlora_quantize_int8_absmax(W, 64, codes, alpha)),
+                             ("dequantize", lambda: q4.qlora_dequantize_int8_absmax(codes, alpha, 64, out=Wb))):
+                for _ in range(2):
+                    fn()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                for _ in range(10):
+                    fn()
+                b.record()
+                b.synchronize()
+                ms = a.elapsed_time(b) / 10
+                out[key][f"{name}_GB/s"] = round(nbytes / (ms * 1e-3) / 1e9, 1)
+                out[key][f"{name}_frac_of_hbm"] = round(nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3)
+        del codes, alpha, Wh
     del weights
     torch.cuda.empty_cache()
     return out

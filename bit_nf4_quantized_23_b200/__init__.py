@@ -22,7 +22,7 @@ __all__ = [
     "NF4Weight", "QloraError", "CODEBOOKS", "qlora_nf4_sizes", "qlora_nf4_codebook", "qlora_codebook_values",
     "qlora_quantize_nf4_dq",
     "qlora_quantize_nf4_dq_noalloc",
-    "qlora_dequantize", "qlora_merge_lora", "qlora_linear_workspace_size", "qlora_linear_fwd", "qlora_linear_fwd_multi", "qlora_linear_bwd",
+    "qlora_dequantize", "qlora_quantize_int8_absmax", "qlora_dequantize_int8_absmax", "qlora_merge_lora", "qlora_linear_workspace_size", "qlora_linear_fwd", "qlora_linear_fwd_multi", "qlora_linear_bwd",
     "qlora_read_device_errors", "qlora_launch_count", "qlora_timing_enable", "qlora_timing_read",
 ]
 
@@ -162,6 +162,39 @@ def qlora_dequantize(w: NF4Weight, out: torch.Tensor | None = None, stream=None)
     _need(out, w.compute_dtype, "out", (w.N, w.K))
     ws = w.c_struct()
     check(lib().qlora_dequantize(byref(ws), _ptr(out), _stream(stream)), "qlora_dequantize")
+    return out
+
+
+def qlora_quantize_int8_absmax(W: torch.Tensor, blocksize: int = 64, codes: torch.Tensor | None = None,
+                               alpha: torch.Tensor | None = None, stream=None):
+    """Blockwise absmax INT8 of a bf16 tensor: alpha = 127 / max|x| per block of
+    `blocksize` consecutive elements, codes = round half away from zero of x * alpha.
+    Returns (codes int8 shaped like W, alpha fp32 [W.numel() // blocksize])."""
+    _need(W, torch.bfloat16, "W")
+    n = W.numel()
+    if codes is None:
+        codes = torch.empty(W.shape, dtype=torch.int8, device=W.device)
+    if alpha is None:
+        alpha = torch.empty(max(n // blocksize, 1), dtype=torch.float32, device=W.device)
+    _need(codes, torch.int8, "codes", tuple(W.shape))
+    _need(alpha, torch.float32, "alpha")
+    if alpha.numel() * blocksize != n:
+        raise ValueError(f"alpha must hold {n // blocksize} scales")
+    check(lib().qlora_quantize_int8_absmax(_ptr(W), n, blocksize, _ptr(codes), _ptr(alpha), _stream(stream)),
+          "qlora_quantize_int8_absmax")
+    return codes, alpha
+
+
+def qlora_dequantize_int8_absmax(codes: torch.Tensor, alpha: torch.Tensor, blocksize: int = 64,
+                                 dtype=torch.bfloat16, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """x_hat = code / alpha per block, rounded to `dtype` (bf16, fp16 or fp32)."""
+    _need(codes, torch.int8, "codes")
+    _need(alpha, torch.float32, "alpha")
+    if out is None:
+        out = torch.empty(codes.shape, dtype=dtype, device=codes.device)
+    _need(out, dtype, "out", tuple(codes.shape))
+    check(lib().qlora_dequantize_int8_absmax(_ptr(codes), _ptr(alpha), codes.numel(), blocksize, _ptr(out),
+                                             _dtype_code(dtype), _stream(stream)), "qlora_dequantize_int8_absmax")
     return out
 
 

@@ -48,6 +48,8 @@ SIGNATURES = {
     "qlora_linear_fwd_multi": (c_int32, [_W, c_void_p, c_int64, c_void_p, c_void_p, c_int32, c_void_p, c_int32,
                                          c_float, c_void_p, c_int32, c_void_p, c_void_p, c_size_t, c_void_p]),
     "qlora_dequantize": (c_int32, [_W, c_void_p, c_void_p]),
+    "qlora_quantize_int8_absmax": (c_int32, [c_void_p, c_int64, c_int32, c_void_p, c_void_p, c_void_p]),
+    "qlora_dequantize_int8_absmax": (c_int32, [c_void_p, c_void_p, c_int64, c_int32, c_void_p, c_int32, c_void_p]),
     "qlora_linear_workspace_size": (c_int32, [c_int64, c_int64, c_int64, c_int32, POINTER(c_size_t)]),
     "qlora_linear_fwd": (c_int32, [_W, c_void_p, c_int64, c_void_p, c_void_p, c_int32, c_float, c_void_p,
                                    c_int32, c_void_p, c_void_p, c_size_t, c_void_p]),

@@ -20,6 +20,10 @@ size_t quantize_workspace_bytes(int64_t nb1);
 qlora_status launch_quantize(const void* W, int64_t N, int64_t K, const qlora_nf4_weight* out,
                              void* workspace, cudaStream_t stream);
 qlora_status launch_dequantize(const qlora_nf4_weight* w, void* W_out, cudaStream_t stream);
+qlora_status launch_int8_quantize(const void* W, int64_t n, int blocksize, int8_t* codes, float* alpha,
+                                  cudaStream_t s);
+qlora_status launch_int8_dequantize(const int8_t* codes, const float* alpha, int64_t n, int blocksize, void* out,
+                                    int out_dtype, cudaStream_t s);
 uint32_t* device_error_word();
 qlora_status launch_split_hi_lo(const float* V, int64_t M, int r, int R, float scale, void* V2, bool f16,
                                 cudaStream_t s);
@@ -224,6 +228,33 @@ qlora_status qlora_merge_lora(const qlora_nf4_weight* w, const void* A, const vo
     QLORA_TRY(check_dev(B));
     QLORA_TRY(check_dev(W_out));
     return launch_merge(w, A, B, r, alpha / (float)r, W_out, static_cast<cudaStream_t>(stream));
+}
+
+static qlora_status check_int8(int64_t n, int32_t blocksize) {
+    if (blocksize != 64 && blocksize != 128 && blocksize != 256) return QLORA_ERR_UNSUPPORTED;
+    if (n < 1 || n % blocksize != 0) return QLORA_ERR_SHAPE;
+    if (n / 8 > (int64_t)INT32_MAX * 256) return QLORA_ERR_SHAPE;
+    return QLORA_OK;
+}
+
+qlora_status qlora_quantize_int8_absmax(const void* W, int64_t n, int32_t blocksize, int8_t* codes, float* alpha,
+                                        void* stream) {
+    QLORA_TRY(check_dev(W));
+    QLORA_TRY(check_dev(codes));
+    QLORA_TRY(check_dev(alpha));
+    QLORA_TRY(check_int8(n, blocksize));
+    return launch_int8_quantize(W, n, blocksize, codes, alpha, static_cast<cudaStream_t>(stream));
+}
+
+qlora_status qlora_dequantize_int8_absmax(const int8_t* codes, const float* alpha, int64_t n, int32_t blocksize,
+                                          void* out, int32_t out_dtype, void* stream) {
+    QLORA_TRY(check_dev(codes));
+    QLORA_TRY(check_dev(alpha));
+    QLORA_TRY(check_dev(out));
+    QLORA_TRY(check_int8(n, blocksize));
+    if (out_dtype != QLORA_DTYPE_BF16 && out_dtype != QLORA_DTYPE_F16 && out_dtype != QLORA_DTYPE_F32)
+        return QLORA_ERR_INVALID_ARG;
+    return launch_int8_dequantize(codes, alpha, n, blocksize, out, out_dtype, static_cast<cudaStream_t>(stream));
 }
 
 qlora_status qlora_dequantize(const qlora_nf4_weight* w, void* W_out, void* stream) {

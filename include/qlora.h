@@ -18,8 +18,11 @@
  *   [QR]  ainexis.cn, walkthrough of "QLoRA: Efficient Finetuning of Quantized
  *         LLMs", section 4.4: backpropagation passes through the frozen 4-bit
  *         weight into the adapters.
- *   [CH9] mdooai.com, "Ch.09 QLoRA 与量化：缩得更小再微调", section "3. 一个
- *         底座，多个适配器": one shared compressed base, one thin adapter per task.
+ *   [CH9] mdooai.com, "Ch.09 QLoRA 与量化：缩得更小再微调", section "2. INT8
+ *         量化" (the absmax INT8 worked example: scale so that the block's largest
+ *         magnitude maps to 127, store rounded integers, divide by the scale to
+ *         recover) and section "3. 一个底座，多个适配器": one shared compressed
+ *         base, one thin adapter per task.
  *   [Q103] agentalpha.top, "Q103: What is QLoRA, and how does it differ from
  *         LoRA", follow-up 1: after fine-tuning, merge the LoRA weights and
  *         dequantize for fast inference.
@@ -286,6 +289,37 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const void* X, const vo
  */
 qlora_status qlora_merge_lora(const qlora_nf4_weight* w, const void* A, const void* B, int32_t r, float alpha,
                               void* W_out, void* stream);
+
+/*
+ * Blockwise absmax INT8 quantization, the 8-bit comparison quantizer of [CH9]
+ * section "2. INT8 量化" (steps 1-3).  For each block b of `blocksize`
+ * consecutive elements of the flat tensor, in fp32 with round-to-nearest-even:
+ *   alpha[b] = 127 / max|x| (IEEE division); 0 for an all-zero block, +inf
+ *              when max|x| < 127 / FLT_MAX;
+ *   codes[i] = round half away from zero of (x[i] * alpha[b]), clamped to
+ *              [-127, 127]; 0 for x[i] = 0.
+ *   W          device bf16 [n], read;  n >= 1 and n % blocksize == 0.
+ *   blocksize  64, 128 or 256.
+ *   codes      device int8 [n], written;  alpha  device fp32 [n / blocksize], written.
+ * Errors: QLORA_ERR_INVALID_ARG (null pointer), QLORA_ERR_SHAPE (n < 1 or
+ * n % blocksize != 0), QLORA_ERR_UNSUPPORTED (another blocksize),
+ * QLORA_ERR_ALIGN.  A block holding Inf or NaN gets alpha 0 and zero codes and
+ * raises the non-finite device flag (qlora_read_device_errors).
+ */
+qlora_status qlora_quantize_int8_absmax(const void* W, int64_t n, int32_t blocksize, int8_t* codes, float* alpha,
+                                        void* stream);
+
+/*
+ * Dequantize blockwise absmax INT8 ([CH9] section "2. INT8 量化", step 4:
+ * divide by the scale):
+ *   out[i] = fp32(codes[i] / alpha[b]) (IEEE division; 0 when alpha[b] = 0),
+ *            rounded to nearest even into out_dtype.
+ *   out        device [n] of out_dtype (QLORA_DTYPE_BF16, _F16 or _F32), written.
+ * Other arguments and errors as qlora_quantize_int8_absmax; a bad out_dtype
+ * returns QLORA_ERR_INVALID_ARG.
+ */
+qlora_status qlora_dequantize_int8_absmax(const int8_t* codes, const float* alpha, int64_t n, int32_t blocksize,
+                                          void* out, int32_t out_dtype, void* stream);
 
 /*
  * Device error flags raised since the last clear (bit 0: a bounded wait timed

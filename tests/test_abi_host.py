@@ -139,3 +139,17 @@ def test_host_validation_before_launch(L):
     assert L.qlora_linear_bwd(ctypes.byref(w), FAKE, FAKE, 16, FAKE, FAKE, 8, 1.0, None, None, 0, None, FAKE,
                               FAKE, 1 << 30, None) == E["QLORA_ERR_INVALID_ARG"]
     assert L.qlora_launch_count() == launches_before
+
+
+def test_int8_argument_errors_on_the_host(L):
+    fake = ctypes.c_void_p(0x10000)             # aligned, never dereferenced: the checks come first
+    odd = ctypes.c_void_p(0x10004)
+    q, d = L.qlora_quantize_int8_absmax, L.qlora_dequantize_int8_absmax
+    assert q(None, 64, 64, fake, fake, None) == 1                     # null W
+    assert q(odd, 64, 64, fake, fake, None) == 3                      # misaligned
+    assert q(fake, 64, 32, fake, fake, None) == 4                     # blocksize
+    assert q(fake, 100, 64, fake, fake, None) == 2                    # n % blocksize
+    assert q(fake, 0, 64, fake, fake, None) == 2                      # empty
+    assert d(fake, fake, 128, 128, fake, 5, None) == 1                # out dtype
+    assert d(fake, None, 128, 128, fake, 0, None) == 1                # null alpha
+    assert d(fake, fake, 192, 128, fake, 0, None) == 2
