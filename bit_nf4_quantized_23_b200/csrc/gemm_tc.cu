@@ -313,58 +313,52 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
         // forward: non-swizzled K-major image (row t at 16 t, chunk c at 4096 c);
         // dX: 128-byte-swizzled 64-row images, one per K-block, read as an MN-major operand
         const uint32_t img = DX ? kc * 8192u + row * 128u : row * 16u;
-        auto unit_block = [&](int it) -> int64_t {
-            const int64_t n = DX ? (int64_t)it * 64 + row : n0 + row;
-            const int64_t k = DX ? n0 + (int64_t)kc * 64 : (int64_t)it * 64;
-            return (n < p.WN && k < p.WK) ? n * blocks_per_row + (k >> 6) : -1;
+        // The unit of K-step `ahead` (the one whose constants load next): its first-level
+        // block index moves by a fixed stride per step (forward: the next block of the same
+        // W row; dX: the same K-block 64 W rows further), and it exists when the thread's
+        // W row (forward) or K-block (dX) is in range, and in dX its row a_n < N.
+        const bool lane_ok = DX ? (n0 + (int64_t)kc * 64 < p.WK) : (n0 + row < p.WN);
+        const int64_t blk_step = DX ? 64 * blocks_per_row : 1;
+        int64_t a_blk = DX ? (int64_t)row * blocks_per_row + (n0 >> 6) + kc : (n0 + row) * blocks_per_row;
+        int64_t a_n = row;
+        auto const_load = [&](int ahead, bool& v, uint32_t& code, float& c2) {
+            v = lane_ok && ahead < ks0 && (!DX || a_n < p.WN);
+            code = 0;
+            c2 = 0.f;
+            if (v) {
+                if (p.c1f) {   // single-level constants: the queue's c2 slot carries c1
+                    c2 = __ldg(p.c1f + a_blk);
+                } else {
+                    code = __ldg(p.c1_codes + a_blk);
+                    c2 = __ldg(p.c2 + (a_blk >> 8));
+                }
+            }
+            a_blk += blk_step;
+            a_n += 64;
         };
-        int64_t qblk[kGemmPrefetch];
+        bool qv[kGemmPrefetch];
         uint32_t qcode[kGemmPrefetch];
         float qc2[kGemmPrefetch];
 #pragma unroll
-        for (int d = 0; d < kGemmPrefetch; ++d) {
-            qblk[d] = d < ks0 ? unit_block(d) : -1;
-            qcode[d] = 0;
-            qc2[d] = 0.f;
-            if (qblk[d] >= 0) {
-                if (p.c1f) {   // single-level constants: the queue's c2 slot carries c1
-                    qc2[d] = __ldg(p.c1f + qblk[d]);
-                } else {
-                    qcode[d] = __ldg(p.c1_codes + qblk[d]);
-                    qc2[d] = __ldg(p.c2 + (qblk[d] >> 8));
-                }
-            }
-        }
+        for (int d = 0; d < kGemmPrefetch; ++d) const_load(d, qv[d], qcode[d], qc2[d]);
         bool ok = true;
-        for (int it = 0; it < ks0 && ok; ++it) {
-            const int s = it % kStages;
-            const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-            const int64_t blk = qblk[0];
+        int s = 0;
+        uint32_t ph = 0;
+        for (int it = 0; it < ks0 && ok; ++it, s = (s + 1 == kStages) ? 0 : s + 1, ph ^= (s == 0) ? 1u : 0u) {
+            const bool valid = qv[0];
             // c1' = fp32(fp32(v8 c2) + mu) with v8 from the shared E4M3 table, or the stored c1
-            const float c1p = blk < 0 ? 0.f : (p.c1f ? qc2[0] : __fadd_rn(__fmul_rn(e4tab[qcode[0]], qc2[0]), mu));
+            const float c1p = !valid ? 0.f : (p.c1f ? qc2[0] : __fadd_rn(__fmul_rn(e4tab[qcode[0]], qc2[0]), mu));
 #pragma unroll
             for (int d = 0; d + 1 < kGemmPrefetch; ++d) {
-                qblk[d] = qblk[d + 1];
+                qv[d] = qv[d + 1];
                 qcode[d] = qcode[d + 1];
                 qc2[d] = qc2[d + 1];
             }
-            {
-                const int ahead = it + kGemmPrefetch;
-                const int64_t b = ahead < ks0 ? unit_block(ahead) : -1;
-                qblk[kGemmPrefetch - 1] = b;
-                if (b >= 0) {
-                    if (p.c1f) {
-                        qc2[kGemmPrefetch - 1] = __ldg(p.c1f + b);
-                    } else {
-                        qcode[kGemmPrefetch - 1] = __ldg(p.c1_codes + b);
-                        qc2[kGemmPrefetch - 1] = __ldg(p.c2 + (b >> 8));
-                    }
-                }
-            }
+            const_load(it + kGemmPrefetch, qv[kGemmPrefetch - 1], qcode[kGemmPrefetch - 1], qc2[kGemmPrefetch - 1]);
             ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_full_a + 8 * s, ph, abort, p.err));
             if (!ok) break;
             const uint32_t row_addr = sB + s * kBStageBytes + img;
-            if (blk < 0) {
+            if (!valid) {
                 if (DX) zero_row(row_addr);
                 else zero_row_kn<kBN * 16>(row_addr);
             } else {
@@ -477,7 +471,7 @@ constexpr int kDecCtasPerSm = 2;                // ~103 KB of shared memory per 
 constexpr int kDecMaxCtas = 1024;
 constexpr int kDecCodeStages = 6;               // codes + token ring (the HBM stream); even: stage parity = group
 constexpr int kDecStages = 4;                   // dequantized-tile ring; stage parity = group
-constexpr int kDecPrefetch = 4;                 // block constants are loaded this many units (of the group) ahead
+constexpr int kDecPrefetch = 2;                 // block constants are loaded this many units (of the group) ahead
 constexpr uint32_t kDecAStage = 128 * 128;      // W_hat tile [128 rows x 64]
 constexpr uint32_t kDecXStage = 16 * 128;       // X tile [16 tokens x 64], 128-byte swizzled rows (TMA)
 constexpr uint32_t kDecCodesStage = 128 * 32;   // packed codes [128 rows x 32 bytes]
@@ -636,24 +630,31 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, const __grid_constant
         const int64_t nb1 = p.N * (p.K / 64);
         const int64_t kb = p.K / 64;
         const float mu = p.c1f ? 0.f : *p.mu;
-        // a unit cursor: tile, step and the first-level block index of row tile*128 + t at step 0
-        struct Cursor { int64_t tile, rowblk; int step; };
+        // a unit cursor: tile, K-step, the first-level block index of W row tile*128 + t at that
+        // step, and whether that row exists (the last tile may be partial); advancing by `by`
+        // units moves the block index by `by`, plus 128 rows less one tile of steps per tile crossed
+        struct Cursor { int64_t tile, blk; int step; bool row_ok; };
         auto advance = [&](Cursor& c, int by) {
             c.step += by;
-            while (c.step >= S) { c.step -= S; ++c.tile; c.rowblk += 128 * kb; }
+            c.blk += by;
+            while (c.step >= S) {
+                c.step -= S;
+                ++c.tile;
+                c.blk += 128 * kb - S;
+                c.row_ok = c.tile * 128 + t < p.N;
+            }
         };
-        Cursor cur{t0, (t0 * 128 + t) * kb, step0};
+        Cursor cur{t0, (t0 * 128 + t) * kb + step0, step0, t0 * 128 + t < p.N};
         advance(cur, g);
         auto const_load = [&](const Cursor& c, uint32_t& code, float& c2) {
             code = 0; c2 = 0.f;
-            if (c.tile * 128 + t >= p.N) return;
-            const int64_t blk = c.rowblk + c.step;
-            if (blk >= nb1) { atomicOr(p.err, ERR_FLAG_BOUNDS); atomicMax(p.dbg, 0x20000000u); return; }
+            if (!c.row_ok) return;
+            if (c.blk >= nb1) { atomicOr(p.err, ERR_FLAG_BOUNDS); atomicMax(p.dbg, 0x20000000u); return; }
             if (p.c1f) {   // single-level constants: the queue's c2 slot carries c1
-                c2 = __ldg(p.c1f + blk);
+                c2 = __ldg(p.c1f + c.blk);
             } else {
-                code = __ldg(p.c1_codes + blk);
-                c2 = __ldg(p.c2 + (blk >> 8));
+                code = __ldg(p.c1_codes + c.blk);
+                c2 = __ldg(p.c2 + (c.blk >> 8));
             }
         };
         uint32_t qcode[kDecPrefetch];
@@ -711,7 +712,7 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, const __grid_constant
             ok = __all_sync(0xffffffffu, w_ok);
             if (!ok) break;
             const uint32_t row_addr = sA + s * kDecAStage + (uint32_t)t * 16u;   // non-swizzled K-major
-            if (cur.tile * 128 + t >= p.N) {
+            if (!cur.row_ok) {
                 zero_row_kn<128 * 16>(row_addr);
             } else {
                 const uint32_t src = sCodes + cs * kDecCodesStage + (uint32_t)t * 32u;
