@@ -630,23 +630,55 @@ def run_ours(args):
                 "avg_launch_ms": ms_l / n_l if n_l else None}
     breakdown = {k: {"launches": v[0], "ms_per_step": v[1] / args.steps} for k, v in kinds.items()}
 
-    # end to end through the public API with host buffers (pinned), copies inside the timed region
+    # end to end through the public API with host buffers (pinned), copies inside the timed region.
+    # The host-to-device copies run on their own stream in the order the kernels need them
+    # (linear i's W, X, A, B, then the dY of the backward's order); each linear's quantize and
+    # forward wait only for its own inputs, so copying overlaps the work already possible.  Same
+    # calls and the same work as the device-timed step; quantize i runs just before forward i.
     e2e = None
     if not args.no_e2e:
-        host = []
-        for L in lins:
-            for name in ("W", "X", "A", "B", "dY"):
-                t = getattr(L, name)
-                if not any(t is h[0] for h in host):
-                    host.append((t, t.cpu().pin_memory()))
+        pinned = {}
+
+        def host_of(t):
+            if id(t) not in pinned:
+                pinned[id(t)] = (t, t.cpu().pin_memory())
+            return pinned[id(t)][1]
+
+        fwd_in = [[(getattr(L, n), host_of(getattr(L, n))) for n in ("W", "X", "A", "B")] for L in lins]
+        bwd_in = [[(L.dY, host_of(L.dY))] for L in lins]
         grads_host = torch.empty(grads.numel(), dtype=torch.float32).pin_memory()
-        h2d = sum(h.numel() * h.element_size() for _, h in host)
+        h2d = sum(h.numel() * h.element_size() for _, h in pinned.values())
         d2h = grads.numel() * 4
+        copy_stream = torch.cuda.Stream(device=device)
 
         def e2e_step():
-            for dev_t, h in host:
-                dev_t.copy_(h, non_blocking=True)
-            step()
+            cur = torch.cuda.current_stream()
+            copy_stream.wait_stream(cur)                 # after the timer starts and the last step's readers
+            done, ev_f, ev_b = set(), [], {}
+            with torch.cuda.stream(copy_stream):
+                for ins in fwd_in:
+                    for dev_t, h in ins:
+                        if id(dev_t) not in done:        # an X shared by several linears is copied once
+                            dev_t.copy_(h, non_blocking=True)
+                            done.add(id(dev_t))
+                    ev_f.append(torch.cuda.Event())
+                    ev_f[-1].record(copy_stream)
+                for i in reversed(range(len(lins))):
+                    for dev_t, h in bwd_in[i]:
+                        dev_t.copy_(h, non_blocking=True)
+                    ev_b[i] = torch.cuda.Event()
+                    ev_b[i].record(copy_stream)
+            for i, L in enumerate(lins):
+                cur.wait_event(ev_f[i])
+                q4.qlora_quantize_nf4_dq(L.W, out=L.w, workspace=L.qws)
+                q4.qlora_linear_fwd(L.w, L.X, L.A, L.B, wl.r, wl.alpha, out=L.Y, U_out=L.U, workspace=L.lws)
+            for i in reversed(range(len(lins))):
+                L = lins[i]
+                cur.wait_event(ev_b[i])
+                q4.qlora_linear_bwd(L.w, L.X, L.dY, L.A, L.B, wl.r, wl.alpha, U_saved=L.U, dX=L.dX,
+                                    dA=L.dA, dB=L.dB, workspace=L.lws)
+            if world > 1:
+                torch.distributed.all_reduce(grads)
             grads_host.copy_(grads, non_blocking=True)
 
         for _ in range(2):
@@ -658,7 +690,9 @@ def run_ours(args):
             torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
             ms_e2e = float(t.item())
         e2e = {"value": flops_rank * world / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
+               "h2d_GB/s": round(h2d / (ms_e2e * 1e-3) / 1e9, 1),
+               "note": "inputs copied on a second stream in the order the kernels need them, overlapping the work"}
 
     quant_bytes = sum((2.0 + PACKED_BYTES_PER_WEIGHT) * L.N * L.K for L in lins)
     q_ms = kinds["quantize"][1] / args.steps
