@@ -109,10 +109,10 @@ LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int32_t r) {
     l.du2_off = o; o += align_up((size_t)M * 2 * R * 2, 256);
     l.b2_off = o;  o += align_up((size_t)N * 2 * R * 2, 256);
     l.bt_off = o;  o += align_up(R * (size_t)N * 2, 256);
-    size_t part = lora_partial_bytes(M, K, (int)R);
-    part = std::max(part, lora_partial_bytes(M, N, (int)R));
-    part = std::max(part, lora_partial_bytes(K, M, (int)R));
-    part = std::max(part, lora_partial_bytes(N, M, (int)R));
+    size_t part = lora_partial_bytes(M, K, (int)R, false);          // U
+    part = std::max(part, lora_partial_bytes(M, N, (int)R, false));  // dU
+    part = std::max(part, lora_partial_bytes(K, M, (int)R, true));   // dA
+    part = std::max(part, lora_partial_bytes(N, M, (int)R, true));   // dB
     if (M <= kDecodeMaxM) part = std::max(part, decode_partial_bytes(N, K));   // decode partial tiles
     l.part_off = o; o += align_up(part, 256);
     l.total = o;
@@ -129,7 +129,7 @@ qlora_status lora_U(const void* X, const void* A, int64_t M, int64_t K, int32_t 
     g.b_rows = r;
     g.f16 = f16;
     QLORA_TRY(launch_lora_gemm(g, s));
-    const int splits = lora_splits(M, (int)((K + 63) / 64));
+    const int splits = lora_splits(M, (int)((K + 63) / 64), R, false);
     return launch_reduce_rows(partial, splits, M, r, R, 1.f, U, s_lora, U2, f16, s);
 }
 
@@ -399,7 +399,7 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const void* X, const vo
             g.partial = partial;
             g.f16 = f16;
             QLORA_TRY(launch_lora_gemm(g, s));
-            QLORA_TRY(launch_reduce_rows(partial, lora_splits(M, (int)((N + 63) / 64)), M, r, R, scale, dUf, scale,
+            QLORA_TRY(launch_reduce_rows(partial, lora_splits(M, (int)((N + 63) / 64), R, false), M, r, R, scale, dUf, scale,
                                          dU2, f16, s));
         }
         if (dX) {   // dX = dY W_hat + dU A
@@ -416,7 +416,7 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const void* X, const vo
             g.partial = partial;
             g.f16 = f16;
             QLORA_TRY(launch_lora_gemm(g, s));
-            QLORA_TRY(launch_reduce_transposed(partial, lora_splits(K, (int)((M + 63) / 64)), K, r, R, dA, s));
+            QLORA_TRY(launch_reduce_transposed(partial, lora_splits(K, (int)((M + 63) / 64), R, true), K, r, R, dA, s));
         }
         {   // dB = s dY^T U = dY^T (s U)
             TimerScope t(QLORA_TIMER_LORA, s);
@@ -425,7 +425,7 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const void* X, const vo
             g.partial = partial;
             g.f16 = f16;
             QLORA_TRY(launch_lora_gemm(g, s));
-            QLORA_TRY(launch_reduce_rows(partial, lora_splits(N, (int)((M + 63) / 64)), N, r, R, 1.f, dB, 0.f,
+            QLORA_TRY(launch_reduce_rows(partial, lora_splits(N, (int)((M + 63) / 64), R, true), N, r, R, 1.f, dB, 0.f,
                                          nullptr, f16, s));
         }
         return QLORA_OK;

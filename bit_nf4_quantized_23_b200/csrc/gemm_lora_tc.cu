@@ -226,13 +226,28 @@ qlora_status launch_lora(const CUtensorMap& tmA, const CUtensorMap& tmB, LoraGem
 
 }  // namespace
 
-int lora_splits(int64_t rows, int ksteps_total) {
+// CTAs per SM the launch below uses: two when three or more stages fit in half of the
+// shared memory, else one.
+int lora_ctas_per_sm(int R, bool mn_major) {
+    const uint32_t stage = kAStage + (mn_major ? (uint32_t)R * 256u : (uint32_t)R * 128u);
+    return (kMaxSmem / 2 - 2048) / stage >= 3 ? 2 : 1;
+}
+
+// Split count of the reduction: the one with the least waves x (a CTA's fixed cost, about two
+// K-steps of streaming, + its K-steps), the smallest on ties (fewer partial tiles).  A launch a
+// few CTAs past one wave would otherwise run a second, nearly empty wave.
+int lora_splits(int64_t rows, int ksteps_total, int R, bool mn_major) {
     const int64_t tiles = (rows + 127) / 128;
-    int64_t splits = (2 * 148 + tiles - 1) / tiles;
-    if (splits > ksteps_total) splits = ksteps_total;
-    if (splits < 1) splits = 1;
-    const int64_t kps = (ksteps_total + splits - 1) / splits;
-    return (int)((ksteps_total + kps - 1) / kps);
+    const int64_t slots = 148 * (int64_t)lora_ctas_per_sm(R, mn_major);
+    int best = 1;
+    int64_t best_cost = INT64_MAX;
+    for (int s = 1; s <= ksteps_total && s <= 64; ++s) {
+        const int64_t kps = (ksteps_total + s - 1) / s;
+        const int64_t eff = (ksteps_total + kps - 1) / kps;          // splits after rounding kps up
+        const int64_t cost = ((tiles * eff + slots - 1) / slots) * (2 + kps);
+        if (cost < best_cost) { best_cost = cost; best = (int)eff; }
+    }
+    return best;
 }
 
 qlora_status launch_lora_gemm(const LoraGemmArgs& a, cudaStream_t stream) {
@@ -240,7 +255,7 @@ qlora_status launch_lora_gemm(const LoraGemmArgs& a, cudaStream_t stream) {
     p.rows = a.rows;
     p.R = a.R;
     p.ksteps_total = (int)((a.red + 63) / 64);
-    const int splits = lora_splits(a.rows, p.ksteps_total);
+    const int splits = lora_splits(a.rows, p.ksteps_total, a.R, a.mn_major);
     p.ksteps_per_split = (p.ksteps_total + splits - 1) / splits;
     p.partial = a.partial;
     p.f16 = a.f16;
@@ -261,9 +276,9 @@ qlora_status launch_lora_gemm(const LoraGemmArgs& a, cudaStream_t stream) {
     return launch_lora<true>(tmA, tmB, p, splits, stream);
 }
 
-size_t lora_partial_bytes(int64_t rows, int64_t red, int R) {
+size_t lora_partial_bytes(int64_t rows, int64_t red, int R, bool mn_major) {
     const int ks = (int)((red + 63) / 64);
-    return (size_t)lora_splits(rows, ks) * (size_t)rows * (size_t)R * sizeof(float);
+    return (size_t)lora_splits(rows, ks, R, mn_major) * (size_t)rows * (size_t)R * sizeof(float);
 }
 
 }  // namespace qlora

@@ -108,8 +108,8 @@ struct LoraGemmArgs {
 };
 
 qlora_status launch_lora_gemm(const LoraGemmArgs& a, cudaStream_t stream);
-int lora_splits(int64_t rows, int ksteps_total);
-size_t lora_partial_bytes(int64_t rows, int64_t red, int R);
+int lora_splits(int64_t rows, int ksteps_total, int R, bool mn_major);
+size_t lora_partial_bytes(int64_t rows, int64_t red, int R, bool mn_major);
 
 bool make_tmap_2d(CUtensorMap* map, bool bf16, const void* base, uint64_t inner, uint64_t outer,
                   uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128);
