@@ -144,11 +144,36 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- traffic from ncu
 
+def _code_only(text: str) -> str:
+    """C/C++/CUDA source without comments or blank-line and trailing-space differences."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        if text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        elif text[i] in "\"'":                       # string and character literals stay as they are
+            q, j = text[i], i + 1
+            while j < n and text[j] != q:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        else:
+            out.append(text[i])
+            i += 1
+    lines = [ln.rstrip() for ln in "".join(out).splitlines()]
+    return "\n".join(ln for ln in lines if ln)
+
+
 def kernel_source_sha():
+    """Hash of the kernel sources' code (comments ignored): the DRAM counters recorded in
+    profiles/traffic.txt stay valid while it is unchanged."""
     h = hashlib.sha256()
     for p in sorted(glob.glob(os.path.join(ROOT, "bit_nf4_quantized_23_b200", "csrc", "*"))):
-        with open(p, "rb") as f:
-            h.update(f.read())
+        with open(p, encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

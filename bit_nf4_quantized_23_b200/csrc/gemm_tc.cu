@@ -18,16 +18,21 @@
 // one or two 128-row fp32 accumulators (256 TMEM columns each).  K-steps of 64
 // reduction elements; STAGES-deep shared-memory ring:
 //   A stage  [BM x 64] bf16, 128-byte swizzled rows, loaded by TMA;
-//   B stage  [256 x 64] (forward: rows n, K-major) or four [64 x 64] images
-//            (dX: rows = reduction n, MN-major with 64-wide MN chunks 8 KiB
-//            apart), written either by the dequant warps from the NF4 codes
-//            or by TMA for the LoRA segment: the two give identical images;
+//   B stage  forward: [256 x 64] rows n, K-major: written by the dequant warps
+//            as a non-swizzled image (8-row core matrices, chunk c of every row
+//            at 4096 c), or loaded by TMA with 128-byte swizzle for the LoRA
+//            steps (the MMA takes the matching descriptor per step);
+//            dX: four [64 x 64] images (rows = reduction n, MN-major, 64-wide
+//            MN chunks 8 KiB apart, 128-byte swizzled), written by the dequant
+//            warps or by TMA for the LoRA steps, the two alike;
 //   codes    the packed 4-bit codes of the B stage (8 KiB), loaded by TMA.
-// Warp roles (320 threads): warp 0 lane 0 issues TMA; warp 1 owns TMEM and
-// its lane 0 issues tcgen05.mma; warps 2-9 expand NF4 -> bf16 (one NF4 block
-// of 64 weights per thread and K-step, through a 16-entry per-block lookup
-// table held in byte-split registers and selected with byte permutes), then
-// run the epilogue (TMEM -> registers -> global, bf16 or fp32).
+// Warp roles (320 threads): warp 0 issues TMA; warp 1 owns TMEM and issues
+// tcgen05.mma (each loop runs on the whole warp, one elected lane issues);
+// warps 2-9 expand NF4 -> bf16 (one NF4 block of 64 weights per thread and
+// K-step, through a 16-entry per-block lookup table held in byte-split
+// registers and selected with byte permutes), then run the epilogue (TMEM ->
+// registers -> global, bf16 or fp32).  CTAs take output tiles in a grouped
+// order (row tiles fastest within groups of 16) so concurrent CTAs share W.
 // No TMA multicast is used anywhere.
 #include <algorithm>
 
