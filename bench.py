@@ -21,7 +21,6 @@ from __future__ import annotations
 import argparse
 import datetime
 import hashlib
-import glob
 import json
 import os
 import subprocess
@@ -167,12 +166,17 @@ def _code_only(text: str) -> str:
     return "\n".join(ln for ln in lines if ln)
 
 
-def kernel_source_sha():
-    """Hash of the kernel sources' code (comments ignored): the DRAM counters recorded in
+# The fused dequant-GEMM's sources: its device and launch code, its parameter structs, the PTX
+# wrappers and the shared helpers it is compiled from.
+FUSED_GEMM_SOURCES = ("gemm_tc.cu", "gemm_tc.cuh", "qlora_internal.cuh", "tc_ptx.cuh")
+
+
+def kernel_source_sha(files=FUSED_GEMM_SOURCES):
+    """Hash of the fused GEMM's sources' code (comments ignored): the DRAM counters recorded in
     profiles/traffic.txt stay valid while it is unchanged."""
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "bit_nf4_quantized_23_b200", "csrc", "*"))):
-        with open(p, encoding="utf-8") as f:
+    for name in sorted(files):
+        with open(os.path.join(ROOT, "bit_nf4_quantized_23_b200", "csrc", name), encoding="utf-8") as f:
             h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 

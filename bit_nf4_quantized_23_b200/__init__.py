@@ -23,7 +23,7 @@ __all__ = [
     "qlora_quantize_nf4_dq",
     "qlora_quantize_nf4_dq_noalloc",
     "qlora_dequantize", "qlora_quantize_int8_absmax", "qlora_dequantize_int8_absmax", "qlora_merge_lora", "qlora_linear_workspace_size", "qlora_linear_fwd", "qlora_linear_fwd_multi", "qlora_linear_bwd",
-    "qlora_read_device_errors", "qlora_launch_count", "qlora_timing_enable", "qlora_timing_read",
+    "qlora_read_device_errors", "qlora_selftest_bounded_wait", "qlora_launch_count", "qlora_timing_enable", "qlora_timing_read",
 ]
 
 
@@ -316,6 +316,17 @@ def qlora_read_device_errors(clear: bool = True, stream=None) -> int:
     f = c_uint32()
     lib().qlora_read_device_errors(_stream(stream), 1 if clear else 0, byref(f))
     return f.value
+
+
+def qlora_selftest_bounded_wait(limit_us: int, device=None, stream=None):
+    """Run the bounded-wait self-test (a wait that nothing completes, limited to `limit_us`);
+    returns (completed, aborted) as read back from the device.  The timeout device flag is
+    left set for qlora_read_device_errors."""
+    result = torch.zeros(2, dtype=torch.int32, device=device or torch.device("cuda"))
+    check(lib().qlora_selftest_bounded_wait(int(limit_us), _ptr(result), _stream(stream)),
+          "qlora_selftest_bounded_wait")
+    r = result.cpu().tolist()
+    return bool(r[0]), bool(r[1])
 
 
 def qlora_launch_count() -> int:

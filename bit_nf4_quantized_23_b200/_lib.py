@@ -57,6 +57,7 @@ SIGNATURES = {
                                    c_void_p, c_void_p, c_int32, c_void_p, c_void_p, c_void_p, c_size_t,
                                    c_void_p]),
     "qlora_read_device_errors": (c_int32, [c_void_p, c_int32, POINTER(c_uint32)]),
+    "qlora_selftest_bounded_wait": (c_int32, [c_uint32, c_void_p, c_void_p]),
     "qlora_launch_count": (c_uint64, []),
     "qlora_timing_enable": (c_int32, [c_int32]),
     "qlora_timing_read": (c_int32, [c_int32, POINTER(c_uint64), POINTER(ctypes.c_double), c_int32]),

@@ -25,6 +25,7 @@ qlora_status launch_int8_quantize(const void* W, int64_t n, int blocksize, int8_
 qlora_status launch_int8_dequantize(const int8_t* codes, const float* alpha, int64_t n, int blocksize, void* out,
                                     int out_dtype, cudaStream_t s);
 uint32_t* device_error_word();
+qlora_status launch_bounded_wait_probe(uint64_t limit_ns, uint32_t* result, cudaStream_t s);
 qlora_status launch_split_hi_lo(const float* V, int64_t M, int r, int R, float scale, void* V2, bool f16,
                                 cudaStream_t s);
 qlora_status launch_dup_cols(const void* B, int64_t N, int r, int R, void* B2, cudaStream_t s);
@@ -508,6 +509,12 @@ qlora_status qlora_read_device_errors(void* stream, int32_t clear, uint32_t* fla
     if (h[0] & ERR_FLAG_TIMEOUT) return QLORA_ERR_TIMEOUT;
     if (h[0] & ERR_FLAG_NONFINITE) return QLORA_ERR_NONFINITE;
     return QLORA_OK;
+}
+
+qlora_status qlora_selftest_bounded_wait(uint32_t limit_us, uint32_t* result, void* stream) {
+    if (limit_us < 1 || limit_us > 1000000) return QLORA_ERR_INVALID_ARG;
+    QLORA_TRY(check_dev(result));
+    return launch_bounded_wait_probe((uint64_t)limit_us * 1000ull, result, static_cast<cudaStream_t>(stream));
 }
 
 uint64_t qlora_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

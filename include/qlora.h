@@ -329,6 +329,21 @@ qlora_status qlora_dequantize_int8_absmax(const int8_t* codes, const float* alph
  */
 qlora_status qlora_read_device_errors(void* stream, int32_t clear, uint32_t* flags);
 
+/*
+ * Failure-detection self-test of the bounded device waits (no page counterpart).
+ * Launches one thread that waits, through the same bounded mbarrier wait every
+ * kernel of the library uses, on a barrier that nothing completes, with a limit
+ * of `limit_us` microseconds.  The wait gives up, raises the timeout device flag
+ * (read it with qlora_read_device_errors, which then returns QLORA_ERR_TIMEOUT)
+ * and the kernel returns: the context stays usable.  Nothing faults or hangs.
+ *   limit_us  1 .. 1,000,000.
+ *   result    device uint32 [2], written: [0] = 1 if the wait completed (never
+ *             expected), [1] = 1 if the wait set the CTA's abort flag.
+ * Errors: QLORA_ERR_INVALID_ARG (limit out of range, null result),
+ * QLORA_ERR_ALIGN.
+ */
+qlora_status qlora_selftest_bounded_wait(uint32_t limit_us, uint32_t* result, void* stream);
+
 /* Number of kernels this library has launched in this process (host counter). */
 uint64_t qlora_launch_count(void);
 

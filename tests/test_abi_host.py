@@ -153,3 +153,11 @@ def test_int8_argument_errors_on_the_host(L):
     assert d(fake, fake, 128, 128, fake, 5, None) == 1                # out dtype
     assert d(fake, None, 128, 128, fake, 0, None) == 1                # null alpha
     assert d(fake, fake, 192, 128, fake, 0, None) == 2
+
+
+def test_selftest_argument_errors_on_the_host(L):
+    fake = ctypes.c_void_p(0x10000)
+    assert L.qlora_selftest_bounded_wait(0, fake, None) == 1          # limit out of range
+    assert L.qlora_selftest_bounded_wait(1000001, fake, None) == 1
+    assert L.qlora_selftest_bounded_wait(1000, None, None) == 1       # null result
+    assert L.qlora_selftest_bounded_wait(1000, ctypes.c_void_p(0x10004), None) == 3
