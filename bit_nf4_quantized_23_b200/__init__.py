@@ -178,7 +178,7 @@ def qlora_quantize_int8_absmax(W: torch.Tensor, blocksize: int = 64, codes: torc
         alpha = torch.empty(max(n // blocksize, 1), dtype=torch.float32, device=W.device)
     _need(codes, torch.int8, "codes", tuple(W.shape))
     _need(alpha, torch.float32, "alpha")
-    if alpha.numel() * blocksize != n:
+    if blocksize <= 0 or alpha.numel() * blocksize != n:
         raise ValueError(f"alpha must hold {n // blocksize} scales")
     check(lib().qlora_quantize_int8_absmax(_ptr(W), n, blocksize, _ptr(codes), _ptr(alpha), _stream(stream)),
           "qlora_quantize_int8_absmax")
@@ -190,6 +190,8 @@ def qlora_dequantize_int8_absmax(codes: torch.Tensor, alpha: torch.Tensor, block
     """x_hat = code / alpha per block, rounded to `dtype` (bf16, fp16 or fp32)."""
     _need(codes, torch.int8, "codes")
     _need(alpha, torch.float32, "alpha")
+    if blocksize <= 0 or alpha.numel() * blocksize != codes.numel():
+        raise ValueError(f"alpha must hold codes.numel() / blocksize = {codes.numel() // max(blocksize, 1)} scales")
     if out is None:
         out = torch.empty(codes.shape, dtype=dtype, device=codes.device)
     _need(out, dtype, "out", tuple(codes.shape))

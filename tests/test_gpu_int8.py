@@ -174,3 +174,9 @@ def test_int8_dequantize_every_code_at_every_reachable_scale():
     got = q4.qlora_dequantize_int8_absmax(torch.from_numpy(codes).to(DEV), torch.from_numpy(alpha).to(DEV),
                                           256, torch.float32).cpu().numpy()
     assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+
+
+def test_int8_dequantize_rejects_a_short_scale_vector():
+    codes, alpha = q4.qlora_quantize_int8_absmax(torch.zeros(256, dtype=torch.bfloat16, device=DEV), 64)
+    with pytest.raises(ValueError):
+        q4.qlora_dequantize_int8_absmax(codes, alpha[:3], 64)
