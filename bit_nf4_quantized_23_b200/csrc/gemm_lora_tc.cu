@@ -233,12 +233,17 @@ int lora_ctas_per_sm(int R, bool mn_major) {
     return (kMaxSmem / 2 - 2048) / stage >= 3 ? 2 : 1;
 }
 
+// SMs assumed by the split rule: B200's 148.  The split count fixes the size of the partial
+// buffer in the caller's workspace, so it must not depend on which device is current when the
+// size is queried.
+constexpr int64_t kSplitRuleSms = 148;
+
 // Split count of the reduction: the one with the least waves x (a CTA's fixed cost, about two
 // K-steps of streaming, + its K-steps), the smallest on ties (fewer partial tiles).  A launch a
 // few CTAs past one wave would otherwise run a second, nearly empty wave.
 int lora_splits(int64_t rows, int ksteps_total, int R, bool mn_major) {
     const int64_t tiles = (rows + 127) / 128;
-    const int64_t slots = 148 * (int64_t)lora_ctas_per_sm(R, mn_major);
+    const int64_t slots = kSplitRuleSms * (int64_t)lora_ctas_per_sm(R, mn_major);
     int best = 1;
     int64_t best_cost = INT64_MAX;
     for (int s = 1; s <= ksteps_total && s <= 64; ++s) {
