@@ -551,6 +551,15 @@ def linear_backward(X, dY, W_hat, A, B, alpha: float, r: int):
     return {"dX": dX, "dA": dA, "dB": dB, "dU": dU}
 
 
+def lora_gradients(X, dY, A, B, alpha: float, r: int):
+    """The adapter gradients alone, for shapes where the full dX is too large to form:
+    dA = (s dY B)^T X and dB = s dY^T (X A^T), in fp64 (the same formulas as linear_backward)."""
+    Xd, dYd, Ad, Bd = _f64(X), _f64(dY), _f64(A), _f64(B)
+    s = lora_scale(alpha, r)
+    dU = s * (dYd @ Bd)
+    return {"dA": dU.T @ Xd, "dB": s * (dYd.T @ (Xd @ Ad.T))}
+
+
 def forward_rows(X, W_hat, A, B, alpha, r, rows):
     """Y for a subset of token rows (the reference for large shapes)."""
     Xs = _f64(X)[rows]

@@ -48,6 +48,31 @@ def test_codebook_shape_zero_and_endpoints():
     assert (Q < 0).sum() == 7 and (Q > 0).sum() == 8
 
 
+def test_codebook_values_match_the_printed_table():
+    # The values written down independently of the oracle (tests/golden/nf4_codebook_values.txt).
+    g = read_golden("nf4_codebook_values.txt")
+    printed = np.array(g["values"], dtype=np.float64)
+    assert printed.shape == (16,)
+    assert np.max(np.abs(o.nf4_codebook_f64() - printed)) <= g["print_precision"] + 1e-12
+    assert np.max(np.abs(Q.astype(np.float64) - printed)) <= g["print_precision"] + 2 ** -24
+
+
+def test_planted_delta_and_spacing_mistakes_miss_the_printed_table():
+    printed = np.array(read_golden("nf4_codebook_values.txt")["values"], dtype=np.float64)
+    tol = read_golden("nf4_codebook_values.txt")["print_precision"]
+
+    def book(delta, pos_div=8.0, neg_div=7.0):
+        pos = [delta - j * (delta - 0.5) / pos_div for j in range(8)]
+        neg = [delta - j * (delta - 0.5) / neg_div for j in range(7)]
+        v = sorted([o.phi_inv_stdlib(p) for p in pos] + [-o.phi_inv_stdlib(p) for p in neg] + [0.0])
+        return np.array(v) / max(v)
+
+    assert np.max(np.abs(book(o.NF4_DELTA) - printed)) <= tol + 1e-12
+    for wrong in (book(0.5 * ((1 - 1 / 31) + (1 - 1 / 32))), book(0.5 * ((1 - 1 / 30) + (1 - 1 / 33))),
+                  book(1 - 1 / 30), book(o.NF4_DELTA, pos_div=7.0), book(o.NF4_DELTA, neg_div=8.0)):
+        assert np.max(np.abs(wrong - printed)) > 100 * tol
+
+
 def test_codebook_equal_probability_mass_per_half():
     # [SD] section 3: each grid point covers the same probability mass of N(0,1).
     q64 = o.nf4_codebook_f64()
@@ -585,6 +610,14 @@ def test_row_subsets_match_full():
                        o.linear_forward(X, Wh, A, B, 4.0, 2)[0][rows], rtol=1e-14, atol=0)
     assert np.allclose(o.backward_dx_rows(dY, Wh, A, B, 4.0, 2, rows),
                        o.linear_backward(X, dY, Wh, A, B, 4.0, 2)["dX"][rows], rtol=1e-14, atol=0)
+
+
+def test_lora_gradients_equal_the_full_backward():
+    X, Wh, A, B, dY = _small_linear(M=7, N=5, K=128, r=3)
+    full = o.linear_backward(X, dY, Wh, A, B, 6.0, 3)
+    part = o.lora_gradients(X, dY, A, B, 6.0, 3)
+    for k in ("dA", "dB"):
+        assert np.allclose(part[k], full[k], rtol=1e-13, atol=1e-15)
 
 
 def test_row_and_column_samplers_match_full_quantize():
