@@ -79,6 +79,38 @@ class NF4Weight:
         return NF4WeightC(self.codes.data_ptr(), p(self.c1_codes), p(self.c2), p(self.mu), self.N, self.K,
                           64, 256, CODEBOOKS[self.codebook], _dtype_code(self.compute_dtype), p(self.c1))
 
+    _BUFFERS = ("codes", "c1_codes", "c2", "mu", "c1")
+
+    def state_dict(self) -> dict:
+        """Host copies of the stored buffers plus the shape and settings that give them meaning:
+        a checkpoint of the frozen quantized weight (torch.save can write it as is)."""
+        d = {"N": self.N, "K": self.K, "codebook": self.codebook, "blocksize": 64, "blocksize2": 256,
+             "compute_dtype": str(self.compute_dtype).replace("torch.", "")}
+        for name in self._BUFFERS:
+            t = getattr(self, name)
+            d[name] = None if t is None else t.detach().to("cpu", copy=True)
+        return d
+
+    @classmethod
+    def from_state_dict(cls, d: dict, device="cuda") -> "NF4Weight":
+        """Rebuild a weight from state_dict() output: the buffers are copied to `device` byte for byte
+        after their sizes are checked against the shape."""
+        N, K = int(d["N"]), int(d["K"])
+        if d.get("blocksize", 64) != 64 or d.get("blocksize2", 256) != 256:
+            raise ValueError("only blocksize 64 and blocksize2 256 are defined")
+        dtype = {"bfloat16": torch.bfloat16, "float16": torch.float16}[d["compute_dtype"]]
+        ref = cls.empty(N, K, device, d["codebook"], d.get("c1") is None, dtype)
+        for name in cls._BUFFERS:
+            t, src = getattr(ref, name), d.get(name)
+            if (t is None) != (src is None):
+                raise ValueError(f"buffer {name!r} does not match the stored settings")
+            if t is not None:
+                if src.dtype != t.dtype or src.numel() != t.numel():
+                    raise ValueError(f"buffer {name!r}: expected {t.numel()} x {t.dtype}, got "
+                                     f"{src.numel()} x {src.dtype}")
+                t.copy_(src.reshape(t.shape))
+        return ref
+
     @staticmethod
     def empty(N: int, K: int, device="cuda", codebook: str = "nf4", double_quant: bool = True,
               compute_dtype: torch.dtype = torch.bfloat16) -> "NF4Weight":
