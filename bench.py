@@ -33,6 +33,9 @@ sys.path.insert(0, ROOT)
 
 METRIC = "QLoRA linear fwd+bwd TFLOP/s and small-M GB/s, as fraction of B200 roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+NOMINAL_HBM_GBS = 8000.0          # HBM3e, the 8 TB/s figure
+NOMINAL_BF16_TFLOPS = 2250.0      # dense bf16 tensor-core peak (NVIDIA's 4.5 PFLOP/s figure is with 2:4 sparsity)
+AT_MAX_CLOCK = 0.97               # median SM clock at or above this share of the maximum: not power-capped
 L2_FLUSH_BYTES = 256 << 20
 PACKED_BYTES_PER_WEIGHT = 0.5 + 1 / 64 + 4 / (64 * 256)     # codes + E4M3 constants + c2
 ALU_OPS_PER_WEIGHT = 2.5        # exact bf16 table expansion: 19 permute/logic ops per 8 weights + 8 per 64-weight table
@@ -306,15 +309,29 @@ def setup_workload(wl, rank, device):
         L.U = torch.empty(M, wl.r, dtype=torch.float32, device=device)
         L.dX = torch.empty(M, K, dtype=torch.bfloat16, device=device)
         lins.append(L)
-    n_grad = sum(wl.r * L.K + L.N * wl.r for L in lins)
-    grads = torch.empty(n_grad, dtype=torch.float32, device=device)
-    off = 0
-    for L in lins:
-        L.dA = grads[off:off + wl.r * L.K].view(wl.r, L.K)
-        off += wl.r * L.K
-        L.dB = grads[off:off + L.N * wl.r].view(L.N, wl.r)
-        off += L.N * wl.r
+    grads = torch.empty(grad_buffer_numel(wl), dtype=torch.float32, device=device)
+    for L, (dA, dB) in zip(lins, grad_views(wl, grads)):
+        L.dA, L.dB = dA, dB
     return lins, grads
+
+
+def grad_buffer_numel(wl):
+    """Length of the flat fp32 buffer that holds every linear's LoRA gradients."""
+    return sum(wl.r * K + N * wl.r for N, K in wl.linears)
+
+
+def grad_views(wl, grads):
+    """Per linear (dA [r,K], dB [N,r]) as views of the flat buffer, linear after linear, dA first.
+    Data parallelism all-reduces this one buffer per step (one collective for all linears)."""
+    views, off = [], 0
+    for N, K in wl.linears:
+        dA = grads[off:off + wl.r * K].view(wl.r, K)
+        off += wl.r * K
+        dB = grads[off:off + N * wl.r].view(N, wl.r)
+        off += N * wl.r
+        views.append((dA, dB))
+    assert off == grads.numel()
+    return views
 
 
 def make_step(wl, lins, grads, world):
@@ -401,6 +418,7 @@ def decode_sweep(device, peaks):
                 "call_us": round(ms * 1e3, 2), "call_GB/s": round(wbytes / (ms * 1e-3) / 1e9, 1),
                 "kernel_us": round(kms * 1e3, 2), "kernel_GB/s": round(wbytes / (kms * 1e-3) / 1e9, 1),
                 "kernel_frac_of_hbm": round(wbytes / (kms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3),
+                "kernel_frac_of_nominal": round(wbytes / (kms * 1e-3) / 1e9 / NOMINAL_HBM_GBS, 3),
                 "kernel_frac_of_alu_roofline": round(wbytes / (kms * 1e-3) / 1e9 / alu_gbs, 3)}
         if i == len(wl.linears) - 1:
             # one base, many adapters: 16 tokens, each on its own adapter, same weight copies
@@ -455,7 +473,7 @@ def dequant_rate(device, peaks, wl):
     ms = a.elapsed_time(b) / reps
     gbs = (PACKED_BYTES_PER_WEIGHT + 2.0) * N * K / (ms * 1e-3) / 1e9
     return {"shape": [N, K], "us": round(ms * 1e3, 1), "GB/s": round(gbs, 1),
-            "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 3),
+            "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 3), "frac_of_nominal": round(gbs / NOMINAL_HBM_GBS, 3),
             "bytes_per_weight": round(PACKED_BYTES_PER_WEIGHT + 2.0, 6)}
 
 
@@ -590,6 +608,91 @@ def compute_dtype_compare(device, peaks, wl):
     return out
 
 
+def e2e_resident(wl, lins, grads, world, device, flush, stream, steps, flops_rank, barrier):
+    import torch
+    import bit_nf4_quantized_23_b200 as q4
+    pinned = {}
+
+    def host_of(t):
+        if id(t) not in pinned:
+            pinned[id(t)] = t.cpu().pin_memory()
+        return pinned[id(t)]
+
+    x_in = [(L.X, host_of(L.X)) for L in lins]
+    dy_in = [(L.dY, host_of(L.dY)) for L in lins]
+    y_out = [(L.Y, torch.empty(L.Y.shape, dtype=L.Y.dtype).pin_memory()) for L in lins]
+    dx_out = [(L.dX, torch.empty(L.dX.shape, dtype=L.dX.dtype).pin_memory()) for L in lins]
+    grads_host = torch.empty(grads.numel(), dtype=torch.float32).pin_memory()
+    h2d = sum(h.numel() * h.element_size() for h in pinned.values())
+    d2h = sum(h.numel() * h.element_size() for _, h in y_out + dx_out) + grads.numel() * 4
+    s_in, s_out = torch.cuda.Stream(device=device), torch.cuda.Stream(device=device)
+
+    def step():
+        cur = torch.cuda.current_stream()
+        s_in.wait_stream(cur)                            # after the timer starts and the last step's readers
+        s_out.wait_stream(cur)
+        done, ev_x, ev_dy = set(), [], {}
+        with torch.cuda.stream(s_in):
+            for dev_t, h in x_in:
+                if id(dev_t) not in done:                # an X shared by several linears is copied once
+                    dev_t.copy_(h, non_blocking=True)
+                    done.add(id(dev_t))
+                ev_x.append(torch.cuda.Event())
+                ev_x[-1].record(s_in)
+            for i in reversed(range(len(lins))):
+                dy_in[i][0].copy_(dy_in[i][1], non_blocking=True)
+                ev_dy[i] = torch.cuda.Event()
+                ev_dy[i].record(s_in)
+        for i, L in enumerate(lins):
+            cur.wait_event(ev_x[i])
+            q4.qlora_linear_fwd(L.w, L.X, L.A, L.B, wl.r, wl.alpha, out=L.Y, U_out=L.U, workspace=L.lws)
+            s_out.wait_stream(cur)
+            with torch.cuda.stream(s_out):
+                y_out[i][1].copy_(y_out[i][0], non_blocking=True)
+        for i in reversed(range(len(lins))):
+            L = lins[i]
+            cur.wait_event(ev_dy[i])
+            q4.qlora_linear_bwd(L.w, L.X, L.dY, L.A, L.B, wl.r, wl.alpha, U_saved=L.U, dX=L.dX,
+                                dA=L.dA, dB=L.dB, workspace=L.lws)
+            s_out.wait_stream(cur)
+            with torch.cuda.stream(s_out):
+                dx_out[i][1].copy_(dx_out[i][0], non_blocking=True)
+        if world > 1:
+            torch.distributed.all_reduce(grads)
+        s_out.wait_stream(cur)
+        with torch.cuda.stream(s_out):
+            grads_host.copy_(grads, non_blocking=True)
+        cur.wait_stream(s_out)                           # the step ends when its results are on the host
+
+    for _ in range(2):
+        step()
+    barrier()
+    n = max(1, min(steps, 5))
+    ms = timed_steps(step, n, flush, stream) / n
+    if world > 1:
+        t = torch.tensor([ms], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": flops_rank * world / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
+            "note": "weights quantized once before the timed region; per step X and dY in, Y, dX, dA and dB "
+                    "out through pinned host memory, overlapping the forward and backward of all linears"}
+
+
+def tensor_peak(peaks, peak_kind, clk):
+    """The bf16 peak a kernel timed in the step is compared with: the burst figure when the SM clock
+    stayed at its maximum during the timed steps (the kernel ran unthrottled), else the sustained
+    figure measured under the power cap."""
+    if peak_kind != "measured":
+        return peaks["bf16_tflops"], "fallback bf16 (burst)"
+    mhz, mx = clk.get("sm_mhz"), clk.get("sm_max_mhz")
+    if mhz and mx and mhz >= AT_MAX_CLOCK * mx:
+        return peaks["bf16_tflops"], (f"measured bf16 burst (MEASURED_PEAKS.json): median SM clock {mhz:.0f} "
+                                      f"of max {mx:.0f} MHz during the timed steps")
+    return peaks["bf16_tflops_sustained"], (f"measured bf16 sustained (MEASURED_PEAKS.json): median SM clock "
+                                            f"{mhz} of max {mx} MHz during the timed steps")
+
+
 def run_ours(args):
     import torch
     import bit_nf4_quantized_23_b200 as q4
@@ -649,14 +752,20 @@ def run_ours(args):
     n_l, ms_l = kinds[dom]
     per_launch_flops = cand[dom] / len(lins)
     achieved = per_launch_flops / (ms_l / n_l * 1e-3) / 1e12 if n_l else None
-    peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    peak, peak_source = tensor_peak(peaks, peak_kind, clk)
+    frac = lambda v, p: round(v / p, 4) if (v and p) else None
     roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": (achieved / peak) if achieved else None,
-                "peak_source": f"{peak_kind} bf16 sustained (MEASURED_PEAKS.json)" if peak_kind == "measured"
-                else "fallback",
+                "frac": frac(achieved, peak), "peak_source": peak_source,
+                "frac_burst": frac(achieved, peaks.get("bf16_tflops")),
+                "frac_sustained": frac(achieved, peaks.get("bf16_tflops_sustained")),
+                "frac_nominal": frac(achieved, NOMINAL_BF16_TFLOPS),
                 "traffic": recorded_traffic(dom),
                 "per_launch_flops": per_launch_flops, "launches": n_l,
                 "avg_launch_ms": ms_l / n_l if n_l else None}
+    step_fractions = {"frac_burst": frac(value / world, peaks.get("bf16_tflops")),
+                      "frac_sustained": frac(value / world, peaks.get("bf16_tflops_sustained")),
+                      "frac_nominal": frac(value / world, NOMINAL_BF16_TFLOPS),
+                      "note": "whole step (quantize included in the time, not in the flops) per GPU"}
     breakdown = {k: {"launches": v[0], "ms_per_step": v[1] / args.steps} for k, v in kinds.items()}
 
     # end to end through the public API with host buffers (pinned), copies inside the timed region.
@@ -723,10 +832,19 @@ def run_ours(args):
                "h2d_GB/s": round(h2d / (ms_e2e * 1e-3) / 1e9, 1),
                "note": "inputs copied on a second stream in the order the kernels need them, overlapping the work"}
 
+    # end to end with the quantized weights resident (a training step after the one-time quantize):
+    # per step the activations X and upstream gradients dY come in from pinned host memory, and Y,
+    # dX and the LoRA gradients go back out.  Copies in run on one side stream in the order the
+    # kernels need them, copies out on another as soon as each result is written.
+    e2e_res = None
+    if not args.no_e2e:
+        e2e_res = e2e_resident(wl, lins, grads, world, device, flush, stream, args.steps, flops_rank, barrier)
+
     quant_bytes = sum((2.0 + PACKED_BYTES_PER_WEIGHT) * L.N * L.K for L in lins)
     q_ms = kinds["quantize"][1] / args.steps
     hbm = {"quantize": {"GB/s": round(quant_bytes / (q_ms * 1e-3) / 1e9, 1),
                         "frac_of_hbm": round(quant_bytes / (q_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3),
+                        "frac_of_nominal": round(quant_bytes / (q_ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS, 3),
                         "ms_per_step": round(q_ms, 4), "bytes_per_weight": round(2.0 + PACKED_BYTES_PER_WEIGHT, 6),
                         "source": "live CUDA events over the timed steps (7 calls per step)"}}
     decode = variants = merge = dtypes = None
@@ -758,7 +876,8 @@ def run_ours(args):
                        "l2": "flushed before every timed step (256 MiB write, outside the timed region)",
                        "step": "quantize all 7 weights + fwd + bwd of all 7 linears"
                                + (" + NCCL all-reduce of dA/dB" if world > 1 else "")},
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+            "roofline": roofline, "step_fractions": step_fractions, "cpu_baseline": cpu, "e2e": e2e,
+            "e2e_resident": e2e_res, "gpu_launches": launches,
             "clocks": clk, "kernels": breakdown, "hbm_bound_ops": hbm, "decode_small_m": decode,
             "quantizer_variants": variants, "merge_requantize": merge, "compute_dtype": dtypes}
     print(json.dumps(line), flush=True)

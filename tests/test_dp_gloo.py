@@ -60,6 +60,57 @@ def test_sharded_lora_gradients_all_reduce_to_full_batch(tmp_path):
     assert np.allclose(reduced, full, rtol=1e-12, atol=1e-12)
 
 
+# A multi-linear workload shaped like the decoder block (square, wide and tall linears; gate and
+# up share their input), small enough for the oracle: the flat gradient buffer of bench.py.
+BLOCK = si.Workload("dp_block", ((64, 64), (64, 64), (192, 64), (192, 64), (64, 192)), 24, 4, 8.0,
+                    dist="t5_outliers")
+
+
+def _block_problem():
+    lins = []
+    for i, (n, k) in enumerate(BLOCK.linears):
+        qw = o.quantize_nf4_dq(si.bf16_bits(si.weight(BLOCK, i)))
+        Wh = o.dequantize(qw["codes"], qw["c1_codes"], qw["c2"], qw["mu"], n, k)
+        A, B = (si.bf16_bits(t) for t in si.lora(BLOCK, i))
+        X = si.bf16_bits(si.activations(BLOCK, k, BLOCK.M))
+        dY = si.bf16_bits(si.grad_output(BLOCK, i, BLOCK.M))
+        lins.append((Wh, X, A, B, dY))
+    return lins
+
+
+def _block_worker(rank, port, out_path):
+    import bench
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=WORLD)
+    rows = np.array_split(np.arange(BLOCK.M), WORLD)[rank]
+    grads = torch.full((bench.grad_buffer_numel(BLOCK),), float("nan"), dtype=torch.float64)
+    for (Wh, X, A, B, dY), (dA, dB) in zip(_block_problem(), bench.grad_views(BLOCK, grads)):
+        g = o.linear_backward(X[rows], dY[rows], Wh, A, B, BLOCK.alpha, BLOCK.r)
+        dA.copy_(torch.from_numpy(g["dA"]))
+        dB.copy_(torch.from_numpy(g["dB"]))
+    dist.all_reduce(grads)                      # the one collective of a data-parallel step
+    if rank == 0:
+        np.save(out_path, grads.numpy())
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_bench_gradient_buffer_all_reduces_to_every_linears_full_batch_gradients(tmp_path):
+    import bench
+    out = str(tmp_path / "grads.npy")
+    mp.spawn(_block_worker, args=(_free_port(), out), nprocs=WORLD, join=True)
+    reduced = torch.from_numpy(np.load(out))
+    assert torch.isfinite(reduced).all()           # every element of the buffer belongs to a view
+    views = bench.grad_views(BLOCK, reduced)
+    assert len(views) == len(BLOCK.linears)
+    for (Wh, X, A, B, dY), (dA, dB) in zip(_block_problem(), views):
+        g = o.linear_backward(X, dY, Wh, A, B, BLOCK.alpha, BLOCK.r)
+        assert dA.shape == g["dA"].shape and dB.shape == g["dB"].shape
+        assert np.allclose(dA.numpy(), g["dA"], rtol=1e-12, atol=1e-12)
+        assert np.allclose(dB.numpy(), g["dB"], rtol=1e-12, atol=1e-12)
+
+
 def test_weak_scaling_accounting():
     import bench
     wl = si.WORKLOADS["block65b"]
