@@ -37,14 +37,7 @@ qlora_status launch_reduce_rows(const float* partial, int splits, int64_t rows, 
 qlora_status launch_reduce_transposed(const float* partial, int splits, int64_t rows, int r, int R, float* out,
                                       cudaStream_t s);
 
-namespace {
-
-std::atomic<uint64_t> g_launches{0};
-
-inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
-
+// Argument checks shared by the entry points (declared in qlora_internal.cuh).
 qlora_status check_blocks(int32_t bs, int32_t bs2) {
     return (bs == 64 && bs2 == 256) ? QLORA_OK : QLORA_ERR_UNSUPPORTED;
 }
@@ -77,6 +70,12 @@ qlora_status check_dev(const void* p) {
     if (!p) return QLORA_ERR_INVALID_ARG;
     return aligned16(p) ? QLORA_OK : QLORA_ERR_ALIGN;
 }
+
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 qlora_status check_lora(int64_t M, int32_t r, float alpha) {
     if (M < 1 || M > (int64_t(1) << 31)) return QLORA_ERR_SHAPE;

@@ -40,6 +40,15 @@ const QuantBuckets& host_buckets(int codebook = QLORA_CODEBOOK_NF4);
 // Host side: count of kernels launched by this library (api.cu).
 void note_launches(int n);
 
+// Host side: argument checks of the entry points (api.cu).  Each returns QLORA_OK or the status
+// the entry point reports: blocksizes (UNSUPPORTED), shape (SHAPE), a weight descriptor (pointers,
+// alignment, codebook, compute dtype), a device pointer (non-null, 16-byte aligned).
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+qlora_status check_blocks(int32_t bs, int32_t bs2);
+qlora_status check_shape(int64_t N, int64_t K);
+qlora_status check_weight(const qlora_nf4_weight* w);
+qlora_status check_dev(const void* p);
+
 // Device error flag word (one per device that loaded the library).  Kernels in
 // quantize.cu set it directly; other kernels get its address as an argument.
 enum : uint32_t { ERR_FLAG_TIMEOUT = 1u, ERR_FLAG_NONFINITE = 2u, ERR_FLAG_BOUNDS = 4u };

@@ -24,6 +24,7 @@
 #include <mutex>
 
 #include "qlora_internal.cuh"
+#include "timing.cuh"
 
 namespace qlora {
 
@@ -61,8 +62,6 @@ void* scratch_address(qlora_status* st) {
     return addr[dev];
 }
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
 }  // namespace
 }  // namespace qlora
 
@@ -70,21 +69,18 @@ extern "C" qlora_status qlora_quantize_nf4_dq_noalloc(const void* W, int64_t N, 
                                                       int32_t blocksize, int32_t blocksize2,
                                                       const qlora_nf4_weight* out, void* stream) {
     using namespace qlora;
-    if (blocksize != 64 || blocksize2 != 256) return QLORA_ERR_UNSUPPORTED;
+    // the same checks as qlora_quantize_nf4_dq, with the size limit ahead of the pointer checks
+    QLORA_TRY(check_blocks(blocksize, blocksize2));
     if (N < 1 || K < 1 || K % 64 != 0) return QLORA_ERR_SHAPE;
     if (N > kNoAllocMaxWeights / K) return QLORA_ERR_TOO_LARGE;
-    if (!W || !out || !out->codes) return QLORA_ERR_INVALID_ARG;
-    if (out->codebook != QLORA_CODEBOOK_NF4 && out->codebook != QLORA_CODEBOOK_UNIFORM4) return QLORA_ERR_INVALID_ARG;
-    if (out->compute_dtype != QLORA_DTYPE_BF16 && out->compute_dtype != QLORA_DTYPE_F16) return QLORA_ERR_INVALID_ARG;
-    if (!out->c1 && (!out->c1_codes || !out->c2 || !out->mu)) return QLORA_ERR_INVALID_ARG;
-    if (!aligned16(W) || !aligned16(out->codes)) return QLORA_ERR_ALIGN;
-    if (out->c1 ? !aligned16(out->c1)
-                : (!aligned16(out->c1_codes) || !aligned16(out->c2) || !aligned16(out->mu)))
-        return QLORA_ERR_ALIGN;
-    if (out->N != N || out->K != K || out->blocksize != 64 || out->blocksize2 != 256) return QLORA_ERR_SHAPE;
+    QLORA_TRY(check_shape(N, K));
+    QLORA_TRY(check_dev(W));
+    QLORA_TRY(check_weight(out));
+    if (out->N != N || out->K != K) return QLORA_ERR_SHAPE;
     if (quantize_workspace_bytes(N * K / 64) > kNoAllocScratchBytes) return QLORA_ERR_TOO_LARGE;
     qlora_status st = QLORA_OK;
     void* scratch = scratch_address(&st);
     if (st != QLORA_OK) return st;
+    TimerScope t(QLORA_TIMER_QUANTIZE, static_cast<cudaStream_t>(stream));
     return launch_quantize(W, N, K, out, scratch, static_cast<cudaStream_t>(stream));
 }

@@ -5,11 +5,11 @@ memory when they quantize (a plugin whose host framework owns all device
 memory and passes only input and output pointers, or a path that must not call
 cudaMalloc/cudaFree).  It keeps its scratch in a static device array of the
 library.  This file is collected last so that a run stopping at the first
-failure has run every other test first; it also passes alone in a fresh process.
+failure has run every other test first; it also passes alone in a fresh process
+(the module fixture builds the library first).
 """
 import ctypes
 
-import numpy as np
 import pytest
 import torch
 
@@ -18,6 +18,20 @@ import synthetic_inputs as si
 from bit_nf4_quantized_23_b200 import _lib
 
 pytestmark = pytest.mark.gpu
+
+# both codebooks, with and without double quantization: with it off the block constants are the
+# output itself and the scratch holds only the partial sums of the mean
+VARIANTS = [("nf4", True), ("uniform4", True), ("nf4", False), ("uniform4", False)]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib_built():
+    from bit_nf4_quantized_23_b200.build import build
+    build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    torch.cuda.set_device(torch.device("cuda:0"))
+    q4.qlora_read_device_errors(clear=True)
+    yield
 
 
 def _noalloc(W, out):
@@ -29,28 +43,32 @@ def _noalloc(W, out):
 
 def _same(a: q4.NF4Weight, b: q4.NF4Weight):
     # integer and bit outputs: exact equality is the tolerance
-    assert torch.equal(a.codes, b.codes)
-    assert torch.equal(a.c1_codes, b.c1_codes)
-    assert torch.equal(a.c2.view(torch.int32), b.c2.view(torch.int32))
-    assert torch.equal(a.mu.view(torch.int32), b.mu.view(torch.int32))
+    for name in ("codes", "c1_codes", "c2", "mu", "c1"):
+        x, y = getattr(a, name), getattr(b, name)
+        assert (x is None) == (y is None), name
+        if x is not None:
+            assert torch.equal(x.view(torch.uint8), y.view(torch.uint8)), name
 
 
-def test_noalloc_matches_workspace_quantize_on_two_calls_in_a_row():
-    from bit_nf4_quantized_23_b200.build import build
-    build()
+def _poison(w: q4.NF4Weight):
+    for name in ("codes", "c1_codes", "c2", "mu", "c1"):
+        t = getattr(w, name)
+        if t is not None:
+            t.view(torch.uint8).fill_(0xAB)
+
+
+@pytest.mark.parametrize("codebook,dq", VARIANTS)
+def test_noalloc_matches_workspace_quantize_on_two_calls_in_a_row(codebook, dq):
     dev = torch.device("cuda:0")
-    torch.cuda.set_device(dev)
     # two different tensors back to back: the second call must not see the first's scratch
     cases = [si.custom_linear(8192, 8192, 1, 1, seed=101, dist="t5")[0],
              si.custom_linear(300, 4160, 1, 1, seed=102)[0]]
     for W_cpu in cases:
         W = W_cpu.to(dev)
         N, K = W.shape
-        ref = q4.qlora_quantize_nf4_dq(W)
-        out = q4.NF4Weight.empty(N, K, dev)
-        for t in (out.codes, out.c1_codes):
-            t.fill_(0xAB)
-        out.c2.fill_(float("nan"))
+        ref = q4.qlora_quantize_nf4_dq(W, codebook=codebook, double_quant=dq)
+        out = q4.NF4Weight.empty(N, K, dev, codebook=codebook, double_quant=dq)
+        _poison(out)
         assert _noalloc(W, out) == 0
         torch.cuda.synchronize()
         _same(out, ref)
