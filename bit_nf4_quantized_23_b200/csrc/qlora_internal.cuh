@@ -100,6 +100,25 @@ __device__ __forceinline__ uint32_t pack16x2_rn(float a, float b, bool f16) {
     return f16 ? pack_f16x2_rn(a, b) : pack_bf16x2_rn(a, b);
 }
 
+// Packed fp32 pairs (sm_100 .f32x2 arithmetic): each element is rounded to nearest even on its
+// own, exactly as the scalar __fmul_rn / __fmaf_rn, but one instruction serves two elements.
+__device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 fma2_rn(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
 // Exact value of an FP8 E4M3 (finite-only) code: sign, 4-bit exponent with
 // bias 7, 3-bit mantissa; exponent field 0 holds the subnormals m * 2^-9.
 __device__ __forceinline__ float e4m3_to_f32(uint32_t c) {

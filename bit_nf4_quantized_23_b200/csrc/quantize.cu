@@ -68,12 +68,15 @@ __device__ __forceinline__ float div_markstein(float w, float m, float y) {
 // of a warp never meet in a shared-memory bank.  The shared address of entry k
 // is table + 8*(32k + lane) = 256 * bits(y) + lane_off (mod 2^32) with
 // lane_off = table + 8*lane - 256 * 0x4B400000, one multiply-add.
-__device__ __forceinline__ uint32_t nf4_code(float x, uint32_t lane_off) {
-    const float y = __fmaf_rn(x, 64.f, 12582976.f);               // 1.5 * 2^23 + 64: bits 0x4B400000 + k
+__device__ __forceinline__ uint32_t nf4_code_at(float x, float y, uint32_t lane_off) {
     const uint32_t addr = __float_as_uint(y) * 256u + lane_off;
     float thr, base;
     asm("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(thr), "=f"(base) : "r"(addr));
     return (uint32_t)__float_as_int(base) + (x > thr ? 1u : 0u);
+}
+
+__device__ __forceinline__ uint32_t nf4_code(float x, uint32_t lane_off) {
+    return nf4_code_at(x, __fmaf_rn(x, 64.f, 12582976.f), lane_off);   // 1.5 * 2^23 + 64: bits 0x4B400000 + k
 }
 
 // One pass over W.  Persistent CTAs loop over chunks of 128 consecutive NF4
@@ -121,16 +124,23 @@ nf4_quantize_blocks(const uint4* __restrict__ W, int64_t nb1, uint4* __restrict_
                 // weights are coded in the order 6,7,4,5,2,3,0,1 of each group of 8 so that
                 // word = 16 * word + code leaves weight 2j in the high nibble of byte j
                 if ((m >= 7.8886091e-31f) && (m <= 1.2676506e30f)) {   // 2^-100 .. 2^100: Markstein division
+                    // the two weights of each 32-bit word go through the division and the bucket
+                    // FMA as one packed pair (the same per-element roundings as the scalar steps)
                     const float y = __frcp_rn(m);
+                    const float2 y2 = make_float2(y, y), nm2 = make_float2(-m, -m);
+                    const float2 k64 = make_float2(64.f, 64.f), kb = make_float2(12582976.f, 12582976.f);
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         uint32_t word = 0;
 #pragma unroll
-                        for (int jj = 0; jj < 8; ++jj) {
-                            const int i = (6 - 2 * (jj >> 1)) + (jj & 1);
-                            const uint32_t pair = w[4 * q + (i >> 1)];
-                            const float v = __uint_as_float((i & 1) ? (pair & 0xFFFF0000u) : (pair << 16));
-                            word = word * 16u + nf4_code(div_markstein(v, m, y), lane_off);
+                        for (int pp = 3; pp >= 0; --pp) {              // elements (6,7), (4,5), (2,3), (0,1)
+                            const uint32_t pair = w[4 * q + pp];
+                            const float2 v = make_float2(__uint_as_float(pair << 16),
+                                                         __uint_as_float(pair & 0xFFFF0000u));
+                            const float2 q0 = mul2_rn(v, y2);
+                            const float2 x = fma2_rn(fma2_rn(nm2, q0, v), y2, q0);   // Markstein, per element
+                            const float2 b = fma2_rn(x, k64, kb);
+                            word = word * 256u + nf4_code_at(x.x, b.x, lane_off) * 16u + nf4_code_at(x.y, b.y, lane_off);
                         }
                         out[q] = word;
                     }
