@@ -57,6 +57,8 @@ def parse_args():
     p.add_argument("--shape", default="2048,22016,8192", help="M,N,K for --case")
     p.add_argument("--rank", type=int, default=64, help="LoRA rank for --case")
     p.add_argument("--reps", type=int, default=3)
+    p.add_argument("--only", choices=["decode", "hbm"], default=None,
+                   help="measurement mode: print only the small-M sweep or the quantize/dequantize rates")
     return p.parse_args()
 
 
@@ -914,10 +916,51 @@ def run_case(args):
     return 0
 
 
+def run_only(args):
+    """One auxiliary measurement on its own (for quick A/B runs): the small-M sweep, or the
+    quantize (7 block weights) and dequantize rates."""
+    import torch
+    import bit_nf4_quantized_23_b200 as q4
+    import synthetic_inputs as si
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    q4._lib.lib()
+    peaks, _ = load_peaks()
+    wl = si.WORKLOADS[args.workload]
+    if args.only == "decode":
+        out = decode_sweep(device, peaks)
+    else:
+        lins, grads = setup_workload(wl, 0, device)
+        for L in lins:
+            q4.qlora_quantize_nf4_dq(L.W, out=L.w, workspace=L.qws)
+        flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+        total_ms = 0.0
+        for _ in range(args.steps):
+            flush_buf.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for L in lins:
+                q4.qlora_quantize_nf4_dq(L.W, out=L.w, workspace=L.qws)
+            b.record()
+            b.synchronize()
+            total_ms += a.elapsed_time(b)
+        q_ms = total_ms / args.steps
+        nbytes = sum((2.0 + PACKED_BYTES_PER_WEIGHT) * L.N * L.K for L in lins)
+        out = {"quantize_7_weights": {"ms": round(q_ms, 4), "GB/s": round(nbytes / (q_ms * 1e-3) / 1e9, 1),
+                                      "frac_of_hbm": round(nbytes / (q_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3)}}
+        del lins, grads
+        torch.cuda.empty_cache()
+        out["dequantize"] = dequant_rate(device, peaks, wl)
+    print(json.dumps({"only": args.only, **out}), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.case:
         return run_case(args)
+    if args.only:
+        return run_only(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

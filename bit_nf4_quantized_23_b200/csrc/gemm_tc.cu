@@ -85,9 +85,12 @@ struct Lut {
 
 __device__ __forceinline__ void build_lut(Lut& t, float c1p, const NF4Tables& tb, bool f16) {
     uint32_t P[8];   // entries 2j, 2j+1 rounded to the compute dtype (bf16 or fp16), packed
+    const float2 c2p = make_float2(c1p, c1p);
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-        P[j] = pack16x2_rn(__fmul_rn(tb.q[2 * j], c1p), __fmul_rn(tb.q[2 * j + 1], c1p), f16);
+    for (int j = 0; j < 8; ++j) {
+        const float2 e = mul2_rn(make_float2(tb.q[2 * j], tb.q[2 * j + 1]), c2p);   // fp32(q * c1'), per element
+        P[j] = pack16x2_rn(e.x, e.y, f16);
+    }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         t.L[j] = prmt(P[2 * j], P[2 * j + 1], 0x6420);
@@ -463,7 +466,9 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
 // the shape.  A CTA's range crosses tiles: each (tile, CTA) piece is a
 // segment, accumulated in one of two TMEM accumulators and written as an fp32
 // partial tile to slot tile + CTA; decode_fixup then sums each tile's slots in
-// CTA order (deterministic) and adds the LoRA term s U B^T in fp32.
+// CTA order (deterministic) and adds the LoRA term s U B^T in fp32.  U = X A^T
+// itself is computed by the producer warps of the CTAs (one fp32 dot product per
+// CTA and turn) while their first code tiles are on the way.
 // Warp roles (320 threads): warp 0 lane 0 streams each unit's packed codes and
 // token tile through a TMA ring (a ring slot is freed by the MMA that read it);
 // warp 1 owns TMEM and issues tcgen05.mma; warps 2-9 are two producer groups of
@@ -488,7 +493,8 @@ constexpr uint32_t kDecOffBars = kDecOffE4 + 256 * 4;
 constexpr uint32_t kDecNumBars = 2 * kDecCodeStages + 2 * kDecStages + 5;
 constexpr uint32_t kDecOffSlot = kDecOffBars + kDecNumBars * 8;
 constexpr uint32_t kDecOffAbort = kDecOffSlot + 4;
-constexpr uint32_t kDecAlloc = kDecOffAbort + 4 + 1024;
+constexpr uint32_t kDecOffRed = kDecOffAbort + 4;             // [8] fp32: per-warp sums of one U entry
+constexpr uint32_t kDecAlloc = kDecOffRed + 32 + 1024;
 constexpr uint32_t kDecSlotFloats = 16 * 128;   // one partial tile: [16 tokens][128 rows] fp32
 static_assert(kDecCodeStages % 2 == 0 && kDecStages % 2 == 0, "ring stages alternate between the two groups");
 static_assert(2 * (kDecAlloc + 1024) <= 233472, "two CTAs per SM");
@@ -550,6 +556,7 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, const __grid_constant
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    grid_dependency_wait();                                   // inputs written by the previous kernel
 
     if (warp == 0) {
         // unit i: codes and token tile into ring slot i % kDecCodeStages, once the MMA that
@@ -629,6 +636,61 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, const __grid_constant
         }
         __syncwarp();
     } else {
+        // U = X A^T (fp32): dot products blockIdx.x, blockIdx.x + G, ... of the r*M, each over the 256
+        // producer threads (16-byte chunks c = t, t + 256, ...; four in flight), then a fixed-order
+        // reduction (xor shuffles, then the eight warp sums in order).  With per-token adapters token m
+        // uses A[aidx[m]]; a token without one (-1) gets U = 0, an index >= n raises the BOUNDS flag.
+        {
+            const int tp = threadIdx.x - 64;
+            float* red = reinterpret_cast<float*>(gbase + kDecOffRed);
+            const int64_t n_dot = (int64_t)p.r * p.M;
+            for (int64_t idx = blockIdx.x; idx < n_dot; idx += gridDim.x) {
+                const int m = (int)(idx / p.r), j = (int)(idx % p.r);
+                int64_t arow = j;
+                bool have = true;
+                if (p.aidx) {
+                    const int a = p.aidx[m];
+                    have = a >= 0 && a < p.n_adapters;
+                    if (a >= p.n_adapters && tp == 0) atomicOr(p.err, ERR_FLAG_BOUNDS);
+                    arow = (int64_t)a * p.r + j;
+                }
+                float acc = 0.f;
+                if (have) {
+                    const uint4* xr = p.X + (int64_t)m * p.K8;
+                    const uint4* ar = p.A + arow * p.K8;
+                    for (int64_t c0 = tp; c0 < p.K8; c0 += 4 * 256) {
+                        uint4 xv[4], av[4];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const int64_t c = c0 + q * 256;
+                            xv[q] = c < p.K8 ? __ldg(xr + c) : make_uint4(0, 0, 0, 0);
+                            av[q] = c < p.K8 ? __ldg(ar + c) : make_uint4(0, 0, 0, 0);
+                        }
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const uint32_t xw[4] = {xv[q].x, xv[q].y, xv[q].z, xv[q].w};
+                            const uint32_t aw[4] = {av[q].x, av[q].y, av[q].z, av[q].w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                acc = __fmaf_rn(from16(xw[e] & 0xFFFFu, p.f16), from16(aw[e] & 0xFFFFu, p.f16), acc);
+                                acc = __fmaf_rn(from16(xw[e] >> 16, p.f16), from16(aw[e] >> 16, p.f16), acc);
+                            }
+                        }
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, o));
+                if (lane == 0) red[warp - 2] = acc;
+                asm volatile("bar.sync 1, 256;" ::: "memory");   // the 8 producer warps
+                if (tp == 0) {
+                    float sum = 0.f;
+                    for (int w = 0; w < 8; ++w) sum = __fadd_rn(sum, red[w]);
+                    p.U[(int64_t)m * p.r + j] = have ? sum : 0.f;
+                }
+                asm volatile("bar.sync 1, 256;" ::: "memory");
+            }
+        }
+
         // producer group g takes units g, g + 2, ...; thread t expands W row tile*128 + t
         const int g = (warp - 2) >> 2;
         const int t = threadIdx.x - 64 - 128 * g;
@@ -744,78 +806,30 @@ tc_decode_nf4(const __grid_constant__ CUtensorMap tmCodes, const __grid_constant
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, 32);
     }
-    // U (the previous kernel) is not read here, but the fixup that follows reads it: this
-    // grid completes only after U's grid has
-    if (threadIdx.x == 0) grid_dependency_wait();
-}
-
-// U[m, j] = sum_k X[m, k] A[j, k] in fp32 (one CTA per (j, m); fixed reduction order).  With
-// per-token adapters (aidx), token m uses A[aidx[m]] and a token without one (-1) gets U = 0.
-__global__ void __launch_bounds__(256)
-decode_lora_u(const uint4* __restrict__ X, const uint4* __restrict__ A, int64_t K8, int r, float* __restrict__ U,
-              const int32_t* __restrict__ aidx, int n_adapters, uint32_t* err, bool f16) {
-    allow_dependents();                                       // the dequant GEMM does not read U
-    const int j = blockIdx.x, m = blockIdx.y;
-    int64_t arow = j;
-    if (aidx) {
-        const int a = aidx[m];
-        if (a < 0 || a >= n_adapters) {                       // no adapter (or an index out of range)
-            if (a >= n_adapters && threadIdx.x == 0) atomicOr(err, ERR_FLAG_BOUNDS);
-            if (threadIdx.x == 0) U[(int64_t)m * r + j] = 0.f;
-            return;
-        }
-        arow = (int64_t)a * r + j;
-    }
-    const uint4* xr = X + (int64_t)m * K8;
-    const uint4* ar = A + arow * K8;
-    float acc = 0.f;
-    for (int64_t c0 = threadIdx.x; c0 < K8; c0 += 4 * 256) {
-        uint4 xv[4], av[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {                         // four 16-byte chunks in flight per thread
-            const int64_t c = c0 + q * 256;
-            xv[q] = c < K8 ? __ldg(xr + c) : make_uint4(0, 0, 0, 0);
-            av[q] = c < K8 ? __ldg(ar + c) : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const uint32_t xw[4] = {xv[q].x, xv[q].y, xv[q].z, xv[q].w};
-            const uint32_t aw[4] = {av[q].x, av[q].y, av[q].z, av[q].w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                acc = __fmaf_rn(from16(xw[e] & 0xFFFFu, f16), from16(aw[e] & 0xFFFFu, f16), acc);
-                acc = __fmaf_rn(from16(xw[e] >> 16, f16), from16(aw[e] >> 16, f16), acc);
-            }
-        }
-    }
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, o));
-    __shared__ float ws[8];
-    if ((threadIdx.x & 31) == 0) ws[threadIdx.x >> 5] = acc;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        float s = 0.f;
-        for (int w = 0; w < 8; ++w) s = __fadd_rn(s, ws[w]);
-        U[(int64_t)m * r + j] = s;
-    }
 }
 
 // Y[m, n] = sum over the CTAs b covering tile n / 128 of partial[tile + b][m][n % 128] (in b
-// order) + scale * sum_j U[m, j] B[n, j], converted to the output type.  One CTA per tile;
-// every group of loads is issued back to back (the kernel is latency-bound, not bandwidth-bound).
+// order) + scale * sum_j U[m, j] B[n, j], converted to the output type.  CTA (tile, y) covers the
+// tile's 128 rows for tokens 4y .. 4y+3; the slots' loads are issued eight slots at a time, so a
+// tile split over a few CTAs costs one round trip to memory (the kernel is latency-bound).
+constexpr int kFixTokens = 4;
+constexpr int kFixSlotBatch = 8;
+
 __global__ void __launch_bounds__(128)
 decode_fixup(const float* __restrict__ partial, int64_t units, int64_t G, int S, int64_t M, int64_t N,
              const float* __restrict__ U, const uint16_t* __restrict__ B, int r, float scale, void* out, int out_f32,
              const int32_t* __restrict__ aidx, int n_adapters, bool f16) {
-    extern __shared__ float us[];                             // us[j * 16 + m] = U[m, j]
-    __shared__ int32_t tok_adapter[16];
+    extern __shared__ float us[];                             // us[j * 4 + q] = U[m0 + q, j]
+    __shared__ int32_t tok_adapter[kFixTokens];
+    const int m0 = (int)blockIdx.y * kFixTokens;
     grid_dependency_wait();                                   // partial tiles and U are complete
-    for (int i = threadIdx.x; i < r * 16; i += 128) {
-        const int j = i >> 4, m = i & 15;
+    for (int i = threadIdx.x; i < r * kFixTokens; i += 128) {
+        const int j = i / kFixTokens, m = m0 + i % kFixTokens;
         us[i] = m < M ? U[(int64_t)m * r + j] : 0.f;
     }
-    if (threadIdx.x < 16) {
-        const int a = (aidx && threadIdx.x < M) ? aidx[threadIdx.x] : 0;
+    if (threadIdx.x < kFixTokens) {
+        const int m = m0 + (int)threadIdx.x;
+        const int a = (aidx && m < M) ? aidx[m] : 0;
         tok_adapter[threadIdx.x] = (a >= 0 && a < n_adapters) ? a : -1;
     }
     __syncthreads();
@@ -829,62 +843,67 @@ decode_fixup(const float* __restrict__ partial, int64_t units, int64_t G, int S,
         return b;
     };
     const int64_t ba = cta_of(tile * S), bz = cta_of(tile * S + S - 1);
-    float acc[16];
+    const int nm = (int)(M - m0 < kFixTokens ? M - m0 : kFixTokens);
+    float acc[kFixTokens];
 #pragma unroll
-    for (int m = 0; m < 16; ++m) acc[m] = 0.f;
-    for (int64_t b = ba; b <= bz; ++b) {
-        const float* pp = partial + (tile + b) * kDecSlotFloats + threadIdx.x;
-        float v[16];
+    for (int q = 0; q < kFixTokens; ++q) acc[q] = 0.f;
+    for (int64_t b0 = ba; b0 <= bz; b0 += kFixSlotBatch) {
+        float v[kFixSlotBatch][kFixTokens];
 #pragma unroll
-        for (int m = 0; m < 16; ++m) v[m] = m < M ? pp[m * 128] : 0.f;
+        for (int s = 0; s < kFixSlotBatch; ++s) {
+            const float* pp = partial + (tile + b0 + s) * kDecSlotFloats + (int64_t)m0 * 128 + threadIdx.x;
 #pragma unroll
-        for (int m = 0; m < 16; ++m) acc[m] = __fadd_rn(acc[m], v[m]);
+            for (int q = 0; q < kFixTokens; ++q) v[s][q] = (b0 + s <= bz && q < nm) ? pp[q * 128] : 0.f;
+        }
+#pragma unroll
+        for (int s = 0; s < kFixSlotBatch; ++s)
+#pragma unroll
+            for (int q = 0; q < kFixTokens; ++q)
+                if (b0 + s <= bz) acc[q] = __fadd_rn(acc[q], v[s][q]);
     }
-    float lora[16];
+    float lora[kFixTokens];
 #pragma unroll
-    for (int m = 0; m < 16; ++m) lora[m] = 0.f;
+    for (int q = 0; q < kFixTokens; ++q) lora[q] = 0.f;
     if (aidx) {
-        // per-token adapters: lora[m] = sum_j U[m, j] B[a(m)][n, j] (ascending j), 0 without one
+        // per-token adapters: lora[q] = sum_j U[m, j] B[a(m)][n, j] (ascending j), 0 without one
 #pragma unroll
-        for (int m = 0; m < 16; ++m) {
-            const int a = m < M ? tok_adapter[m] : -1;
+        for (int q = 0; q < kFixTokens; ++q) {
+            const int a = q < nm ? tok_adapter[q] : -1;
             if (a < 0) continue;
             const uint16_t* br = B + ((int64_t)a * N + n) * r;
             float d = 0.f;
             for (int j0 = 0; j0 < r; j0 += 8) {
                 float bv[8];
 #pragma unroll
-                for (int q = 0; q < 8; ++q) bv[q] = j0 + q < r ? from16(br[j0 + q], f16) : 0.f;
+                for (int k = 0; k < 8; ++k) bv[k] = j0 + k < r ? from16(br[j0 + k], f16) : 0.f;
 #pragma unroll
-                for (int q = 0; q < 8; ++q)
-                    if (j0 + q < r) d = __fmaf_rn(us[(j0 + q) * 16 + m], bv[q], d);
+                for (int k = 0; k < 8; ++k)
+                    if (j0 + k < r) d = __fmaf_rn(us[(j0 + k) * kFixTokens + q], bv[k], d);
             }
-            lora[m] = d;
+            lora[q] = d;
         }
-    }
-    const uint16_t* brow = B + n * r;
-    for (int j0 = 0; j0 < (aidx ? 0 : r); j0 += 8) {
-        float bv[8];
+    } else {
+        const uint16_t* brow = B + n * r;
+        for (int j0 = 0; j0 < r; j0 += 8) {
+            float bv[8];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) bv[q] = j0 + q < r ? from16(brow[j0 + q], f16) : 0.f;
+            for (int k = 0; k < 8; ++k) bv[k] = j0 + k < r ? from16(brow[j0 + k], f16) : 0.f;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            if (j0 + q >= r) continue;
-            const float4* uj = reinterpret_cast<const float4*>(us + (j0 + q) * 16);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const float4 u4 = uj[c];
-                lora[4 * c + 0] = __fmaf_rn(u4.x, bv[q], lora[4 * c + 0]);
-                lora[4 * c + 1] = __fmaf_rn(u4.y, bv[q], lora[4 * c + 1]);
-                lora[4 * c + 2] = __fmaf_rn(u4.z, bv[q], lora[4 * c + 2]);
-                lora[4 * c + 3] = __fmaf_rn(u4.w, bv[q], lora[4 * c + 3]);
+            for (int k = 0; k < 8; ++k) {
+                if (j0 + k >= r) continue;
+                const float4 u4 = *reinterpret_cast<const float4*>(us + (j0 + k) * kFixTokens);
+                lora[0] = __fmaf_rn(u4.x, bv[k], lora[0]);
+                lora[1] = __fmaf_rn(u4.y, bv[k], lora[1]);
+                lora[2] = __fmaf_rn(u4.z, bv[k], lora[2]);
+                lora[3] = __fmaf_rn(u4.w, bv[k], lora[3]);
             }
         }
     }
 #pragma unroll
-    for (int m = 0; m < 16; ++m) {
-        if (m < M) {
-            const float y = __fmaf_rn(scale, lora[m], acc[m]);
+    for (int q = 0; q < kFixTokens; ++q) {
+        if (q < nm) {
+            const int64_t m = m0 + q;
+            const float y = __fmaf_rn(scale, lora[q], acc[q]);
             if (out_f32) static_cast<float*>(out)[m * N + n] = y;
             else static_cast<uint16_t*>(out)[m * N + n] = (uint16_t)to16_rn(y, f16);
         }
@@ -988,16 +1007,22 @@ qlora_status launch_tc_decode(const DecodeArgs& a, cudaStream_t stream) {
             return QLORA_ERR_CUDA;
         configured = true;
     }
-    decode_lora_u<<<dim3((unsigned)a.r, (unsigned)a.M), 256, 0, stream>>>(
-        static_cast<const uint4*>(a.X), static_cast<const uint4*>(a.A), K / 8, a.r, a.U, a.aidx, a.n_adapters, p.err,
-        p.f16 != 0);
-    QLORA_CHECK_LAUNCH();
-    // the three kernels are chained with programmatic dependent launch (the dequant GEMM
-    // overlaps the U kernel and the launch gaps; see grid_dependency_wait in each)
+    p.X = static_cast<const uint4*>(a.X);
+    p.A = static_cast<const uint4*>(a.A);
+    p.K8 = K / 8;
+    p.r = a.r;
+    p.U = a.U;
+    p.aidx = a.aidx;
+    p.n_adapters = a.n_adapters;
+    // both kernels are launched with programmatic dependent launch: the dequant GEMM's prologue
+    // (barriers, TMEM, tables) overlaps the previous kernel's tail and it waits for that kernel
+    // before reading anything; the fixup waits for the GEMM's partial tiles and U
     (void)launch_dependent(tc_decode_nf4, dim3((unsigned)p.grid), dim3(kDecThreads), kDecAlloc, stream, tmCodes,
                            tmX, p);
     QLORA_CHECK_LAUNCH();
-    (void)launch_dependent(decode_fixup, dim3((unsigned)tiles), dim3(128), (size_t)a.r * 16 * sizeof(float), stream,
+    const unsigned ty = (unsigned)((a.M + kFixTokens - 1) / kFixTokens);
+    (void)launch_dependent(decode_fixup, dim3((unsigned)tiles, ty), dim3(128),
+                           (size_t)a.r * kFixTokens * sizeof(float), stream,
                            (const float*)a.partial, p.units, p.grid, (int)p.ksteps, a.M, N, (const float*)a.U,
                            static_cast<const uint16_t*>(a.B), a.r, a.scale, a.out, (int)a.out_f32, a.aidx,
                            (int)a.n_adapters, p.f16 != 0);

@@ -58,6 +58,14 @@ struct DecodeParams {
     uint32_t* err;
     uint32_t* dbg;          // second device word: where a self-check or a wait gave up
     NF4Tables tb;
+    // U = X A^T, computed by the producer warps before their first unit (written for the fixup)
+    const uint4* X;         // [M, K] 16-bit, as 16-byte chunks
+    const uint4* A;         // [r, K] (or [n_adapters, r, K] with aidx)
+    int64_t K8;             // K / 8
+    int32_t r;
+    float* U;               // [M, r] fp32
+    const int32_t* aidx;    // per-token adapter (-1: none) or NULL
+    int32_t n_adapters;
 };
 
 struct DecodeArgs {
