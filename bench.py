@@ -769,6 +769,8 @@ def run_ours(args):
                       "frac_nominal": frac(value / world, NOMINAL_BF16_TFLOPS),
                       "note": "whole step (quantize included in the time, not in the flops) per GPU"}
     breakdown = {k: {"launches": v[0], "ms_per_step": v[1] / args.steps} for k, v in kinds.items()}
+    breakdown["lora"]["note"] = ("event time of the LoRA-side kernels; the backward's dA/dB run on a side stream "
+                                 "beside the dX GEMM, so part of this time overlaps it")
 
     # end to end through the public API with host buffers (pinned), copies inside the timed region.
     # The host-to-device copies run on their own stream in the order the kernels need them

@@ -133,6 +133,55 @@ qlora_status lora_U(const void* X, const void* A, int64_t M, int64_t K, int32_t 
     return launch_reduce_rows(partial, splits, M, r, R, 1.f, U, s_lora, U2, f16, s);
 }
 
+// The backward's adapter-gradient work (dA, dB and their reductions) runs on a second stream of
+// the lowest priority, forked from the caller's stream after dU is ready and joined back before
+// the call returns: it reads only dU, X, dY and U, none of which the dX GEMM writes, so it can
+// fill the SMs that the dX GEMM's last wave of tiles leaves idle.  One side stream per device,
+// created on first use; calls from several host threads share it (their adapter work is then
+// serialised on it, which is correct but not concurrent).
+cudaStream_t side_stream() {
+    static std::mutex mu;
+    static cudaStream_t streams[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!streams[dev]) {
+        int least = 0, greatest = 0;
+        if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) return nullptr;
+        cudaStream_t st = nullptr;
+        if (cudaStreamCreateWithPriority(&st, cudaStreamNonBlocking, least) != cudaSuccess) return nullptr;
+        streams[dev] = st;
+    }
+    return streams[dev];
+}
+
+// dA = dU^T X (computed as dA^T [K, R] = X^T dU) and dB = s dY^T U = dY^T (s U) from the hi/lo
+// operands dU2 and U2, on stream g; both use the split-partial region in turn.
+qlora_status lora_gradients_tc(const void* X, const void* dY, int64_t M, int64_t N, int64_t K, int32_t r,
+                               int32_t R, bool f16, float* dA, float* dB, const void* U2, const void* dU2,
+                               float* partial, cudaStream_t g) {
+    {
+        TimerScope t(QLORA_TIMER_LORA, g);
+        LoraGemmArgs a{};
+        a.mn_major = true; a.A = X; a.lda = K; a.B = dU2; a.ldb = 2 * R; a.rows = K; a.red = M; a.R = R;
+        a.partial = partial;
+        a.f16 = f16;
+        QLORA_TRY(launch_lora_gemm(a, g));
+        QLORA_TRY(launch_reduce_transposed(partial, lora_splits(K, (int)((M + 63) / 64), R, true), K, r, R, dA, g));
+    }
+    {
+        TimerScope t(QLORA_TIMER_LORA, g);
+        LoraGemmArgs a{};
+        a.mn_major = true; a.A = dY; a.lda = N; a.B = U2; a.ldb = 2 * R; a.rows = N; a.red = M; a.R = R;
+        a.partial = partial;
+        a.f16 = f16;
+        QLORA_TRY(launch_lora_gemm(a, g));
+        QLORA_TRY(launch_reduce_rows(partial, lora_splits(N, (int)((M + 63) / 64), R, true), N, r, R, 1.f, dB, 0.f,
+                                     nullptr, f16, g));
+    }
+    return QLORA_OK;
+}
+
 // Output dtypes a layer may write: fp32, or its 16-bit compute dtype.
 qlora_status check_out_dtype(int32_t dt, const qlora_nf4_weight* w) {
     return (dt == QLORA_DTYPE_F32 || dt == w->compute_dtype) ? QLORA_OK : QLORA_ERR_INVALID_ARG;
@@ -402,34 +451,39 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const void* X, const vo
             QLORA_TRY(launch_reduce_rows(partial, lora_splits(M, (int)((N + 63) / 64), R, false), M, r, R, scale, dUf, scale,
                                          dU2, f16, s));
         }
+        // fork: the adapter gradients go to the side stream once dU (and U2) are written
+        // (the caller's stream may be the null stream, so the fork is flagged, not inferred from g)
+        const bool forked = dX != nullptr;
+        cudaStream_t g = forked ? side_stream() : s;
+        cudaEvent_t fork = nullptr, join = nullptr;
+        if (forked && !g) return QLORA_ERR_CUDA;
+        if (forked) {
+            if (cudaEventCreateWithFlags(&fork, cudaEventDisableTiming) != cudaSuccess) return QLORA_ERR_CUDA;
+            if (cudaEventCreateWithFlags(&join, cudaEventDisableTiming) != cudaSuccess) {
+                cudaEventDestroy(fork);
+                return QLORA_ERR_CUDA;
+            }
+            const bool ok = cudaEventRecord(fork, s) == cudaSuccess && cudaStreamWaitEvent(g, fork, 0) == cudaSuccess;
+            cudaEventDestroy(fork);
+            if (!ok) { cudaEventDestroy(join); return QLORA_ERR_CUDA; }
+        }
+        qlora_status st = QLORA_OK;
         if (dX) {   // dX = dY W_hat + dU A
             TcGemmArgs a{};
             a.w = w; a.A0 = dY; a.A1 = dU2; a.B1 = A; a.b1_r = r; a.Rpad = R;   // A [r, K] read directly
             a.p.M = M; a.p.Nout = K; a.p.out = dX; a.p.ldo = K; a.p.out_f32 = (dx_dtype == QLORA_DTYPE_F32);
             TimerScope t(QLORA_TIMER_DX_MAIN, s);
-            QLORA_TRY(launch_tc_gemm_nf4(a, true, s));
+            st = launch_tc_gemm_nf4(a, true, s);
         }
-        {   // dA = dU^T X, computed as dA^T [K, R] = X^T dU
-            TimerScope t(QLORA_TIMER_LORA, s);
-            LoraGemmArgs g{};
-            g.mn_major = true; g.A = X; g.lda = K; g.B = dU2; g.ldb = 2 * R; g.rows = K; g.red = M; g.R = R;
-            g.partial = partial;
-            g.f16 = f16;
-            QLORA_TRY(launch_lora_gemm(g, s));
-            QLORA_TRY(launch_reduce_transposed(partial, lora_splits(K, (int)((M + 63) / 64), R, true), K, r, R, dA, s));
+        if (st == QLORA_OK) st = lora_gradients_tc(X, dY, M, N, K, r, R, f16, dA, dB, U2, dU2, partial, g);
+        if (forked) {   // join: the caller's stream resumes after the adapter gradients too
+            const bool ok = cudaEventRecord(join, g) == cudaSuccess && cudaStreamWaitEvent(s, join, 0) == cudaSuccess;
+            cudaEventDestroy(join);
+            if (!ok && st == QLORA_OK) st = QLORA_ERR_CUDA;
         }
-        {   // dB = s dY^T U = dY^T (s U)
-            TimerScope t(QLORA_TIMER_LORA, s);
-            LoraGemmArgs g{};
-            g.mn_major = true; g.A = dY; g.lda = N; g.B = U2; g.ldb = 2 * R; g.rows = N; g.red = M; g.R = R;
-            g.partial = partial;
-            g.f16 = f16;
-            QLORA_TRY(launch_lora_gemm(g, s));
-            QLORA_TRY(launch_reduce_rows(partial, lora_splits(N, (int)((M + 63) / 64), R, true), N, r, R, 1.f, dB, 0.f,
-                                         nullptr, f16, s));
-        }
-        return QLORA_OK;
+        return st;
     }
+
 
     // CUDA-core path for N % 8 != 0.
     const float* U = U_saved;
