@@ -35,6 +35,7 @@
 // order (row tiles fastest within groups of 16) so concurrent CTAs share W.
 // No TMA multicast is used anywhere.
 #include <algorithm>
+#include <cstdlib>
 
 #include <cuda.h>
 
@@ -175,6 +176,42 @@ __device__ __forceinline__ void raster_tile(int64_t t, int64_t mtiles, int64_t n
     const int64_t local = t % per_group;
     mt = first + local % gm;
     nt = local / gm;
+}
+
+// Store 32 consecutive output columns nb .. nb+31 of row m (fp32, or rounded to the 16-bit
+// compute dtype); columns at or past Nout are skipped.
+__device__ __forceinline__ void store_row32(const TcGemmParams& p, int64_t m, int64_t nb, const uint32_t (&v)[32]) {
+    const bool full = (nb + 32 <= p.Nout);
+    if (p.out_f32) {
+        float* dst = static_cast<float*>(p.out) + m * p.ldo + nb;
+        if (full && (p.ldo & 3) == 0) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                reinterpret_cast<uint4*>(dst)[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                if (nb + i < p.Nout) dst[i] = __uint_as_float(v[i]);
+        }
+    } else {
+        uint16_t* dst = static_cast<uint16_t*>(p.out) + m * p.ldo + nb;
+        const bool h = p.f16 != 0;
+        if (full && (p.ldo & 7) == 0) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                uint4 o;
+                o.x = pack16x2_rn(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]), h);
+                o.y = pack16x2_rn(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]), h);
+                o.z = pack16x2_rn(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]), h);
+                o.w = pack16x2_rn(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]), h);
+                reinterpret_cast<uint4*>(dst)[i] = o;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                if (nb + i < p.Nout) dst[i] = (uint16_t)to16_rn(__uint_as_float(v[i]), h);
+        }
+    }
 }
 
 template <int NUM_ACC, bool DX>
@@ -413,35 +450,7 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
                     ptx::tmem_ld_32x32b_x32(tmem + ((quad * 32u) << 16) + h * 256 + c * 32, v);
                     ptx::tmem_ld_wait();
                     if (m >= p.M) continue;
-                    const bool full = (nb + 32 <= p.Nout);
-                    if (p.out_f32) {
-                        float* dst = static_cast<float*>(p.out) + m * p.ldo + nb;
-                        if (full && (p.ldo & 3) == 0) {
-#pragma unroll
-                            for (int i = 0; i < 8; ++i)
-                                reinterpret_cast<uint4*>(dst)[i] =
-                                    make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-                        } else {
-                            for (int i = 0; i < 32 && nb + i < p.Nout; ++i) dst[i] = __uint_as_float(v[i]);
-                        }
-                    } else {
-                        uint16_t* dst = static_cast<uint16_t*>(p.out) + m * p.ldo + nb;
-                        if (full && (p.ldo & 7) == 0) {
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                uint4 o;
-                                const bool h = p.f16 != 0;
-                                o.x = pack16x2_rn(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]), h);
-                                o.y = pack16x2_rn(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]), h);
-                                o.z = pack16x2_rn(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]), h);
-                                o.w = pack16x2_rn(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]), h);
-                                reinterpret_cast<uint4*>(dst)[i] = o;
-                            }
-                        } else {
-                            for (int i = 0; i < 32 && nb + i < p.Nout; ++i)
-                                dst[i] = (uint16_t)to16_rn(__uint_as_float(v[i]), p.f16 != 0);
-                        }
-                    }
+                    store_row32(p, m, nb, v);
                 }
             }
         }
@@ -452,6 +461,295 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
     if (warp == 1) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, 256 * NUM_ACC);
+    }
+}
+
+// ---------------------------------------------------------------------------- fwd / dX on CTA pairs
+//
+// The same forward (Y = X W_hat^T + U2 B2^T) and dX (dX = dY W_hat + dU2 A2), computed by clusters
+// of two CTAs that share each MMA (tcgen05 cta_group::2, M = 256 tokens x N = 256 output columns
+// per instruction).  A pair's tile is 512 tokens x 256 output columns: CTA rank r holds tokens
+// m0 + 256 r + [0, 256) (two 128-row halves, one per accumulator) and supplies output columns
+// nr0 = n0 + 128 r + [0, 128) of operand B, so it expands only its half of the W tile (forward:
+// W rows nr0 + [0, 128) of each K-step; dX: the two 64-weight blocks of columns nr0 + [0, 128) of
+// each of the step's 64 W rows).  Each W tile is dequantized once per 512 tokens instead of once
+// per 256, which halves the producers' work per MMA flop.
+// Every CTA loads its own tiles (no load is shared between the two); the loads of the token
+// tiles (and of the LoRA operands) count their bytes on the leader's (rank 0) barrier, because
+// the leader issues the MMAs, which read both CTAs' shared memory.
+// Warp roles as in the single-CTA kernel; the two producer groups of 4 warps take alternate
+// K-steps (stage parity = group, 4 stages).
+// Barriers, per CTA unless marked "leader":
+//   full_a[s]  (leader) 1 arrival (the leader's expect-tx) + the token-tile bytes of both CTAs
+//              (and, on LoRA steps, the B-operand bytes of both);
+//   full_b[s]  (leader) 8 arrivals: the 4 producer warps of the stage's group in both CTAs;
+//   codes[s]   1 arrival (this CTA's expect-tx) + this CTA's code-tile bytes;
+//   empty[s]   1 arrival: the leader's commit after the MMAs that read stage s (it commits once
+//              to its own barrier and once to the peer's, by cluster address);
+//   acc        1 arrival: the leader's commit after the last MMA.
+constexpr int kPairStages = 4;
+constexpr uint32_t kPairAStage = 256 * 128;                  // 256 tokens x 64, 128-byte swizzled rows
+constexpr uint32_t kPairBStage = 128 * 128;                  // 128 W rows x 64
+constexpr uint32_t kPairCodesStage = 128 * 32;               // fwd: 128 W rows x 32 bytes; dX: 64 rows x 64 bytes
+constexpr uint32_t kPairOffB = kPairStages * kPairAStage;
+constexpr uint32_t kPairOffCodes = kPairOffB + kPairStages * kPairBStage;
+constexpr uint32_t kPairOffE4 = kPairOffCodes + kPairStages * kPairCodesStage;
+constexpr uint32_t kPairOffBars = kPairOffE4 + 256 * 4;
+constexpr uint32_t kPairNumBars = 4 * kPairStages + 1;
+constexpr uint32_t kPairOffSlot = kPairOffBars + kPairNumBars * 8;
+constexpr uint32_t kPairOffAbort = kPairOffSlot + 4;
+constexpr uint32_t kPairAlloc = kPairOffAbort + 4 + 1024;
+static_assert(kPairAlloc <= 232448, "shared memory of one CTA");
+
+template <bool DX>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+tc_gemm_nf4_pair(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmCodes,
+                 const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1, TcGemmParams p) {
+    grid_dependency_wait();                                   // operands written by the previous kernel
+    allow_dependents();
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t base = (ptx::smem_addr(smem_raw) + 1023u) & ~1023u;
+    uint8_t* gbase = smem_raw + (base - ptx::smem_addr(smem_raw));
+    const uint32_t sA = base, sB = base + kPairOffB, sCodes = base + kPairOffCodes;
+    const uint32_t bar_full_a = base + kPairOffBars;
+    const uint32_t bar_full_b = bar_full_a + 8 * kPairStages;
+    const uint32_t bar_codes = bar_full_b + 8 * kPairStages;
+    const uint32_t bar_empty = bar_codes + 8 * kPairStages;
+    const uint32_t bar_acc = bar_empty + 8 * kPairStages;
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gbase + kPairOffSlot);
+    volatile int* abort = reinterpret_cast<volatile int*>(gbase + kPairOffAbort);
+
+    const uint32_t rank = ptx::cluster_ctarank();
+    const bool leader = rank == 0;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int64_t mt, nt;
+    raster_tile(blockIdx.x >> 1, (p.M + 511) / 512, (p.Nout + kBN - 1) / kBN, mt, nt);
+    const int64_t m0 = mt * 512 + 256 * (int64_t)rank;       // this CTA's first token
+    const int64_t n0 = nt * kBN;                              // the pair's output column tile
+    const int64_t nr0 = n0 + 128 * (int64_t)rank;             // this CTA's output columns (forward: W rows)
+    const int ks0 = p.ksteps0, ktotal = p.ksteps0 + p.ksteps1;
+    float* e4tab = reinterpret_cast<float*>(gbase + kPairOffE4);
+    if (threadIdx.x < 256) e4tab[threadIdx.x] = e4m3_to_f32(threadIdx.x);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kPairStages; ++s) {
+            ptx::mbar_init(bar_full_a + 8 * s, 1);
+            ptx::mbar_init(bar_full_b + 8 * s, 8);
+            ptx::mbar_init(bar_codes + 8 * s, 1);
+            ptx::mbar_init(bar_empty + 8 * s, 1);
+        }
+        ptx::mbar_init(bar_acc, 1);
+        *abort = 0;
+        ptx::fence_barrier_init();
+        ptx::fence_proxy_async_smem();
+        ptx::tma_prefetch_map(&tmA0);
+        ptx::tma_prefetch_map(&tmCodes);
+        ptx::tma_prefetch_map(&tmA1);
+        ptx::tma_prefetch_map(&tmB1);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc_pair(base + kPairOffSlot, 512);
+        ptx::tmem_relinquish_pair();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::cluster_sync();                                      // both CTAs' barriers exist before any remote signal
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lead_full_a = ptx::mapa_shared(bar_full_a, 0);
+    const uint32_t lead_full_b = ptx::mapa_shared(bar_full_b, 0);
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA (both CTAs)
+        int issued = 0;
+        int s = 0;
+        uint32_t ph = 0;
+        for (int it = 0; it < ktotal; ++it) {
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_empty + 8 * s, ph ^ 1u, abort, p.err))) break;
+            issued = it + 1;
+            if (ptx::elect_one_sync()) {
+                const uint32_t a_dst = sA + s * kPairAStage;
+                if (it < ks0) {
+                    if (leader) ptx::mbar_arrive_expect_tx(bar_full_a + 8 * s, 2 * kPairAStage);
+                    ptx::tma_load_2d_pair(a_dst, &tmA0, it * 64, (int32_t)m0, lead_full_a + 8 * s);
+                    ptx::mbar_arrive_expect_tx(bar_codes + 8 * s, kPairCodesStage);
+                    if (!DX)
+                        ptx::tma_load_2d(sCodes + s * kPairCodesStage, &tmCodes, it * 32, (int32_t)nr0, bar_codes + 8 * s);
+                    else
+                        ptx::tma_load_2d(sCodes + s * kPairCodesStage, &tmCodes, (int32_t)(nr0 / 2), it * 64,
+                                         bar_codes + 8 * s);
+                } else {
+                    const int j = it - ks0;
+                    const int jb = p.b1_wrap ? j % p.b1_wrap : j;   // hi and lo steps share the B1 tile
+                    if (leader) ptx::mbar_arrive_expect_tx(bar_full_a + 8 * s, 2 * (kPairAStage + kPairBStage));
+                    ptx::tma_load_2d_pair(a_dst, &tmA1, j * 64, (int32_t)m0, lead_full_a + 8 * s);
+                    if (!DX) {
+                        ptx::tma_load_2d_pair(sB + s * kPairBStage, &tmB1, jb * 64, (int32_t)nr0, lead_full_a + 8 * s);
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 2; ++c)
+                            ptx::tma_load_2d_pair(sB + s * kPairBStage + c * 8192, &tmB1, (int32_t)(nr0 + c * 64), jb * 64,
+                                                  lead_full_a + 8 * s);
+                    }
+                }
+            }
+            __syncwarp();
+            if (++s == kPairStages) { s = 0; ph ^= 1u; }
+        }
+        if (*abort) {   // drain what this CTA can observe: its code tiles, and (leader) the token tiles
+            for (int it = max(0, issued - kPairStages); it < issued; ++it) {
+                const uint32_t ph_i = (uint32_t)(it / kPairStages) & 1u;
+                if (it < ks0) ptx::mbar_wait_drain(bar_codes + 8 * (it % kPairStages), ph_i);
+                if (leader) ptx::mbar_wait_drain(bar_full_a + 8 * (it % kPairStages), ph_i);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (leader only)
+        if (leader) {
+            const uint32_t idesc = ptx::idesc_set_f16(ptx::idesc_bf16_f32(256, kBN, DX ? 1 : 0), p.f16 != 0);
+            const uint64_t adesc0 = ptx::smem_desc_sw128(sA, 16, 1024);
+            // forward: LoRA steps read 128B-swizzled TMA tiles, W_hat steps the non-swizzled K-major image;
+            // dX: both are two MN-major 64-column images 8 KiB apart
+            const uint64_t bdesc0 = DX ? ptx::smem_desc_sw128(sB, 8192, 1024) : ptx::smem_desc_sw128(sB, 16, 1024);
+            const uint64_t bdesc0_kn = ptx::smem_desc_kmajor_none(sB, 128 * 16, 128);
+            const uint32_t peer_empty = ptx::mapa_shared(bar_empty, 1);
+            const uint32_t peer_acc = ptx::mapa_shared(bar_acc, 1);
+            bool ok = true;
+            int s = 0;
+            uint32_t ph = 0;
+            for (int it = 0; it < ktotal && ok; ++it) {
+                bool w = ptx::mbar_wait(bar_full_a + 8 * s, ph, abort, p.err);
+                if (w && it < ks0) w = ptx::mbar_wait(bar_full_b + 8 * s, ph, abort, p.err);
+                ok = __all_sync(0xffffffffu, w);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                if (ptx::elect_one_sync()) {
+                    const uint64_t ad = adesc0 + ((uint32_t)s * (kPairAStage >> 4));
+                    const bool kn = !DX && it < ks0;
+                    const uint64_t bd = (kn ? bdesc0_kn : bdesc0) + ((uint32_t)s * (kPairBStage >> 4));
+                    const uint32_t kstep = DX ? (2048 >> 4) : kn ? ((2 * 128 * 16) >> 4) : (32 >> 4);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)
+                            ptx::mma_bf16_ss_pair(tmem + h * 256, ad + h * (16384 >> 4) + kk * (32 >> 4),
+                                                  bd + kk * kstep, idesc, (it | kk) != 0 ? 1u : 0u);
+                    }
+                    ptx::mma_commit_pair(bar_empty + 8 * s);          // this CTA's stage
+                    ptx::mma_commit_pair(peer_empty + 8 * s);         // the peer's stage
+                }
+                __syncwarp();
+                if (++s == kPairStages) { s = 0; ph ^= 1u; }
+            }
+            if (ptx::elect_one_sync()) {
+                ptx::mma_commit_pair(bar_acc);
+                ptx::mma_commit_pair(peer_acc);
+                if (*abort) ptx::mbar_wait_drain(bar_acc, 0);   // issued MMAs finish before TMEM is freed
+            }
+            __syncwarp();
+        }
+    } else {
+        // ------------------------------------------------------------ dequant producers (both CTAs)
+        // group g expands the K-steps it = g, g + 2, ...; thread t of the group: forward: W row nr0 + t,
+        // K-block it; dX: W row 64 it + (t & 63), K-block (nr0 >> 6) + kc with kc = t >> 6
+        const int g = (warp - 2) >> 2;
+        const int t = threadIdx.x - 64 - 128 * g;
+        const float mu = p.c1f ? 0.f : *p.mu;
+        const int64_t blocks_per_row = p.WK / 64;
+        const uint32_t row = DX ? (uint32_t)(t & 63) : (uint32_t)t;
+        const uint32_t kc = DX ? (uint32_t)(t >> 6) : 0u;
+        const bool lane_ok = DX ? (nr0 + (int64_t)kc * 64 < p.WK) : (nr0 + t < p.WN);
+        // block of the step whose constants load next, moving by a fixed stride per group step
+        // (forward: 2 blocks along the row; dX: 128 W rows down)
+        int64_t a_blk = DX ? ((int64_t)g * 64 + row) * blocks_per_row + (nr0 >> 6) + kc : (nr0 + t) * blocks_per_row + g;
+        const int64_t blk_step = DX ? 128 * blocks_per_row : 2;
+        int64_t a_n = (int64_t)g * 64 + row;                  // dX: the W row of that step
+        auto const_load = [&](int step, bool& v, uint32_t& code, float& c2) {
+            v = lane_ok && step < ks0 && (!DX || a_n < p.WN);
+            code = 0;
+            c2 = 0.f;
+            if (v) {
+                if (p.c1f) {
+                    c2 = __ldg(p.c1f + a_blk);
+                } else {
+                    code = __ldg(p.c1_codes + a_blk);
+                    c2 = __ldg(p.c2 + (a_blk >> 8));
+                }
+            }
+            a_blk += blk_step;
+            a_n += 128;
+        };
+        bool qv[kGemmPrefetch];
+        uint32_t qcode[kGemmPrefetch];
+        float qc2[kGemmPrefetch];
+#pragma unroll
+        for (int d = 0; d < kGemmPrefetch; ++d) const_load(g + 2 * d, qv[d], qcode[d], qc2[d]);
+        bool ok = true;
+        for (int it = g; it < ks0 && ok; it += 2) {
+            const int s = it & (kPairStages - 1);
+            const uint32_t ph = (uint32_t)(it / kPairStages) & 1u;
+            const bool valid = qv[0];
+            const float c1p = !valid ? 0.f : (p.c1f ? qc2[0] : __fadd_rn(__fmul_rn(e4tab[qcode[0]], qc2[0]), mu));
+#pragma unroll
+            for (int d = 0; d + 1 < kGemmPrefetch; ++d) {
+                qv[d] = qv[d + 1];
+                qcode[d] = qcode[d + 1];
+                qc2[d] = qc2[d + 1];
+            }
+            const_load(it + 2 * kGemmPrefetch, qv[kGemmPrefetch - 1], qcode[kGemmPrefetch - 1], qc2[kGemmPrefetch - 1]);
+            ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_codes + 8 * s, ph, abort, p.err));
+            if (!ok) break;
+            // forward: non-swizzled K-major image of 128 rows (row t at 16 t, chunk c at 2048 c);
+            // dX: 128-byte-swizzled 64-row images, one per K-block, read as an MN-major operand
+            const uint32_t row_addr = sB + s * kPairBStage + (DX ? kc * 8192u + row * 128u : row * 16u);
+            if (!valid) {
+                if (DX) zero_row(row_addr);
+                else zero_row_kn<128 * 16>(row_addr);
+            } else {
+                // codes: forward 128 rows x 32 bytes; dX 64 rows x 64 bytes (this CTA's two blocks)
+                const uint32_t src = sCodes + s * kPairCodesStage + (DX ? row * 64u + kc * 32u : row * 32u);
+                const uint4 c0 = ld_shared_v4(src);
+                const uint4 c1 = ld_shared_v4(src + 16u);
+                Lut lut;
+                build_lut(lut, c1p, p.tb, p.f16 != 0);
+                if (DX) expand_block_row(row_addr, row & 7u, c0, c1, lut);
+                else expand_block_row_kn<128 * 16>(row_addr, c0, c1, lut);
+            }
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive_cluster(lead_full_b + 8 * s);
+        }
+
+        // ------------------------------------------------------------ epilogue
+        const bool acc_ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_acc, 0, abort, p.err));
+        ptx::tc_fence_after();
+        if (acc_ok) {
+            const uint32_t quad = (uint32_t)(warp & 3);
+            const int half = (warp - 2) >> 2;
+#pragma unroll 1
+            for (int h = 0; h < 2; ++h) {
+                const int64_t m = m0 + h * 128 + quad * 32 + lane;
+#pragma unroll 1
+                for (int cc = 0; cc < kBN / 64; ++cc) {
+                    const int c = half * (kBN / 64) + cc;
+                    const int64_t nb = n0 + c * 32;
+                    if (nb >= p.Nout) break;
+                    uint32_t v[32];
+                    ptx::tmem_ld_32x32b_x32(tmem + ((quad * 32u) << 16) + h * 256 + c * 32, v);
+                    ptx::tmem_ld_wait();
+                    if (m >= p.M) continue;
+                    store_row32(p, m, nb, v);
+                }
+            }
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::cluster_sync();                                      // no CTA leaves while its peer may still signal it
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc_pair(tmem, 512);
     }
 }
 
@@ -963,6 +1261,47 @@ static qlora_status launch_one(const TcGemmArgs& a, cudaStream_t stream) {
     return QLORA_OK;
 }
 
+// The forward on CTA pairs: clusters of 2, one pair per 512 x 256 output tile.
+template <bool DX>
+static qlora_status launch_pair(const TcGemmArgs& a, cudaStream_t stream) {
+    static bool configured = false;   // attribute set once per instantiation (idempotent, so races are benign)
+    auto kern = tc_gemm_nf4_pair<DX>;
+    if (!configured) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPairAlloc) != cudaSuccess)
+            return QLORA_ERR_CUDA;
+        configured = true;
+    }
+    const int64_t pairs = ((a.p.Nout + kBN - 1) / kBN) * ((a.p.M + 511) / 512);
+    if (2 * pairs > INT32_MAX) return QLORA_ERR_SHAPE;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * pairs));
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = kPairAlloc;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    (void)cudaLaunchKernelEx(&cfg, kern, a.tmA0, a.tmCodes, a.tmA1, a.tmB1, a.p);
+    QLORA_CHECK_LAUNCH();
+    return QLORA_OK;
+}
+
+// Whether the forward and dX run on CTA pairs: more than 256 tokens (a pair's tile covers 512),
+// unless the environment variable QLORA_PAIR_GEMM is set to 0 (the single-CTA kernels then run).
+static bool use_pairs(int64_t M) {
+    static const bool enabled = [] {
+        const char* e = std::getenv("QLORA_PAIR_GEMM");
+        return !(e && e[0] == '0');
+    }();
+    return enabled && M > 256;
+}
+
 // Splits of the reduction so that tiles x splits fills one wave of CTAs.
 static int64_t decode_grid(int64_t units, int sms) {
     return std::max<int64_t>(1, std::min<int64_t>({units, (int64_t)kDecCtasPerSm * sms, (int64_t)kDecMaxCtas}));
@@ -1034,13 +1373,19 @@ qlora_status launch_tc_gemm_nf4(TcGemmArgs& a, bool dx, cudaStream_t stream) {
     const uint32_t bm = a.p.M > 128 ? 256 : 128;
     const qlora_nf4_weight* w = a.w;
     const int64_t N = w->N, K = w->K;
+    const bool pair = use_pairs(a.p.M);
+    const uint32_t wrows = pair ? 128 : 256;          // forward: W rows one CTA loads codes (and LoRA B rows) for
     // segment 0: A (X or dY) and the packed codes
     if (!dx) {
         if (!make_tmap_2d(&a.tmA0, true, a.A0, K, a.p.M, K * 2, 64, bm, true)) return QLORA_ERR_CUDA;
-        if (!make_tmap_2d(&a.tmCodes, false, w->codes, K / 2, N, K / 2, 32, 256, false)) return QLORA_ERR_CUDA;
+        if (!make_tmap_2d(&a.tmCodes, false, w->codes, K / 2, N, K / 2, 32, wrows, false)) return QLORA_ERR_CUDA;
     } else {
         if (!make_tmap_2d(&a.tmA0, true, a.A0, N, a.p.M, N * 2, 64, bm, true)) return QLORA_ERR_CUDA;
-        if (!make_tmap_2d(&a.tmCodes, false, w->codes, K / 2, N, K / 2, 128, 64, true)) return QLORA_ERR_CUDA;
+        if (pair) {   // this CTA's 64 bytes (two blocks) of each of the step's 64 W rows, unswizzled
+            if (!make_tmap_2d(&a.tmCodes, false, w->codes, K / 2, N, K / 2, 64, 64, false)) return QLORA_ERR_CUDA;
+        } else {
+            if (!make_tmap_2d(&a.tmCodes, false, w->codes, K / 2, N, K / 2, 128, 64, true)) return QLORA_ERR_CUDA;
+        }
     }
     // segment 1: LoRA operands, [M, 2R] and [N, 2R] (forward) or [2R, K] (dX)
     const int64_t R2 = 2 * (int64_t)a.Rpad;
@@ -1048,13 +1393,13 @@ qlora_status launch_tc_gemm_nf4(TcGemmArgs& a, bool dx, cudaStream_t stream) {
     if (a.b1_r > 0) {   // B [N, r] or A [r, K] directly
         const uint64_t r = (uint64_t)a.b1_r;
         if (!dx) {
-            if (!make_tmap_2d(&a.tmB1, true, a.B1, r, N, r * 2, 64, 256, true)) return QLORA_ERR_CUDA;
+            if (!make_tmap_2d(&a.tmB1, true, a.B1, r, N, r * 2, 64, wrows, true)) return QLORA_ERR_CUDA;
         } else {
             if (!make_tmap_2d(&a.tmB1, true, a.B1, K, r, K * 2, 64, 64, true)) return QLORA_ERR_CUDA;
         }
         a.p.b1_wrap = (int32_t)(R2 / 128);
     } else if (!dx) {
-        if (!make_tmap_2d(&a.tmB1, true, a.B1, R2, N, R2 * 2, 64, 256, true)) return QLORA_ERR_CUDA;
+        if (!make_tmap_2d(&a.tmB1, true, a.B1, R2, N, R2 * 2, 64, wrows, true)) return QLORA_ERR_CUDA;
     } else {
         if (!make_tmap_2d(&a.tmB1, true, a.B1, K, R2, K * 2, 64, 64, true)) return QLORA_ERR_CUDA;
     }
@@ -1070,6 +1415,7 @@ qlora_status launch_tc_gemm_nf4(TcGemmArgs& a, bool dx, cudaStream_t stream) {
     a.p.tb = host_tables(w->codebook);
     a.p.err = device_error_word();
     if (!a.p.err) return QLORA_ERR_CUDA;
+    if (pair) return dx ? launch_pair<true>(a, stream) : launch_pair<false>(a, stream);
     if (bm == 256) return dx ? launch_one<2, true>(a, stream) : launch_one<2, false>(a, stream);
     return dx ? launch_one<1, true>(a, stream) : launch_one<1, false>(a, stream);
 }
