@@ -269,9 +269,13 @@ __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// Arrive on an mbarrier of any CTA of the cluster (release at cluster scope).
+// Arrive on an mbarrier of any CTA of the cluster by its cluster address (default semantics).  The
+// producers that signal the pair leader this way have made their shared-memory writes visible to
+// the async proxy first (fence.proxy.async), and the reader is the leader's MMA, which reads this
+// CTA's shared memory through that proxy; a cluster-scope release here cost a full memory barrier
+// per arrival.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
 }
 
 // TMA tile load into this CTA's shared memory whose completion bytes count on the mbarrier at
