@@ -35,6 +35,7 @@
 // order (row tiles fastest within groups of 16) so concurrent CTAs share W.
 // No TMA multicast is used anywhere.
 #include <algorithm>
+#include <climits>
 #include <cstdlib>
 
 #include <cuda.h>
@@ -179,9 +180,10 @@ __device__ __forceinline__ void raster_tile(int64_t t, int64_t mtiles, int64_t n
 }
 
 // Store 32 consecutive output columns nb .. nb+31 of row m (fp32, or rounded to the 16-bit
-// compute dtype); columns at or past Nout are skipped.
-__device__ __forceinline__ void store_row32(const TcGemmParams& p, int64_t m, int64_t nb, const uint32_t (&v)[32]) {
-    const bool full = (nb + 32 <= p.Nout);
+// compute dtype); columns at or past nlim (the end of the tile or of the row) are skipped.
+__device__ __forceinline__ void store_row32(const TcGemmParams& p, int64_t m, int64_t nb, int64_t nlim,
+                                            const uint32_t (&v)[32]) {
+    const bool full = (nb + 32 <= nlim);
     if (p.out_f32) {
         float* dst = static_cast<float*>(p.out) + m * p.ldo + nb;
         if (full && (p.ldo & 3) == 0) {
@@ -191,7 +193,7 @@ __device__ __forceinline__ void store_row32(const TcGemmParams& p, int64_t m, in
         } else {
 #pragma unroll
             for (int i = 0; i < 32; ++i)
-                if (nb + i < p.Nout) dst[i] = __uint_as_float(v[i]);
+                if (nb + i < nlim) dst[i] = __uint_as_float(v[i]);
         }
     } else {
         uint16_t* dst = static_cast<uint16_t*>(p.out) + m * p.ldo + nb;
@@ -209,7 +211,7 @@ __device__ __forceinline__ void store_row32(const TcGemmParams& p, int64_t m, in
         } else {
 #pragma unroll
             for (int i = 0; i < 32; ++i)
-                if (nb + i < p.Nout) dst[i] = (uint16_t)to16_rn(__uint_as_float(v[i]), h);
+                if (nb + i < nlim) dst[i] = (uint16_t)to16_rn(__uint_as_float(v[i]), h);
         }
     }
 }
@@ -450,7 +452,7 @@ tc_gemm_nf4(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CU
                     ptx::tmem_ld_32x32b_x32(tmem + ((quad * 32u) << 16) + h * 256 + c * 32, v);
                     ptx::tmem_ld_wait();
                     if (m >= p.M) continue;
-                    store_row32(p, m, nb, v);
+                    store_row32(p, m, nb, p.Nout, v);
                 }
             }
         }
@@ -523,10 +525,12 @@ tc_gemm_nf4_pair(const __grid_constant__ CUtensorMap tmA0, const __grid_constant
     const bool leader = rank == 0;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int64_t mt, nt;
-    raster_tile(blockIdx.x >> 1, (p.M + 511) / 512, (p.Nout + kBN - 1) / kBN, mt, nt);
+    const int bn = DX ? kBN : p.bn;                           // output columns of the pair tile
+    const int hb = bn / 2;                                    // of which this CTA supplies
+    raster_tile(blockIdx.x >> 1, (p.M + 511) / 512, (p.Nout + bn - 1) / bn, mt, nt);
     const int64_t m0 = mt * 512 + 256 * (int64_t)rank;       // this CTA's first token
-    const int64_t n0 = nt * kBN;                              // the pair's output column tile
-    const int64_t nr0 = n0 + 128 * (int64_t)rank;             // this CTA's output columns (forward: W rows)
+    const int64_t n0 = nt * bn;                               // the pair's output column tile
+    const int64_t nr0 = n0 + hb * (int64_t)rank;              // this CTA's output columns (forward: W rows)
     const int ks0 = p.ksteps0, ktotal = p.ksteps0 + p.ksteps1;
     float* e4tab = reinterpret_cast<float*>(gbase + kPairOffE4);
     if (threadIdx.x < 256) e4tab[threadIdx.x] = e4m3_to_f32(threadIdx.x);
@@ -572,7 +576,7 @@ tc_gemm_nf4_pair(const __grid_constant__ CUtensorMap tmA0, const __grid_constant
                 if (it < ks0) {
                     if (leader) ptx::mbar_arrive_expect_tx(bar_full_a + 8 * s, 2 * kPairAStage);
                     ptx::tma_load_2d_pair(a_dst, &tmA0, it * 64, (int32_t)m0, lead_full_a + 8 * s);
-                    ptx::mbar_arrive_expect_tx(bar_codes + 8 * s, kPairCodesStage);
+                    ptx::mbar_arrive_expect_tx(bar_codes + 8 * s, DX ? kPairCodesStage : 32u * (uint32_t)hb);
                     if (!DX)
                         ptx::tma_load_2d(sCodes + s * kPairCodesStage, &tmCodes, it * 32, (int32_t)nr0, bar_codes + 8 * s);
                     else
@@ -581,7 +585,9 @@ tc_gemm_nf4_pair(const __grid_constant__ CUtensorMap tmA0, const __grid_constant
                 } else {
                     const int j = it - ks0;
                     const int jb = p.b1_wrap ? j % p.b1_wrap : j;   // hi and lo steps share the B1 tile
-                    if (leader) ptx::mbar_arrive_expect_tx(bar_full_a + 8 * s, 2 * (kPairAStage + kPairBStage));
+                    if (leader)
+                        ptx::mbar_arrive_expect_tx(bar_full_a + 8 * s,
+                                                   2 * (kPairAStage + (DX ? kPairBStage : 128u * (uint32_t)hb)));
                     ptx::tma_load_2d_pair(a_dst, &tmA1, j * 64, (int32_t)m0, lead_full_a + 8 * s);
                     if (!DX) {
                         ptx::tma_load_2d_pair(sB + s * kPairBStage, &tmB1, jb * 64, (int32_t)nr0, lead_full_a + 8 * s);
@@ -606,7 +612,7 @@ tc_gemm_nf4_pair(const __grid_constant__ CUtensorMap tmA0, const __grid_constant
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer (leader only)
         if (leader) {
-            const uint32_t idesc = ptx::idesc_set_f16(ptx::idesc_bf16_f32(256, kBN, DX ? 1 : 0), p.f16 != 0);
+            const uint32_t idesc = ptx::idesc_set_f16(ptx::idesc_bf16_f32(256, bn, DX ? 1 : 0), p.f16 != 0);
             const uint64_t adesc0 = ptx::smem_desc_sw128(sA, 16, 1024);
             // forward: LoRA steps read 128B-swizzled TMA tiles, W_hat steps the non-swizzled K-major image;
             // dX: both are two MN-major 64-column images 8 KiB apart
@@ -658,7 +664,8 @@ tc_gemm_nf4_pair(const __grid_constant__ CUtensorMap tmA0, const __grid_constant
         const int64_t blocks_per_row = p.WK / 64;
         const uint32_t row = DX ? (uint32_t)(t & 63) : (uint32_t)t;
         const uint32_t kc = DX ? (uint32_t)(t >> 6) : 0u;
-        const bool lane_ok = DX ? (nr0 + (int64_t)kc * 64 < p.WK) : (nr0 + t < p.WN);
+        const bool lane_ok = DX ? (nr0 + (int64_t)kc * 64 < p.WK) : (t < hb && nr0 + t < p.WN);
+        const bool in_tile = DX || t < hb;                    // forward rows past a narrow tile are never read
         // block of the step whose constants load next, moving by a fixed stride per group step
         // (forward: 2 blocks along the row; dX: 128 W rows down)
         int64_t a_blk = DX ? ((int64_t)g * 64 + row) * blocks_per_row + (nr0 >> 6) + kc : (nr0 + t) * blocks_per_row + g;
@@ -702,7 +709,9 @@ tc_gemm_nf4_pair(const __grid_constant__ CUtensorMap tmA0, const __grid_constant
             // forward: non-swizzled K-major image of 128 rows (row t at 16 t, chunk c at 2048 c);
             // dX: 128-byte-swizzled 64-row images, one per K-block, read as an MN-major operand
             const uint32_t row_addr = sB + s * kPairBStage + (DX ? kc * 8192u + row * 128u : row * 16u);
-            if (!valid) {
+            if (!in_tile) {
+                // nothing to write
+            } else if (!valid) {
                 if (DX) zero_row(row_addr);
                 else zero_row_kn<128 * 16>(row_addr);
             } else {
@@ -733,12 +742,13 @@ tc_gemm_nf4_pair(const __grid_constant__ CUtensorMap tmA0, const __grid_constant
                 for (int cc = 0; cc < kBN / 64; ++cc) {
                     const int c = half * (kBN / 64) + cc;
                     const int64_t nb = n0 + c * 32;
-                    if (nb >= p.Nout) break;
+                    const int64_t nlim = min(p.Nout, n0 + bn);
+                    if (nb >= nlim) break;
                     uint32_t v[32];
                     ptx::tmem_ld_32x32b_x32(tmem + ((quad * 32u) << 16) + h * 256 + c * 32, v);
                     ptx::tmem_ld_wait();
                     if (m >= p.M) continue;
-                    store_row32(p, m, nb, v);
+                    store_row32(p, m, nb, nlim, v);
                 }
             }
         }
@@ -1271,7 +1281,8 @@ static qlora_status launch_pair(const TcGemmArgs& a, cudaStream_t stream) {
             return QLORA_ERR_CUDA;
         configured = true;
     }
-    const int64_t pairs = ((a.p.Nout + kBN - 1) / kBN) * ((a.p.M + 511) / 512);
+    const int bn = DX ? kBN : a.p.bn;
+    const int64_t pairs = ((a.p.Nout + bn - 1) / bn) * ((a.p.M + 511) / 512);
     if (2 * pairs > INT32_MAX) return QLORA_ERR_SHAPE;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(2 * pairs));
@@ -1300,6 +1311,54 @@ static bool use_pairs(int64_t M) {
         return !(e && e[0] == '0');
     }();
     return enabled && M > 256;
+}
+
+// Forward pair-tile width: the multiple of 16 in {256, 240, 224} that minimises waves x width,
+// the time of the launch when every pair runs one tile at a time (ties to the wider tile), with
+// as many pairs in a wave as clusters of 2 fit on the GPU at once.  For example W[8192, *] at
+// M = 2048: 256 gives 128 pair tiles (1.73 waves of 74 pairs, the second 73% full), 224 gives
+// 148 (two full waves) of 7/8 the work each.  Now that the producers expand half a W tile per
+// CTA the MMAs bound a tile, so its time follows its width.
+static int pair_tile_width(int64_t M, int64_t N) {
+    static int slots = 0;
+    if (slots == 0) {
+        int dev = 0, sms = 148;
+        if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * (unsigned)sms);
+        cfg.blockDim = dim3(kGemmThreads);
+        cfg.dynamicSmemBytes = kPairAlloc;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaFuncSetAttribute(tc_gemm_nf4_pair<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kPairAlloc) != cudaSuccess ||
+            cudaOccupancyMaxActiveClusters(&n, tc_gemm_nf4_pair<false>, &cfg) != cudaSuccess || n < 1) {
+            (void)cudaGetLastError();
+            n = sms / 2;
+        }
+        slots = n;
+    }
+    static const int forced = [] {   // QLORA_PAIR_BN=256|240|224 forces the width (tuning override)
+        const char* e = std::getenv("QLORA_PAIR_BN");
+        const int v = e ? std::atoi(e) : 0;
+        return (v == 256 || v == 240 || v == 224) ? v : 0;
+    }();
+    if (forced) return forced;
+    const int64_t mtiles = (M + 511) / 512;
+    int best = kBN;
+    int64_t best_cost = INT64_MAX;
+    for (int bn : {256, 240, 224}) {
+        const int64_t tiles = mtiles * ((N + bn - 1) / bn);
+        const int64_t cost = (tiles + slots - 1) / slots * bn;
+        if (cost < best_cost) { best_cost = cost; best = bn; }
+    }
+    return best;
 }
 
 // Splits of the reduction so that tiles x splits fills one wave of CTAs.
@@ -1374,7 +1433,8 @@ qlora_status launch_tc_gemm_nf4(TcGemmArgs& a, bool dx, cudaStream_t stream) {
     const qlora_nf4_weight* w = a.w;
     const int64_t N = w->N, K = w->K;
     const bool pair = use_pairs(a.p.M);
-    const uint32_t wrows = pair ? 128 : 256;          // forward: W rows one CTA loads codes (and LoRA B rows) for
+    a.p.bn = (pair && !dx) ? pair_tile_width(a.p.M, N) : kBN;
+    const uint32_t wrows = pair ? (uint32_t)a.p.bn / 2 : 256;   // forward: W rows one CTA loads codes (and LoRA B rows) for
     // segment 0: A (X or dY) and the packed codes
     if (!dx) {
         if (!make_tmap_2d(&a.tmA0, true, a.A0, K, a.p.M, K * 2, 64, bm, true)) return QLORA_ERR_CUDA;

@@ -22,6 +22,8 @@ struct TcGemmParams {
     int64_t ldo;
     int32_t out_f32;
     int32_t b1_wrap;        // 0, or R/64 when B1 is the undoubled B / A: LoRA step j reads its step j % b1_wrap
+    int32_t bn;             // forward on CTA pairs: output columns per pair tile (256, 240 or 224; each CTA
+                            // supplies bn / 2 of them); 256 everywhere else
     uint32_t* err;
     NF4Tables tb;
 };
