@@ -216,6 +216,23 @@ def test_decode_stream_k_layouts(M, N, K, r, y_f32):
     check_linear_full(W, X, A, B, dY, r, alpha=2.0 * r, y_dtype=dt, dx_dtype=dt)
 
 
+# dX with more than 256 tokens on CTA pairs (512-token x 256-column pair tiles): one tile short of
+# its tokens, column tails of 128 and 64 columns, tiles whose K-steps are almost all LoRA steps
+# (N = 64, 192), a long reduction, and fp32 output.  Two calls give the same bits.
+@pytest.mark.parametrize("M,N,K,r,dx_f32", [(512, 192, 8192, 16, False), (1024, 4096, 640, 64, True),
+                                            (300, 64, 4992, 8, False), (777, 1000, 1344, 16, True)])
+def test_dx_pair_layouts(M, N, K, r, dx_f32):
+    W, X, A, B, dY = si.custom_linear(N, K, M, r, seed=5 * M + N + K + r)
+    dt = torch.float32 if dx_f32 else torch.bfloat16
+    w = check_linear_full(W, X, A, B, dY, r, alpha=2.0 * r, dx_dtype=dt)
+    Xd, Ad, Bd, dYd = (t.to(DEV) for t in (X, A, B, dY))
+    _, U = q4.qlora_linear_fwd(w, Xd, Ad, Bd, r, 2.0 * r)
+    dX1, _, _ = q4.qlora_linear_bwd(w, Xd, dYd, Ad, Bd, r, 2.0 * r, U_saved=U, dx_dtype=dt)
+    dX2, _, _ = q4.qlora_linear_bwd(w, Xd, dYd, Ad, Bd, r, 2.0 * r, U_saved=U, dx_dtype=dt)
+    torch.cuda.synchronize()
+    assert torch.equal(dX1, dX2)
+
+
 def test_recompute_U_and_no_dX():
     W, X, A, B, dY = si.custom_linear(128, 256, 24, 8, seed=77)
     w = quantize_on_gpu(W)
