@@ -39,7 +39,8 @@ AT_MAX_CLOCK = 0.97               # median SM clock at or above this share of th
 L2_FLUSH_BYTES = 256 << 20
 PACKED_BYTES_PER_WEIGHT = 0.5 + 1 / 64 + 4 / (64 * 256)     # codes + E4M3 constants + c2
 ALU_OPS_PER_WEIGHT = 2.5        # exact bf16 table expansion: 19 permute/logic ops per 8 weights + 8 per 64-weight table
-ALU_OPS_PER_CLK_SM = 62.0       # byte-permute / logic issue rate per SM, measured
+ALU_OPS_PER_CLK_SM = 64.0       # ALU pipe: 2 warp-instructions per clock per SM (ncu's peak_sustained for
+                                # sm__inst_executed_pipe_alu), 32 lanes each
 
 
 def parse_args():
@@ -379,12 +380,12 @@ def decode_sweep(device, peaks):
     props = torch.cuda.get_device_properties(device)
     l2 = props.L2_cache_size
     # ALU roofline of an exact bf16 dequant (every weight through a per-block 16-entry table):
-    # >= 2.5 byte-permute/logic ops per weight on a pipe that issues 62 per clock per SM
+    # >= 2.5 byte-permute/logic ops per weight on a pipe that issues 64 per clock per SM
     alu_gbs = (ALU_OPS_PER_CLK_SM * props.multi_processor_count * peaks.get("sm_max_mhz", 1965.0) * 1e6
                / ALU_OPS_PER_WEIGHT * PACKED_BYTES_PER_WEIGHT / 1e9)
     out = {"alu_roofline_GB/s": round(alu_gbs, 1),
-           "alu_roofline_basis": f"{ALU_OPS_PER_WEIGHT} ALU ops/weight, {ALU_OPS_PER_CLK_SM} ops/clk/SM (measured "
-                                 "pipe probe), SMs x max SM clock"}
+           "alu_roofline_basis": f"{ALU_OPS_PER_WEIGHT} ALU ops/weight, {ALU_OPS_PER_CLK_SM} ops/clk/SM (ncu: "
+                                 "sm__inst_executed_pipe_alu peak_sustained 2 warp-instr/clk/SM), SMs x max SM clock"}
     for i, (N, K) in enumerate(wl.linears):
         W = si.weight(wl, i).to(device)
         A, B = (t.to(device) for t in si.lora(wl, i))
