@@ -11,9 +11,12 @@
 //                        absmax c1 per block, and the fp64 sum of each
 //                        warp's 16 c1 values over a fixed pairwise tree.
 //   tree_sum_pass        fp64 pairwise-tree sums of 1024 partials per CTA,
-//                        repeated until one value is left.
-//   dq_blocks            per group of 256 blocks: mu from the tree sum,
-//                        d = c1 - mu, c2 = max|d|, E4M3 code of d / c2.
+//                        repeated while more than 1024 partials are left
+//                        (once from 2^20 to 2^30 weights, none below).
+//   dq_blocks            the last tree level (at most 1024 partials) in
+//                        each CTA, then per group of 256 blocks: mu from
+//                        the total, d = c1 - mu, c2 = max|d|, E4M3 code
+//                        of d / c2.
 // Every tree is over aligned power-of-two ranges with zero padding, so the
 // total equals a pairwise tree over all c1 padded to a power of two.
 #include <algorithm>
@@ -209,14 +212,32 @@ tree_sum_pass(const double* __restrict__ in, int64_t n, double* __restrict__ out
 // shuffles), x2 = fp32(d / c2) correctly rounded (Markstein as above for c2 in
 // [2^-100, 2^100], IEEE division outside), then its E4M3 code.
 __global__ void __launch_bounds__(kDqThreads)
-dq_blocks(const float* __restrict__ c1, int64_t nb1, const double* __restrict__ total,
+dq_blocks(const float* __restrict__ c1, int64_t nb1, const double* __restrict__ level, int np,
           uint8_t* __restrict__ c1_codes, float* __restrict__ c2_out, float* __restrict__ mu_out) {
-    grid_dependency_wait();                                   // c1 and the tree sum are complete
+    grid_dependency_wait();                                   // c1 and the tree's partial sums are complete
     const int lane = threadIdx.x & 31;
+    // the last tree level, np <= 1024 partials, in warp 0 of every CTA: lane l sums partials
+    // 32l .. 32l+31 pairwise, then the 32 lane sums pairwise by xor shuffles -- the same tree as a
+    // tree_sum_pass over them (zero padding included)
+    __shared__ double total;
+    if (threadIdx.x < 32) {
+        double v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = 32 * lane + j < np ? level[32 * lane + j] : 0.0;
+#pragma unroll
+        for (int w = 1; w < 32; w <<= 1)
+#pragma unroll
+            for (int j = 0; j < 32; j += 2 * w) v[j] += v[j + w];
+        double s = v[0];
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+        if (lane == 0) total = s;
+    }
+    __syncthreads();
     const int64_t g = (int64_t)blockIdx.x * (kDqThreads / 32) + (threadIdx.x >> 5);   // group
     const int64_t nb2 = (nb1 + 255) / 256;
     if (g >= nb2) return;
-    const float mu = __double2float_rn(__ddiv_rn(*total, (double)nb1));
+    const float mu = __double2float_rn(__ddiv_rn(total, (double)nb1));
     const int64_t i0 = g * 256 + lane * 8;
     float d[8];
     if (i0 + 8 <= nb1) {
@@ -295,7 +316,7 @@ qlora_status launch_quantize(const void* W, int64_t N, int64_t K, const qlora_nf
         host_buckets(out->codebook));
     QLORA_CHECK_LAUNCH();
     if (out->c1) return QLORA_OK;                             // single-level quantization: done
-    while (p > 1) {
+    while (p > kTreeThreads) {   // dq_blocks sums the last level (at most kTreeThreads partials) itself
         const int64_t np = (p + kTreeThreads - 1) / kTreeThreads;
         double* next = reinterpret_cast<double*>(ws);
         ws += align_up((size_t)np * sizeof(double), 256);
@@ -307,7 +328,7 @@ qlora_status launch_quantize(const void* W, int64_t N, int64_t K, const qlora_nf
     }
     const int64_t nb2 = (nb1 + 255) / 256;
     (void)launch_dependent(dq_blocks, dim3((unsigned)((nb2 + kDqThreads / 32 - 1) / (kDqThreads / 32))),
-                           dim3(kDqThreads), 0, stream, (const float*)c1, nb1, (const double*)level,
+                           dim3(kDqThreads), 0, stream, (const float*)c1, nb1, (const double*)level, (int)p,
                            out->c1_codes, out->c2, out->mu);
     QLORA_CHECK_LAUNCH();
     return QLORA_OK;
