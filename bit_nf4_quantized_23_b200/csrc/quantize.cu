@@ -92,7 +92,7 @@ __global__ void __launch_bounds__(kQuantThreads, kCtasPerSm)
 nf4_quantize_blocks(const uint4* __restrict__ W, int64_t nb1, uint4* __restrict__ codes,
                     float* __restrict__ c1_out, double* __restrict__ warp_sums_out, int64_t n_chunks,
                     QuantBuckets qb) {
-    allow_dependents();                                       // the tree passes may be scheduled now
+    allow_dependents();                                       // the tree pass (or the DQ kernel) may be scheduled now
     __shared__ float2 table[kTableWords];
     for (int i = threadIdx.x; i < kTableWords; i += kQuantThreads) table[i] = qb.e[i >> 5];
     __syncthreads();
