@@ -93,7 +93,7 @@ inline int32_t rank_pad(int32_t r) { return (r + 63) / 64 * 64; }
 //   U2  bf16 [M,2R]       hi/lo split of s*U
 //   dU2 bf16 [M,2R]       hi/lo split of dU
 //   B2  bf16 [N,2R]       [B | B] (only when r % 8 != 0; otherwise the GEMM reads B itself)
-//   Bt  bf16 [R,N]        B^T, zero-padded
+//   Bt  bf16 [R,N]        B^T, zero-padded (the dU GEMM reads it only when r % 8 != 0)
 //   partial fp32          split-reduction partial sums of the LoRA GEMMs
 struct LinearWs {
     size_t u_off, du_off, u2_off, du2_off, b2_off, bt_off, part_off, total;
@@ -435,23 +435,30 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const void* X, const vo
         void* Bt = ws + lw.bt_off;
         float* dUf = reinterpret_cast<float*>(ws + lw.du_off);
         float* partial = reinterpret_cast<float*>(ws + lw.part_off);
-        {
+        // the dU GEMM reads B [N, r] itself as an MN-major operand when its rows are 16-byte strided
+        // (r % 8 == 0); otherwise from B^T, zero-padded to R rows
+        const bool b_direct = r % 8 == 0;
+        if (!b_direct) {
             TimerScope t(QLORA_TIMER_LORA, s);
             QLORA_TRY(launch_transpose_pad(B, N, r, R, Bt, s));
-            if (U_saved) QLORA_TRY(launch_split_hi_lo(U_saved, M, r, R, scale, U2, f16, s));
         }
-        if (!U_saved) QLORA_TRY(lora_U(X, A, M, K, r, R, scale, nullptr, U2, partial, f16, s));
         {   // dU = s dY B  ->  dU (fp32) and its hi/lo split
             TimerScope t(QLORA_TIMER_LORA, s);
             LoraGemmArgs g{};
-            g.mn_major = false; g.A = dY; g.lda = N; g.B = Bt; g.ldb = N; g.rows = M; g.red = N; g.R = R;
+            g.mn_major = false; g.A = dY; g.lda = N; g.rows = M; g.red = N; g.R = R;
+            if (b_direct) {
+                g.B = B; g.ldb = r; g.b_mn = true; g.b_cols = r;
+            } else {
+                g.B = Bt; g.ldb = N;
+            }
             g.partial = partial;
             g.f16 = f16;
             QLORA_TRY(launch_lora_gemm(g, s));
             QLORA_TRY(launch_reduce_rows(partial, lora_splits(M, (int)((N + 63) / 64), R, false), M, r, R, scale, dUf, scale,
                                          dU2, f16, s));
         }
-        // fork: the adapter gradients go to the side stream once dU (and U2) are written
+        // fork: the adapter gradients go to the side stream once dU is written; U2 (hi/lo of s U),
+        // which only the dB GEMM reads, is prepared there too
         // (the caller's stream may be the null stream, so the fork is flagged, not inferred from g)
         const bool forked = dX != nullptr;
         cudaStream_t g = forked ? side_stream() : s;
@@ -474,6 +481,14 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const void* X, const vo
             a.p.M = M; a.p.Nout = K; a.p.out = dX; a.p.ldo = K; a.p.out_f32 = (dx_dtype == QLORA_DTYPE_F32);
             TimerScope t(QLORA_TIMER_DX_MAIN, s);
             st = launch_tc_gemm_nf4(a, true, s);
+        }
+        if (st == QLORA_OK) {
+            if (U_saved) {
+                TimerScope t(QLORA_TIMER_LORA, g);
+                st = launch_split_hi_lo(U_saved, M, r, R, scale, U2, f16, g);
+            } else {
+                st = lora_U(X, A, M, K, r, R, scale, nullptr, U2, partial, f16, g);
+            }
         }
         if (st == QLORA_OK) st = lora_gradients_tc(X, dY, M, N, K, r, R, f16, dA, dB, U2, dU2, partial, g);
         if (forked) {   // join: the caller's stream resumes after the adapter gradients too

@@ -12,13 +12,15 @@
 // reduction, so the reduction is split over CTAs (deterministic: every split
 // writes its own fp32 partial tile, a reduce kernel adds them in fixed order).
 //
-// Two operand modes:
+// Three operand modes:
 //   K-major  A [rows, red] and B [R, red], both with the reduction contiguous
-//            (X with A, dY with B^T); one MMA per 16-wide step.
+//            (X with A); one MMA per 16-wide step.
 //   MN-major A from S [red, rows] (X or dY, rows contiguous) and B from the
 //            bf16 hi/lo split V2 [red, 2R] of dU or s*U; two MMAs per step
 //            (hi then lo) into the same fp32 accumulator, so the fp32 factor
 //            keeps ~16 significant bits.
+//   K-major A, MN-major B: A [rows, red] and B [red, r] itself (dY with B):
+//            one MMA per step; columns r .. R-1 of B read as zero.
 // Roles (192 threads): warp 0 lane 0 TMA, warp 1 TMEM owner + MMA issuer,
 // warps 2-5 epilogue (TMEM -> fp32 partial tile).  No TMA multicast.
 #include <cuda.h>
@@ -51,7 +53,9 @@ __host__ __device__ inline LoraLayout lora_layout(uint32_t stages, uint32_t b_st
     return l;
 }
 
-template <bool MN>
+enum : int { kModeK = 0, kModeMN = 1, kModeKA_MNB = 2 };
+
+template <int MODE>
 __global__ void __launch_bounds__(kThreads, 2)
 tc_lora_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, LoraGemmParams p) {
     grid_dependency_wait();                                   // operands written by the previous kernel
@@ -100,6 +104,7 @@ tc_lora_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
 
     if (warp == 0) {
         // TMA issuer: the whole warp runs the loop, one elected lane issues the copies
+        constexpr bool MN = MODE == kModeMN;
         const uint32_t b_bytes = MN ? (uint32_t)R * 256u : (uint32_t)R * 128u;
         int issued = 0;
         for (int i = 0; i < nk; ++i) {
@@ -112,9 +117,12 @@ tc_lora_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                 const int ks = k_begin + i;
                 const uint32_t a_dst = sA + s * kAStage, b_dst = sB + s * kBStage;
                 ptx::mbar_arrive_expect_tx(fb, kAStage + b_bytes);
-                if (!MN) {
+                if (MODE == kModeK) {
                     ptx::tma_load_2d(a_dst, &tmA, ks * 64, (int32_t)row0, fb);
                     ptx::tma_load_2d(b_dst, &tmB, ks * 64, 0, fb);
+                } else if (MODE == kModeKA_MNB) {
+                    ptx::tma_load_2d(a_dst, &tmA, ks * 64, (int32_t)row0, fb);
+                    for (int c = 0; c < R / 64; ++c) ptx::tma_load_2d(b_dst + c * 8192, &tmB, c * 64, ks * 64, fb);
                 } else {
                     ptx::tma_load_2d(a_dst, &tmA, (int32_t)row0, ks * 64, fb);
                     ptx::tma_load_2d(a_dst + 8192, &tmA, (int32_t)row0 + 64, ks * 64, fb);
@@ -133,7 +141,8 @@ tc_lora_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
         }
     } else if (warp == 1) {
         // MMA issuer: the whole warp runs the loop, one elected lane issues the MMAs and commits
-        const uint32_t idesc = ptx::idesc_set_f16(ptx::idesc_bf16_f32_ab(128, R, MN ? 1 : 0, MN ? 1 : 0), p.f16 != 0);
+        const uint32_t idesc = ptx::idesc_set_f16(
+            ptx::idesc_bf16_f32_ab(128, R, MODE == kModeMN ? 1 : 0, MODE != kModeK ? 1 : 0), p.f16 != 0);
         bool ok = true;
         for (int i = 0; i < nk && ok; ++i) {
             const int s = i % kStages;
@@ -146,9 +155,12 @@ tc_lora_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                     const uint32_t acc = (i | kk) != 0 ? 1u : 0u;
-                    if (!MN) {
+                    if (MODE == kModeK) {
                         ptx::mma_bf16_ss(tmem, ptx::smem_desc_sw128(a_base + kk * 32, 16, 1024),
                                          ptx::smem_desc_sw128(b_base + kk * 32, 16, 1024), idesc, acc);
+                    } else if (MODE == kModeKA_MNB) {   // B: R/64 MN-major 64-column images, 8 KiB apart
+                        ptx::mma_bf16_ss(tmem, ptx::smem_desc_sw128(a_base + kk * 32, 16, 1024),
+                                         ptx::smem_desc_sw128(b_base + kk * 2048, 8192, 1024), idesc, acc);
                     } else {
                         const uint64_t ad = ptx::smem_desc_sw128(a_base + kk * 2048, 8192, 1024);
                         ptx::mma_bf16_ss(tmem, ad, ptx::smem_desc_sw128(b_base + kk * 2048, 8192, 1024), idesc,
@@ -196,17 +208,19 @@ tc_lora_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
     }
 }
 
-template <bool MN>
+template <int MODE>
 qlora_status launch_lora(const CUtensorMap& tmA, const CUtensorMap& tmB, LoraGemmParams& p, int splits,
                          cudaStream_t stream) {
+    constexpr bool MN = MODE == kModeMN;
     static bool configured = false;
-    auto kern = tc_lora_gemm<MN>;
+    auto kern = tc_lora_gemm<MODE>;
     if (!configured) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaxSmem) != cudaSuccess)
             return QLORA_ERR_CUDA;
         configured = true;
     }
-    // B stage: K-major R rows x 128 B, or the hi and lo MN-major images (2 x R/64 chunks of 8 KiB).
+    // B stage: K-major R rows x 128 B or R/64 MN-major chunks of 8 KiB (the same bytes), or the hi
+    // and lo MN-major images (2 x R/64 chunks of 8 KiB).
     // Two CTAs per SM (one's epilogue overlaps the other's main loop) when three or more stages
     // fit in half of the shared memory, else one CTA with up to six stages.
     const uint32_t b_stage = MN ? (uint32_t)p.R * 256u : (uint32_t)p.R * 128u;
@@ -271,14 +285,18 @@ qlora_status launch_lora_gemm(const LoraGemmArgs& a, cudaStream_t stream) {
     if (!a.mn_major) {
         // A [rows, red] and B [R, red], reduction contiguous
         if (!make_tmap_2d(&tmA, true, a.A, a.red, a.rows, a.lda * 2, 64, 128, true)) return QLORA_ERR_CUDA;
+        if (a.b_mn) {   // B [red, b_cols] with its columns contiguous; columns past b_cols read as zero
+            if (!make_tmap_2d(&tmB, true, a.B, (uint64_t)a.b_cols, a.red, a.ldb * 2, 64, 64, true)) return QLORA_ERR_CUDA;
+            return launch_lora<kModeKA_MNB>(tmA, tmB, p, splits, stream);
+        }
         const uint64_t b_rows = a.b_rows > 0 ? (uint64_t)a.b_rows : (uint64_t)a.R;   // rows past it read as zero
         if (!make_tmap_2d(&tmB, true, a.B, a.red, b_rows, a.ldb * 2, 64, (uint32_t)a.R, true)) return QLORA_ERR_CUDA;
-        return launch_lora<false>(tmA, tmB, p, splits, stream);
+        return launch_lora<kModeK>(tmA, tmB, p, splits, stream);
     }
     // S [red, rows] with rows contiguous, V2 [red, 2R] (hi | lo)
     if (!make_tmap_2d(&tmA, true, a.A, a.rows, a.red, a.lda * 2, 64, 64, true)) return QLORA_ERR_CUDA;
     if (!make_tmap_2d(&tmB, true, a.B, 2 * (uint64_t)a.R, a.red, a.ldb * 2, 64, 64, true)) return QLORA_ERR_CUDA;
-    return launch_lora<true>(tmA, tmB, p, splits, stream);
+    return launch_lora<kModeMN>(tmA, tmB, p, splits, stream);
 }
 
 size_t lora_partial_bytes(int64_t rows, int64_t red, int R, bool mn_major) {

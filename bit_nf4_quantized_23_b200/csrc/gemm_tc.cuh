@@ -113,6 +113,9 @@ struct LoraGemmArgs {
     int64_t rows, red;
     int32_t R;
     int64_t b_rows;    // K-major B: rows present in memory (B rows past it, up to R, read as zero); 0: R
+    bool b_mn;         // with mn_major false: B is [red, b_cols] with its columns contiguous (ldb >= b_cols,
+                       // ldb * 2 a multiple of 16); columns b_cols .. R-1 read as zero
+    int64_t b_cols;
     float* partial;
     int32_t f16;       // operands in fp16 instead of bf16
 };
